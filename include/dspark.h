@@ -1,0 +1,207 @@
+/*
+ * dspark.h: C ABI of the fused DSpark draft-training loss for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  For draft logits laid out [B, N, K, V] (batch, sampled anchor
+ * blocks, block positions, vocabulary) and the frozen target's next-token
+ * distribution, the three position-weighted terms of the DSpark objective
+ * (Megatron-Bridge API doc, bridge.training.post_training.dspark.loss, module
+ * docstring and dspark_loss):
+ *   loss = sum_r w_r * (ce_alpha*CE_r + l1_alpha*L1_r + conf_alpha*BCE_r)
+ *   CE_r  = logsumexp(z_r) - z_r[target_id]
+ *   L1_r  = sum_j |softmax(z_r)_j - softmax(t_r)_j|    (raw L1, no 1/2)
+ *   BCE_r = binary cross-entropy of the confidence logit c_r against the detached
+ *           label clamp(1 - 0.5*L1_r, 0, 1)
+ *   w_r   = m_r * exp(-k/gamma), m = cumulative product of eval_mask along the block
+ *           (TorchSpec pull request #132, scope list) times block_keep
+ * plus the acceptance report (accept = 1 - 0.5*L1, tau = 1 + sum_k prod_{j<=k}
+ * accept_j per block; Megatron-Bridge API doc, _acceptance_report), the gradient of
+ * grad_scale*loss with respect to the base draft logits, and, when the optional heads
+ * are given, the low-rank Markov correction z = base + markov_w2 . markov_w1[prev_id]
+ * (zero row on invalid slots) and the linear confidence head c = proj . [h ; e] + b
+ * (NeMo RL design doc "DSpark Auxiliary Heads", Inputs and Outputs, Checkpoint
+ * Contract) with their weight gradients.
+ *
+ * Return contract (Megatron-Bridge API doc, module docstring, Return contract): the
+ * library returns the UNNORMALISED weighted numerator, the supervised-token count and
+ * [numerator, denominator] report pairs.  It never divides by a local denominator;
+ * the caller sums numerators and denominators over micro-batches and data-parallel
+ * ranks and divides once (that is the calculate_per_token_loss=True convention).
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless stated otherwise.  The caller owns every
+ *    buffer; the library allocates nothing and keeps no state between calls except
+ *    what it writes into the caller's workspace.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *    the call returns without synchronising.  dspark_check_status() synchronises.
+ *  - Errors the host can see (bad sizes, NULL buffers, misalignment, short workspace,
+ *    a teacher-dependent term without a teacher) are returned before anything is
+ *    enqueued.  Errors only the device can see (an id out of range, a bounded wait
+ *    that ran out) set a flag in the workspace; the offending row is skipped (it
+ *    contributes nothing and its dlogits row is zero) and dspark_check_status()
+ *    reports the flag.
+ *  - Row r = (b*N + n)*K + k.  Logit rows have a leading dimension `*_ld` in
+ *    elements; ld*sizeof(element) must be a multiple of 16 bytes, V*sizeof(element)
+ *    must be a multiple of 16 bytes, and row pointers must be 16-byte aligned.
+ *  - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef DSPARK_H
+#define DSPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSPARK_API __attribute__((visibility("default")))
+#else
+#define DSPARK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* dspark_stream_t;
+
+typedef enum {
+  DSPARK_OK = 0,
+  DSPARK_ERR_INVALID_ARG = 1,     /* a size, pointer or parameter is not acceptable   */
+  DSPARK_ERR_MISSING_TARGET = 2,  /* L1 or confidence term requested with no teacher
+                                     (the ValueError of dspark_loss in the API doc)    */
+  DSPARK_ERR_ID_OUT_OF_RANGE = 3, /* device: a target/prev id outside its vocabulary  */
+  DSPARK_ERR_ALIGNMENT = 4,       /* a pointer or row stride breaks the 16-byte rule   */
+  DSPARK_ERR_WORKSPACE = 5,       /* workspace NULL or smaller than required          */
+  DSPARK_ERR_UNSUPPORTED = 6,     /* a shape/dtype combination this build does not run */
+  DSPARK_ERR_DEVICE_TIMEOUT = 7,  /* device: a bounded wait gave up                   */
+  DSPARK_ERR_CUDA = 8             /* the CUDA runtime reported an error               */
+} dspark_status_t;
+
+typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype_t;
+
+/* Report pair order: report[2*i] = numerator, report[2*i + 1] = denominator. */
+enum {
+  DSPARK_REP_LOSS = 0,   /* [sum w*(a_ce CE + a_l1 L1 + a_c BCE), num_tokens]          */
+  DSPARK_REP_CE = 1,     /* [sum w*CE, num_tokens]                                      */
+  DSPARK_REP_L1 = 2,     /* [sum w*L1, num_tokens]  (raw L1)                            */
+  DSPARK_REP_CONF = 3,   /* [sum w*BCE, num_tokens]  (0 numerator without confidence)   */
+  DSPARK_REP_ACCEPT = 4, /* [sum m*accept, num_tokens]      "dspark accept rate"        */
+  DSPARK_REP_TAU = 5,    /* [sum keep*tau_block, sum keep]  "dspark tau"                */
+  DSPARK_REP_COUNT = 6
+};
+
+/*
+ * One micro-batch: DSparkForwardOutput of the Megatron-Bridge API doc plus the head
+ * inputs of the NeMo RL design doc.  Unused optional pointers are NULL.
+ */
+typedef struct {
+  int64_t B, N, K, V;          /* R = B*N*K rows of V logits                            */
+  int64_t logits_dtype;        /* dspark_dtype_t of draft, target and dlogits            */
+  const void* draft_logits;    /* [R, V] base draft logits, row stride draft_ld          */
+  int64_t draft_ld;
+  const void* target_logits;   /* [R, V] teacher logits (row stride target_ld) or NULL   */
+  int64_t target_ld;
+  const int64_t* target_ids;   /* [R] teacher-forced next token, in [0, V)               */
+  const uint8_t* eval_mask;    /* [R] nonzero = position enabled; cut to its prefix      */
+  const uint8_t* block_keep;   /* [B*N] kept-anchor mask, or NULL = all kept             */
+  const float* confidence_logits; /* [R] given confidence logits, or NULL                */
+  /* teacher from the target's final hidden states (used when target_logits is NULL) */
+  const void* target_hidden;   /* bf16 [R, target_hidden_size], already final-normed    */
+  const void* lm_head;         /* bf16 [V, target_hidden_size]                          */
+  int64_t target_hidden_size;
+  /* Markov head (all NULL / 0 when absent) */
+  const int64_t* prev_ids;     /* [R] previous token, in [0, target_vocab)              */
+  const uint8_t* valid;        /* [R] nonzero = valid slot (also used by the conf head) */
+  int64_t target_vocab;
+  const void* markov_w1;       /* bf16 [target_vocab, markov_rank]                      */
+  const void* markov_w2;       /* bf16 [V, markov_rank]                                 */
+  int64_t markov_rank;
+  /* confidence head (NULL when absent; exclusive with confidence_logits) */
+  const void* draft_hidden;    /* bf16 [R, hidden_size]                                 */
+  int64_t hidden_size;
+  const void* conf_w;          /* bf16 [hidden_size (+ markov_rank)]: proj.weight       */
+  const float* conf_b;         /* [1] proj.bias                                         */
+  int64_t conf_with_markov;    /* 1: proj input is [hidden ; markov embedding]          */
+} dspark_problem_t;
+
+typedef struct {
+  float ce_alpha;              /* 0.1 in the API doc's signature                        */
+  float l1_alpha;              /* 0.9                                                   */
+  float conf_alpha;            /* 1.0 (used only with a confidence source)              */
+  float gamma;                 /* 4.0                                                   */
+  int32_t gamma_enabled;       /* 0 = no positional decay (loss_decay_gamma=None)       */
+  int32_t invalid_row_mode;    /* 0: invalid Markov slot -> all-zero corrected row;
+                                  1: invalid slot keeps its base row (bias removed)     */
+} dspark_params_t;
+
+/* Forward outputs.  Scalars are device buffers; per-row outputs are optional. */
+typedef struct {
+  float* loss_num;             /* [1] unnormalised weighted numerator                   */
+  int64_t* num_tokens;         /* [1] supervised-token count (exact)                    */
+  float* report;               /* [2*DSPARK_REP_COUNT] pairs, or NULL                   */
+  float* ce_rows;              /* [R] CE per row (0 where unsupervised), or NULL        */
+  float* l1_rows;              /* [R] raw L1 per row, or NULL                           */
+  float* accept_rows;          /* [R] m*accept per row, or NULL                         */
+  float* conf_rows;            /* [R] confidence logit used per row, or NULL            */
+} dspark_fwd_out_t;
+
+/* Backward outputs.  dlogits is written for EVERY row (zeros where unsupervised). */
+typedef struct {
+  const float* grad_scale;     /* device scalar g = d(objective)/d(loss_num); NULL = 1  */
+  void* dlogits;               /* [R, V] dL/d(base draft logits), logits dtype          */
+  int64_t dlogits_ld;
+  float* dconf;                /* [R] dL/dc, or NULL                                    */
+  float* dW1;                  /* fp32 [target_vocab, rank]: ALWAYS accumulated (+=)    */
+  float* dW2;                  /* fp32 [V, rank]                                        */
+  float* dconf_w;              /* fp32 [hidden_size (+ rank)]                           */
+  float* dconf_b;              /* fp32 [1]                                              */
+  void* dhidden;               /* bf16 [R, hidden_size], written for every row, or NULL */
+  int64_t accumulate;          /* 1: dW2, dconf_w, dconf_b += ; 0: overwritten          */
+} dspark_grads_t;
+
+/* Bytes of device workspace dspark_loss_fwd / dspark_loss_bwd need for `prob`
+ * (0 on an invalid problem).  Independent of the pointers' values. */
+DSPARK_API size_t dspark_workspace_size(const dspark_problem_t* prob);
+
+/*
+ * Forward, and with `grads` != NULL the fused backward in the same sweep (the
+ * gradient scale g must then be known before the call, e.g. 1 under per-token
+ * loss).  Writes every field of `out` that is non-NULL; leaves in `ws` the per-row
+ * statistics dspark_loss_bwd recomputes from.  `ws` must hold
+ * dspark_workspace_size(prob) bytes, 256-byte aligned.
+ */
+DSPARK_API dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_params_t* params,
+                                const dspark_fwd_out_t* out, const dspark_grads_t* grads,
+                                void* ws, size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * Backward alone, after a dspark_loss_fwd(..., grads = NULL) on the same problem,
+ * params and workspace: one more pass over the logits, recomputing the probabilities
+ * from the per-row statistics saved in `ws`.
+ */
+DSPARK_API dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_params_t* params,
+                                const dspark_grads_t* grads, const void* ws, size_t ws_bytes,
+                                dspark_stream_t stream);
+
+/*
+ * Acceptance report alone (Megatron-Bridge API doc, _acceptance_report) from per-row
+ * raw L1 values: accept_r = clamp(1 - 0.5*l1_r, 0, 1) on supervised rows (m from
+ * eval_mask and block_keep as above), tau_block = 1 + sum_k prod_{j<=k} m_j*accept_j.
+ * Writes accept_pair[2] = [sum m*accept, sum m], tau_pair[2] = [sum keep*tau, sum keep]
+ * and, if non-NULL, accept_rows[R] = m*accept.
+ */
+DSPARK_API dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
+                                  const uint8_t* eval_mask, const uint8_t* block_keep,
+                                  float* accept_pair, float* tau_pair, float* accept_rows,
+                                  dspark_stream_t stream);
+
+/* Synchronises `stream` and returns the first device-side error recorded in `ws`
+ * by the last call that used it (DSPARK_OK if none). */
+DSPARK_API dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream);
+
+/* Static English text for a status code. */
+DSPARK_API const char* dspark_status_string(dspark_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSPARK_H */

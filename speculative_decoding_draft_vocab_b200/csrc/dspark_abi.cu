@@ -1,0 +1,223 @@
+// The C ABI of include/dspark.h: host-side validation, workspace carving and the
+// launch sequence of each entry point.  No allocation, no synchronisation (except
+// dspark_check_status, whose job it is).
+#include <cstdint>
+#include <cstring>
+
+#include "internal.cuh"
+
+using namespace dspark;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t elem_size(int64_t dtype) { return dtype == DSPARK_BF16 ? 2 : 4; }
+
+// Which optional parts a problem uses.
+struct Shape {
+  int64_t R;
+  bool has_target_rows;  // teacher given as logits
+  bool has_lm_head;      // teacher from hidden states
+  bool has_teacher;
+  bool has_markov;
+  bool has_conf_given;
+  bool has_conf_head;
+};
+
+dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* prm, Shape* sh) {
+  if (p == nullptr) return DSPARK_ERR_INVALID_ARG;
+  if (p->B <= 0 || p->N <= 0 || p->K <= 0 || p->V <= 0) return DSPARK_ERR_INVALID_ARG;
+  if (p->logits_dtype != DSPARK_F32 && p->logits_dtype != DSPARK_BF16) return DSPARK_ERR_INVALID_ARG;
+  if (p->B * p->N * p->K > (int64_t(1) << 31) - 1) return DSPARK_ERR_UNSUPPORTED;
+  if (p->V > (int64_t(1) << 30)) return DSPARK_ERR_UNSUPPORTED;
+  if (!p->draft_logits || !p->target_ids || !p->eval_mask) return DSPARK_ERR_INVALID_ARG;
+  const size_t es = elem_size(p->logits_dtype);
+  if (p->draft_ld < p->V) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(p->draft_logits) || (p->draft_ld * es) % 16 || (p->V * es) % 16)
+    return DSPARK_ERR_ALIGNMENT;
+  Shape s{};
+  s.R = p->B * p->N * p->K;
+  s.has_target_rows = p->target_logits != nullptr;
+  s.has_lm_head = p->lm_head != nullptr || p->target_hidden != nullptr;
+  s.has_teacher = s.has_target_rows || s.has_lm_head;
+  s.has_markov = p->markov_w2 != nullptr || p->markov_w1 != nullptr || p->prev_ids != nullptr;
+  s.has_conf_given = p->confidence_logits != nullptr;
+  s.has_conf_head = p->conf_w != nullptr || p->draft_hidden != nullptr;
+  if (s.has_target_rows) {
+    if (p->target_ld < p->V) return DSPARK_ERR_INVALID_ARG;
+    if (!aligned16(p->target_logits) || (p->target_ld * es) % 16) return DSPARK_ERR_ALIGNMENT;
+  }
+  if (s.has_target_rows && s.has_lm_head) return DSPARK_ERR_INVALID_ARG;
+  if (s.has_conf_given && s.has_conf_head) return DSPARK_ERR_INVALID_ARG;
+  if (prm != nullptr) {
+    if (!s.has_teacher && (prm->l1_alpha != 0.f || s.has_conf_given || s.has_conf_head))
+      return DSPARK_ERR_MISSING_TARGET;
+    if (prm->gamma_enabled && !(prm->gamma > 0.f)) return DSPARK_ERR_INVALID_ARG;
+    if (prm->invalid_row_mode != 0 && prm->invalid_row_mode != 1) return DSPARK_ERR_INVALID_ARG;
+  }
+  // The Markov head, the confidence head and the teacher-from-hidden path run in
+  // their own kernels; this build accepts them only once those are present.
+  if (s.has_markov || s.has_conf_head || s.has_lm_head) return DSPARK_ERR_UNSUPPORTED;
+  if (!sweep_supported(int(p->logits_dtype), p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
+  *sh = s;
+  return DSPARK_OK;
+}
+
+inline dspark_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+
+dspark_status_t check_ws(const dspark_problem_t* p, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return DSPARK_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DSPARK_ERR_ALIGNMENT;
+  if (ws_bytes < ws_offsets(p->B * p->N * p->K).bytes) return DSPARK_ERR_WORKSPACE;
+  return DSPARK_OK;
+}
+
+dspark_status_t check_grads(const dspark_problem_t* p, const dspark_grads_t* g) {
+  if (g == nullptr || g->dlogits == nullptr) return DSPARK_ERR_INVALID_ARG;
+  const size_t es = elem_size(p->logits_dtype);
+  if (g->dlogits_ld < p->V) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(g->dlogits) || (g->dlogits_ld * es) % 16) return DSPARK_ERR_ALIGNMENT;
+  return DSPARK_OK;
+}
+
+SweepArgs sweep_args(const dspark_problem_t* p, const dspark_params_t* prm, const WsView& ws,
+                     const dspark_grads_t* g) {
+  SweepArgs a{};
+  a.draft = p->draft_logits;
+  a.ld_d = p->draft_ld;
+  a.target = p->target_logits;
+  a.ld_t = p->target_ld;
+  a.dlogits = g ? g->dlogits : nullptr;
+  a.ld_g = g ? g->dlogits_ld : 0;
+  a.tids = p->target_ids;
+  a.grad_scale = g ? g->grad_scale : nullptr;
+  a.ws = ws;
+  a.V = p->V;
+  a.ce_alpha = prm->ce_alpha;
+  a.l1_alpha = p->target_logits ? prm->l1_alpha : 0.f;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dspark_status_string(dspark_status_t s) {
+  switch (s) {
+    case DSPARK_OK: return "ok";
+    case DSPARK_ERR_INVALID_ARG: return "invalid argument";
+    case DSPARK_ERR_MISSING_TARGET: return "L1 or confidence term requested without target logits";
+    case DSPARK_ERR_ID_OUT_OF_RANGE: return "a target or previous-token id is outside its vocabulary";
+    case DSPARK_ERR_ALIGNMENT: return "pointer or row stride is not 16-byte aligned";
+    case DSPARK_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSPARK_ERR_UNSUPPORTED: return "shape or option not supported by this build";
+    case DSPARK_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+    case DSPARK_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+size_t dspark_workspace_size(const dspark_problem_t* prob) {
+  if (prob == nullptr || prob->B <= 0 || prob->N <= 0 || prob->K <= 0) return 0;
+  return ws_offsets(prob->B * prob->N * prob->K).bytes;
+}
+
+dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_params_t* params,
+                                const dspark_fwd_out_t* out, const dspark_grads_t* grads,
+                                void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  if (params == nullptr || out == nullptr) return DSPARK_ERR_INVALID_ARG;
+  Shape sh{};
+  dspark_status_t st = check_problem(prob, params, &sh);
+  if (st != DSPARK_OK) return st;
+  if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
+  if (grads && (st = check_grads(prob, grads)) != DSPARK_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsView v = ws_layout(ws, sh.R);
+
+  PrologueArgs pa{};
+  pa.B = prob->B; pa.N = prob->N; pa.K = prob->K; pa.V = prob->V; pa.Vt = prob->target_vocab;
+  pa.eval_mask = prob->eval_mask;
+  pa.block_keep = prob->block_keep;
+  pa.target_ids = prob->target_ids;
+  pa.prev_ids = nullptr;
+  pa.valid = prob->valid;
+  pa.gamma = params->gamma;
+  pa.gamma_enabled = params->gamma_enabled;
+  pa.ws = v;
+  cudaError_t e = launch_prologue(pa, s);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  SweepArgs sa = sweep_args(prob, params, v, grads);
+  e = launch_sweep(int(prob->logits_dtype), sh.has_target_rows, sa, s);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  FinalizeArgs fa{};
+  fa.B = prob->B; fa.N = prob->N; fa.K = prob->K;
+  fa.block_keep = prob->block_keep;
+  fa.confidence_logits = prob->confidence_logits;
+  fa.has_conf = sh.has_conf_given || sh.has_conf_head;
+  fa.ce_alpha = params->ce_alpha;
+  fa.l1_alpha = params->l1_alpha;
+  fa.conf_alpha = params->conf_alpha;
+  fa.grad_scale = grads ? grads->grad_scale : nullptr;
+  fa.ws = v;
+  fa.loss_num = out->loss_num;
+  fa.num_tokens = out->num_tokens;
+  fa.report = out->report;
+  fa.ce_rows = out->ce_rows;
+  fa.l1_rows = out->l1_rows;
+  fa.accept_rows = out->accept_rows;
+  fa.conf_rows = out->conf_rows;
+  fa.dconf = grads ? grads->dconf : nullptr;
+  return cuda_status(launch_finalize(fa, s));
+}
+
+dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_params_t* params,
+                                const dspark_grads_t* grads, const void* ws, size_t ws_bytes,
+                                dspark_stream_t stream) {
+  if (params == nullptr) return DSPARK_ERR_INVALID_ARG;
+  Shape sh{};
+  dspark_status_t st = check_problem(prob, params, &sh);
+  if (st != DSPARK_OK) return st;
+  if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
+  if ((st = check_grads(prob, grads)) != DSPARK_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsView v = ws_layout(const_cast<void*>(ws), sh.R);
+  SweepArgs sa = sweep_args(prob, params, v, grads);
+  cudaError_t e = launch_bwd_stream(int(prob->logits_dtype), sh.has_target_rows, sa, sh.R, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (grads->dconf) {
+    if (!(sh.has_conf_given || sh.has_conf_head)) {
+      e = cudaMemsetAsync(grads->dconf, 0, sizeof(float) * sh.R, s);
+    } else {
+      e = launch_conf_grad(sh.R, prob->confidence_logits, params->conf_alpha, grads->grad_scale, v,
+                           grads->dconf, s);
+    }
+  }
+  return cuda_status(e);
+}
+
+dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
+                                  const uint8_t* eval_mask, const uint8_t* block_keep,
+                                  float* accept_pair, float* tau_pair, float* accept_rows,
+                                  dspark_stream_t stream) {
+  if (B <= 0 || N <= 0 || K <= 0) return DSPARK_ERR_INVALID_ARG;
+  if (!l1_rows || !eval_mask || !accept_pair || !tau_pair) return DSPARK_ERR_INVALID_ARG;
+  return cuda_status(launch_acceptance(B, N, K, l1_rows, eval_mask, block_keep, accept_pair,
+                                       tau_pair, accept_rows, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream) {
+  if (ws == nullptr) return DSPARK_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  uint32_t flags = 0;
+  if (cudaMemcpy(&flags, ws, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  if (flags & kFlagIdOutOfRange) return DSPARK_ERR_ID_OUT_OF_RANGE;
+  if (flags & kFlagTimeout) return DSPARK_ERR_DEVICE_TIMEOUT;
+  return DSPARK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Mask prologue: the contiguous-prefix supervision mask, the per-position loss
+// weights, the supervised-token count and the two ordered row lists the sweep
+// walks (supervised rows, then rows whose dlogits are only zero-filled).
+//
+// m[b,n,k] = prod_{j<=k} eval[b,n,j] * keep[b,n]  (TorchSpec pull request #132,
+// scope list: cumprod prefix mask; Megatron-Bridge API doc, DSparkForwardOutput)
+// w[b,n,k] = m * exp(-k/gamma)                     (Megatron-Bridge API doc,
+// _loss_weight_mask; k is the 0-based block position)
+// Integer work is exact; one CTA does it all (R is a few thousand rows).
+#include "internal.cuh"
+
+namespace dspark {
+
+constexpr int kPrologueThreads = 1024;
+
+__global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const PrologueArgs a) {
+  const int tid = threadIdx.x;
+  const int64_t nblk = a.B * a.N;
+  const int64_t R = nblk * a.K;
+  WsHeader* hdr = a.ws.hdr;
+  if (tid == 0) {
+    hdr->status = 0;
+    hdr->done = 0;
+  }
+  __syncthreads();
+
+  // ---- masks and weights, one thread per block of K positions
+  uint32_t flags = 0;
+  for (int64_t blk = tid; blk < nblk; blk += kPrologueThreads) {
+    bool run = a.block_keep == nullptr || a.block_keep[blk] != 0;
+    for (int64_t k = 0; k < a.K; ++k) {
+      const int64_t r = blk * a.K + k;
+      run = run && a.eval_mask[r] != 0;
+      bool mm = run;
+      if (mm) {
+        const int64_t t = a.target_ids[r];
+        if (t < 0 || t >= a.V) { flags |= kFlagIdOutOfRange; mm = false; }
+        if (a.prev_ids != nullptr && a.valid[r] != 0) {
+          const int64_t pv = a.prev_ids[r];
+          if (pv < 0 || pv >= a.Vt) { flags |= kFlagIdOutOfRange; mm = false; }
+        }
+      }
+      a.ws.m[r] = mm ? 1 : 0;
+      a.ws.w[r] = !mm ? 0.f : (a.gamma_enabled ? expf(-float(k) / a.gamma) : 1.f);
+    }
+  }
+  if (flags) atomicOr(&hdr->status, flags);
+  __syncthreads();
+
+  // ---- ordered compaction of the two row lists
+  __shared__ int warp_sup[kPrologueThreads / 32];
+  __shared__ int base_sup;
+  const int lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) base_sup = 0;
+  __syncthreads();
+  for (int64_t r0 = 0; r0 < R; r0 += kPrologueThreads) {
+    const int64_t r = r0 + tid;
+    const bool s = r < R && a.ws.m[r] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, s);
+    if (lane == 0) warp_sup[warp] = __popc(bal);
+    __syncthreads();
+    int before = base_sup;
+    for (int i = 0; i < warp; ++i) before += warp_sup[i];
+    before += __popc(bal & ((1u << lane) - 1u));
+    if (r < R) {
+      if (s) a.ws.sup_list[before] = int32_t(r);
+      else a.ws.zero_list[r - before] = int32_t(r);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int tot = 0;
+      for (int i = 0; i < kPrologueThreads / 32; ++i) tot += warp_sup[i];
+      base_sup += tot;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    hdr->n_sup = base_sup;
+    hdr->n_zero = int32_t(R - base_sup);
+    hdr->num_tokens = base_sup;
+  }
+}
+
+cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s) {
+  prologue_kernel<<<1, kPrologueThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace dspark

@@ -1,0 +1,529 @@
+// Row sweep: fused DSpark forward + backward over full-vocabulary rows.
+//
+// One thread-block cluster owns one supervised row at a time.  Each CTA of the
+// cluster owns a contiguous 16-byte-aligned segment of the vocabulary; the segment
+// of the next rows is streamed into shared memory by 1-D bulk async copies (TMA,
+// no multicast) while the current row is processed from registers, so every logit
+// is read from HBM exactly once.  The exponentials are taken once per element and
+// kept in registers for the rest of the row; the three row-wide reductions
+// (logsumexp; L1 and S; nothing else) combine per-CTA partials through distributed
+// shared memory, in the same fixed order in every CTA, so every CTA sees bitwise
+// the same row scalars.  dlogits are written in the same sweep.
+//
+// Per row r with corrected draft z and teacher t (Megatron-Bridge API doc,
+// bridge.training.post_training.dspark.loss, _chunk_terms / dspark_loss):
+//   lse_d = log sum exp z,  lse_t = log sum exp t,  CE = lse_d - z[id]
+//   p = exp(z - lse_d), q = exp(t - lse_t), L1 = sum |p - q| (raw), S = sum p*sign(p-q)
+//   dL/dz_j = g*w*[ce_alpha*(p_j - [j = id]) + l1_alpha*p_j*(sign(p_j - q_j) - S)]
+// Everything is computed in base 2: offsets are kept as x*log2(e).
+#include <cuda_bf16.h>
+#include <algorithm>
+#include <mutex>
+
+#include "internal.cuh"
+#include "ptx.cuh"
+
+namespace dspark {
+
+template <typename T> struct VecTraits;
+template <> struct VecTraits<float> { static constexpr int EPV = 4; };
+template <> struct VecTraits<__nv_bfloat16> { static constexpr int EPV = 8; };
+
+template <typename T> __device__ __forceinline__ void unpack16(const uint4 q, float* o);
+template <> __device__ __forceinline__ void unpack16<float>(const uint4 q, float* o) {
+  o[0] = __uint_as_float(q.x); o[1] = __uint_as_float(q.y);
+  o[2] = __uint_as_float(q.z); o[3] = __uint_as_float(q.w);
+}
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 q, float* o) {
+  o[0] = bf16lo(q.x); o[1] = bf16hi(q.x); o[2] = bf16lo(q.y); o[3] = bf16hi(q.y);
+  o[4] = bf16lo(q.z); o[5] = bf16hi(q.z); o[6] = bf16lo(q.w); o[7] = bf16hi(q.w);
+}
+
+template <typename T> __device__ __forceinline__ uint4 pack16(const float* o);
+template <> __device__ __forceinline__ uint4 pack16<float>(const float* o) {
+  return make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                    __float_as_uint(o[3]));
+}
+template <> __device__ __forceinline__ uint4 pack16<__nv_bfloat16>(const float* o) {
+  return make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                    pack_bf16(o[6], o[7]));
+}
+
+template <typename T> __device__ __forceinline__ float load_elem(const uint8_t* p);
+template <> __device__ __forceinline__ float load_elem<float>(const uint8_t* p) {
+  return *reinterpret_cast<const float*>(p);
+}
+template <> __device__ __forceinline__ float load_elem<__nv_bfloat16>(const uint8_t* p) {
+  return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t*>(p)) << 16);
+}
+
+// (max, sum 2^(x - max)) in base-2 units; max = -inf marks an empty partial.
+struct MS {
+  float m, s;
+};
+__device__ __forceinline__ MS ms_combine(MS a, MS b) {
+  const float m = fmaxf(a.m, b.m);
+  if (m == -INFINITY) return MS{m, 0.f};
+  const float sa = (a.m == -INFINITY) ? 0.f : a.s * ex2(a.m - m);
+  const float sb = (b.m == -INFINITY) ? 0.f : b.s * ex2(b.m - m);
+  return MS{m, sa + sb};
+}
+__device__ __forceinline__ MS ms_shfl(MS v, int off) {
+  return MS{__shfl_xor_sync(0xffffffffu, v.m, off), __shfl_xor_sync(0xffffffffu, v.s, off)};
+}
+
+struct Ctrl {
+  uint64_t mbar[2];
+  float4 slotA;     // this CTA's (max, sum) partials of draft and teacher
+  float4 slotB;     // this CTA's (L1, S) partials
+  float4 red[32];   // per-warp partials
+  float4 bcast[2];  // row scalars broadcast to the CTA
+  float ztid;       // raw draft logit at the target id (owner CTA only)
+};
+
+template <typename T, int CL, int NT, int NV, bool HAS_T>
+__global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
+  constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int NE = NV * EPV;
+  constexpr int NW = NT / 32;
+  constexpr int NTENS = HAS_T ? 2 : 1;
+  static_assert(NW <= 32, "one warp combines the per-warp partials");
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t cid = cluster_id_x();
+  const uint32_t G = nclusters_x();
+  const uint32_t seg_bytes = uint32_t(a.seg_vec) * 16u;
+  const int nbuf = a.nbuf;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + size_t(nbuf) * NTENS * seg_bytes);
+  WsHeader* hdr = a.ws.hdr;
+
+  const int v0 = int(rank) * a.seg_vec;
+  const int nvec = max(0, min(a.seg_vec, a.vvec - v0));
+  const uint32_t bytes = uint32_t(nvec) * 16u;
+  const int n_sup = hdr->n_sup;
+  const int n_zero = hdr->n_zero;
+  const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
+  const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
+  const uint8_t* target = static_cast<const uint8_t*>(a.target);
+  const bool bwd = a.dlogits != nullptr;
+  const float g = a.grad_scale ? *a.grad_scale : 1.f;
+
+  auto buf = [&](int b, int tsel) -> uint8_t* {
+    return smem + (size_t(b) * NTENS + tsel) * seg_bytes;
+  };
+  const uint32_t bar0 = smem_u32(&ctrl->mbar[0]);
+  const uint32_t bar1 = smem_u32(&ctrl->mbar[1]);
+  uint64_t policy = 0;
+
+  auto issue = [&](int j) {  // thread 0: stream row j's segment into buffer j % nbuf
+    const int b = j % nbuf;
+    const uint32_t bar = b ? bar1 : bar0;
+    const int64_t row = a.ws.sup_list[cid + size_t(j) * G];
+    mbar_arrive_expect_tx(bar, NTENS * bytes);
+    if (bytes) {
+      bulk_g2s(smem_u32(buf(b, 0)), draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * sizeof(T),
+               bytes, bar, policy);
+      if constexpr (HAS_T)
+        bulk_g2s(smem_u32(buf(b, 1)),
+                 target + (size_t(row) * a.ld_t + size_t(v0) * EPV) * sizeof(T), bytes, bar,
+                 policy);
+    }
+  };
+
+  if (tid == 0) {
+    policy = l2_policy_evict_first();
+    mbar_init(bar0, 1);
+    mbar_init(bar1, 1);
+    fence_mbar_init();
+    for (int j = 0; j < min(nbuf, my_n); ++j) issue(j);
+  }
+  __syncthreads();
+
+  for (int j = 0; j < my_n; ++j) {
+    const int b = j % nbuf;
+    const uint32_t phase = uint32_t(j / nbuf) & 1u;
+    const int64_t row = a.ws.sup_list[cid + size_t(j) * G];
+    const int64_t tok = a.tids[row];
+    const int tv = int(tok / EPV) - v0;  // target id's vector inside this segment
+    const int te = int(tok % EPV);
+
+    if (!mbar_wait_bounded(b ? bar1 : bar0, phase)) {
+      if (tid == 0) atomicOr(&hdr->status, kFlagTimeout);
+    }
+
+    // ---- segment -> registers
+    float xz[NE];
+    float xt[HAS_T ? NE : 1];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int v = tid + i * NT;
+      if (v < nvec) {
+        unpack16<T>(*reinterpret_cast<const uint4*>(buf(b, 0) + size_t(v) * 16), &xz[i * EPV]);
+        if constexpr (HAS_T)
+          unpack16<T>(*reinterpret_cast<const uint4*>(buf(b, 1) + size_t(v) * 16), &xt[i * EPV]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) {
+          xz[i * EPV + e] = -INFINITY;
+          if constexpr (HAS_T) xt[i * EPV + e] = -INFINITY;
+        }
+      }
+    }
+    if (tid == 0 && tv >= 0 && tv < nvec)
+      ctrl->ztid = load_elem<T>(buf(b, 0) + size_t(tv) * 16 + size_t(te) * sizeof(T));
+    __syncthreads();  // the buffer is free again
+    if (tid == 0 && j + nbuf < my_n) issue(j + nbuf);
+
+    // ---- pass 1: per-thread max, exponentials kept in registers, sums
+    float mz = -INFINITY, mt = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+      mz = fmaxf(mz, xz[e]);
+      if constexpr (HAS_T) mt = fmaxf(mt, xt[e]);
+    }
+    const float oz = (mz == -INFINITY) ? 0.f : mz * kLog2e;
+    const float ot = (mt == -INFINITY) ? 0.f : mt * kLog2e;
+    float sz = 0.f, st = 0.f;
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+      xz[e] = ex2(fmaf(xz[e], kLog2e, -oz));
+      sz += xz[e];
+      if constexpr (HAS_T) {
+        xt[e] = ex2(fmaf(xt[e], kLog2e, -ot));
+        st += xt[e];
+      }
+    }
+    MS pz{mz == -INFINITY ? -INFINITY : oz, sz};
+    MS pt{mt == -INFINITY ? -INFINITY : ot, st};
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      pz = ms_combine(pz, ms_shfl(pz, off));
+      if constexpr (HAS_T) pt = ms_combine(pt, ms_shfl(pt, off));
+    }
+    if (lane == 0) ctrl->red[warp] = make_float4(pz.m, pz.s, pt.m, pt.s);
+    __syncthreads();
+    if (warp == 0) {
+      const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      MS qz{r4.x, r4.y}, qt{r4.z, r4.w};
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        qz = ms_combine(qz, ms_shfl(qz, off));
+        if constexpr (HAS_T) qt = ms_combine(qt, ms_shfl(qt, off));
+      }
+      if (lane == 0) ctrl->slotA = make_float4(qz.m, qz.s, qt.m, qt.s);
+    }
+    cluster_sync();
+    if (warp == 0) {
+      float4 r4 = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      if (lane < CL) r4 = dsmem_ld_f4(dsmem_map(smem_u32(&ctrl->slotA), uint32_t(lane)));
+      MS qz{r4.x, r4.y}, qt{r4.z, r4.w};
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        qz = ms_combine(qz, ms_shfl(qz, off));
+        if constexpr (HAS_T) qt = ms_combine(qt, ms_shfl(qt, off));
+      }
+      if (lane == 0)
+        ctrl->bcast[0] = make_float4(qz.m + log2f(qz.s), HAS_T ? qt.m + log2f(qt.s) : 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    const float lz2 = ctrl->bcast[0].x;  // lse_d in base-2 units
+    const float lt2 = ctrl->bcast[0].y;
+    const float az = (mz == -INFINITY) ? 0.f : ex2(oz - lz2);  // p = e * az
+    const float at = (!HAS_T || mt == -INFINITY) ? 0.f : ex2(ot - lt2);
+
+    // ---- pass 2: L1 and S
+    float L1 = 0.f, S = 0.f;
+    if constexpr (HAS_T) {
+      float l1p = 0.f, sp = 0.f;
+#pragma unroll
+      for (int e = 0; e < NE; ++e) {
+        const float p = xz[e] * az, q = xt[e] * at, d = p - q;
+        l1p += fabsf(d);
+        sp += d > 0.f ? p : (d < 0.f ? -p : 0.f);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        l1p += __shfl_xor_sync(0xffffffffu, l1p, off);
+        sp += __shfl_xor_sync(0xffffffffu, sp, off);
+      }
+      if (lane == 0) ctrl->red[warp] = make_float4(l1p, sp, 0.f, 0.f);
+      __syncthreads();
+      if (warp == 0) {
+        const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+        float x = r4.x, y = r4.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          x += __shfl_xor_sync(0xffffffffu, x, off);
+          y += __shfl_xor_sync(0xffffffffu, y, off);
+        }
+        if (lane == 0) ctrl->slotB = make_float4(x, y, 0.f, 0.f);
+      }
+      cluster_sync();
+      if (warp == 0) {
+        float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane < CL) r4 = dsmem_ld_f4(dsmem_map(smem_u32(&ctrl->slotB), uint32_t(lane)));
+        float x = r4.x, y = r4.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          x += __shfl_xor_sync(0xffffffffu, x, off);
+          y += __shfl_xor_sync(0xffffffffu, y, off);
+        }
+        if (lane == 0) ctrl->bcast[1] = make_float4(x, y, 0.f, 0.f);
+      }
+      __syncthreads();
+      L1 = ctrl->bcast[1].x;
+      S = ctrl->bcast[1].y;
+    }
+
+    // ---- per-row statistics
+    float* st_row = a.ws.stats + size_t(row) * kStride;
+    if (tid == 0) {
+      if (rank == 0) {
+        st_row[kStLseD] = lz2 * kLn2;
+        st_row[kStLseT] = lt2 * kLn2;
+        st_row[kStL1] = L1;
+        st_row[kStS] = S;
+      }
+      if (tv >= 0 && tv < nvec) {
+        st_row[kStCE] = lz2 * kLn2 - ctrl->ztid;
+        st_row[kStZT] = ctrl->ztid;
+      }
+    }
+
+    // ---- pass 3: dlogits
+    if (bwd) {
+      const float gw = g * a.ws.w[row];
+      const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
+      const float kpos = cce + cl1 * (1.f - S);
+      const float kneg = cce + cl1 * (-1.f - S);
+      const float kzero = cce - cl1 * S;
+      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int v = tid + i * NT;
+        if (v < nvec) {
+          float o[EPV];
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) {
+            const float p = xz[i * EPV + e] * az;
+            if constexpr (HAS_T) {
+              const float d = p - xt[i * EPV + e] * at;
+              o[e] = p * (d > 0.f ? kpos : (d < 0.f ? kneg : kzero));
+            } else {
+              o[e] = p * cce;
+            }
+          }
+          if (v == tv) {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e)
+              if (e == te) o[e] -= cce;
+          }
+          *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<T>(o);
+        }
+      }
+    }
+  }
+
+  // ---- rows outside the supervision mask: dlogits = 0
+  if (bwd && n_zero > 0) {
+    const int first = ((int(cid) - n_sup) % int(G) + int(G)) % int(G);
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    for (int zi = first; zi < n_zero; zi += int(G)) {
+      const int64_t row = a.ws.zero_list[zi];
+      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
+      for (int v = tid; v < nvec; v += NT) *reinterpret_cast<uint4*>(out + size_t(v) * 16) = z4;
+    }
+  }
+  // no CTA leaves while a peer may still read its shared memory
+  cluster_sync();
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+struct LaunchCache {
+  std::mutex mu;
+  int dev = -1;
+  size_t smem = 0;
+  const void* fn = nullptr;
+  int clusters = 0;
+};
+
+template <typename T, int CL, int NT, int NV, bool HAS_T>
+cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
+  constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int NTENS = HAS_T ? 2 : 1;
+  SweepArgs a = a0;
+  a.vvec = int32_t(a.V / EPV);
+  a.seg_vec = (a.vvec + CL - 1) / CL;
+  const size_t per_buf = size_t(a.seg_vec) * 16 * NTENS;
+  const size_t ctrl = sizeof(Ctrl);
+  constexpr size_t kMaxSmem = 227 * 1024;
+  a.nbuf = (2 * per_buf + ctrl <= kMaxSmem) ? 2 : 1;
+  const size_t smem = a.nbuf * per_buf + ctrl;
+  if (smem > kMaxSmem) return cudaErrorInvalidValue;
+
+  auto kern = sweep_kernel<T, CL, NT, NV, HAS_T>;
+  static LaunchCache cache;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int clusters = 0;
+  {
+    std::lock_guard<std::mutex> lk(cache.mu);
+    if (cache.dev != dev || cache.smem != smem) {
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxSmem));
+      if (err != cudaSuccess) return err;
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(CL, 1, 1);
+      q.blockDim = dim3(NT, 1, 1);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = CL;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      q.attrs = at;
+      q.numAttrs = 1;
+      int n = 0;
+      err = cudaOccupancyMaxActiveClusters(&n, kern, &q);
+      if (err != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        int sms = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        n = sms / CL > 0 ? sms / CL : 1;
+      }
+      cache.dev = dev;
+      cache.smem = smem;
+      cache.clusters = n;
+    }
+    clusters = cache.clusters;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(clusters * CL), 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CL;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Capacity of a (CL, NT, NV) build = CL * NT * NV * elements-per-vector.
+struct Build {
+  int cl, nt, nv;
+};
+constexpr Build kBf16Builds[] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}};
+constexpr Build kF32Builds[] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 5}, {8, 512, 10}};
+
+int pick_build(int dtype, int64_t V) {
+  const Build* b = dtype == DSPARK_BF16 ? kBf16Builds : kF32Builds;
+  const int epv = dtype == DSPARK_BF16 ? 8 : 4;
+  for (int i = 0; i < 4; ++i)
+    if (int64_t(b[i].cl) * b[i].nt * b[i].nv * epv >= V) return i;
+  return -1;
+}
+
+template <typename T, bool HT>
+cudaError_t dispatch(const Build* builds, int i, const SweepArgs& a, cudaStream_t s) {
+  (void)builds;
+  if constexpr (sizeof(T) == 2) {
+    switch (i) {
+      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<T, 4, 512, 4, HT>(a, s);
+      case 3: return launch_cfg<T, 8, 512, 5, HT>(a, s);
+    }
+  } else {
+    switch (i) {
+      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<T, 4, 512, 5, HT>(a, s);
+      case 3: return launch_cfg<T, 8, 512, 10, HT>(a, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool sweep_supported(int dtype, int64_t V, bool /*has_target*/) { return pick_build(dtype, V) >= 0; }
+
+cudaError_t launch_sweep(int dtype, bool has_target, const SweepArgs& a, cudaStream_t s) {
+  const int i = pick_build(dtype, a.V);
+  if (i < 0) return cudaErrorInvalidValue;
+  if (dtype == DSPARK_BF16)
+    return has_target ? dispatch<__nv_bfloat16, true>(kBf16Builds, i, a, s)
+                      : dispatch<__nv_bfloat16, false>(kBf16Builds, i, a, s);
+  return has_target ? dispatch<float, true>(kF32Builds, i, a, s)
+                    : dispatch<float, false>(kF32Builds, i, a, s);
+}
+
+// ------------------------------------------------------- backward-only stream
+// dlogits from saved row statistics: one more read of the logits, no reductions.
+template <typename T, bool HAS_T>
+__global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a, const int64_t R) {
+  constexpr int EPV = VecTraits<T>::EPV;
+  const int vvec = int(a.V / EPV);
+  for (int64_t row = blockIdx.y; row < R; row += gridDim.y) {
+  uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * a.ld_g * sizeof(T);
+  const bool sup = a.ws.m[row] != 0;
+  if (!sup) {
+    for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x)
+      *reinterpret_cast<uint4*>(out + size_t(v) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    continue;
+  }
+  const float* st = a.ws.stats + size_t(row) * kStride;
+  const float g = a.grad_scale ? *a.grad_scale : 1.f;
+  const float gw = g * a.ws.w[row];
+  const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
+  const float S = st[kStS];
+  const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S), kzero = cce - cl1 * S;
+  const float lz2 = st[kStLseD] * kLog2e, lt2 = st[kStLseT] * kLog2e;
+  const int64_t tok = a.tids[row];
+  const uint8_t* zr = static_cast<const uint8_t*>(a.draft) + size_t(row) * a.ld_d * sizeof(T);
+  const uint8_t* tr = static_cast<const uint8_t*>(a.target) + size_t(row) * a.ld_t * sizeof(T);
+  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x) {
+    float z[EPV], t[EPV], o[EPV];
+    unpack16<T>(*reinterpret_cast<const uint4*>(zr + size_t(v) * 16), z);
+    if constexpr (HAS_T) unpack16<T>(*reinterpret_cast<const uint4*>(tr + size_t(v) * 16), t);
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) {
+      const float p = ex2(fmaf(z[e], kLog2e, -lz2));
+      if constexpr (HAS_T) {
+        const float d = p - ex2(fmaf(t[e], kLog2e, -lt2));
+        o[e] = p * (d > 0.f ? kpos : (d < 0.f ? kneg : kzero));
+      } else {
+        o[e] = p * cce;
+      }
+      if (int64_t(v) * EPV + e == tok) o[e] -= cce;
+    }
+    *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<T>(o);
+  }
+  }
+}
+
+cudaError_t launch_bwd_stream(int dtype, bool has_target, const SweepArgs& a, int64_t R,
+                              cudaStream_t s) {
+  const int epv = dtype == DSPARK_BF16 ? 8 : 4;
+  const int64_t vvec = a.V / epv;
+  const unsigned gx = unsigned(std::min<int64_t>((vvec + 1023) / 1024, 64));
+  dim3 grid(gx > 0 ? gx : 1, unsigned(std::min<int64_t>(R, 65535)), 1);
+  if (dtype == DSPARK_BF16) {
+    if (has_target) bwd_stream_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(a, R);
+    else bwd_stream_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(a, R);
+  } else {
+    if (has_target) bwd_stream_kernel<float, true><<<grid, 256, 0, s>>>(a, R);
+    else bwd_stream_kernel<float, false><<<grid, 256, 0, s>>>(a, R);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace dspark

@@ -1,0 +1,193 @@
+"""PyTorch-facing wrapper of the C ABI: builds the ABI structs from CUDA tensors,
+allocates the outputs with torch, and calls the library on the current stream.
+
+Argument marshalling only.  Nothing here computes any part of the loss.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import abi
+from .synthetic import DSparkInputs
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: Optional[torch.Tensor], dtype, name):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def problem_struct(inp: DSparkInputs) -> abi.dspark_problem_t:
+    """The dspark_problem_t describing ``inp`` (tensors must stay alive)."""
+    ldt = torch.float32 if inp.dtype == "f32" else torch.bfloat16
+    p = abi.dspark_problem_t()
+    p.B, p.N, p.K, p.V = inp.B, inp.N, inp.K, inp.V
+    p.logits_dtype = abi.DSPARK_F32 if inp.dtype == "f32" else abi.DSPARK_BF16
+    d = _need(inp.draft_logits, ldt, "draft_logits")
+    p.draft_logits, p.draft_ld = _ptr(d), inp.V
+    if inp.target_logits is not None:
+        p.target_logits = _ptr(_need(inp.target_logits, ldt, "target_logits"))
+        p.target_ld = inp.V
+    p.target_ids = _ptr(_need(inp.target_ids, torch.int64, "target_ids"))
+    p.eval_mask = _ptr(_need(inp.eval_mask, torch.uint8, "eval_mask"))
+    p.block_keep = _ptr(_need(inp.block_keep, torch.uint8, "block_keep"))
+    p.confidence_logits = _ptr(_need(inp.confidence_logits, torch.float32, "confidence_logits"))
+    if inp.lm_head is not None:
+        p.target_hidden = _ptr(_need(inp.target_hidden, torch.bfloat16, "target_hidden"))
+        p.lm_head = _ptr(_need(inp.lm_head, torch.bfloat16, "lm_head"))
+        p.target_hidden_size = inp.lm_head.shape[1]
+    if inp.markov_w2 is not None:
+        p.prev_ids = _ptr(_need(inp.prev_ids, torch.int64, "prev_ids"))
+        p.markov_w1 = _ptr(_need(inp.markov_w1, torch.bfloat16, "markov_w1"))
+        p.markov_w2 = _ptr(_need(inp.markov_w2, torch.bfloat16, "markov_w2"))
+        p.target_vocab = inp.markov_w1.shape[0]
+        p.markov_rank = inp.markov_w2.shape[1]
+    if inp.valid is not None:
+        p.valid = _ptr(_need(inp.valid, torch.uint8, "valid"))
+    if inp.conf_w is not None:
+        p.draft_hidden = _ptr(_need(inp.draft_hidden, torch.bfloat16, "draft_hidden"))
+        p.hidden_size = inp.draft_hidden.shape[-1]
+        p.conf_w = _ptr(_need(inp.conf_w, torch.bfloat16, "conf_w"))
+        p.conf_b = _ptr(_need(inp.conf_b, torch.float32, "conf_b"))
+        p.conf_with_markov = 1 if inp.conf_with_markov else 0
+    return p
+
+
+def params_struct(inp: DSparkInputs, invalid_row_mode: int = 0) -> abi.dspark_params_t:
+    prm = abi.dspark_params_t()
+    prm.ce_alpha, prm.l1_alpha, prm.conf_alpha = inp.ce_alpha, inp.l1_alpha, inp.conf_alpha
+    if inp.target_logits is None and inp.lm_head is None:
+        prm.l1_alpha = 0.0
+    prm.gamma = inp.gamma if inp.gamma is not None else 1.0
+    prm.gamma_enabled = 0 if inp.gamma is None else 1
+    prm.invalid_row_mode = invalid_row_mode
+    return prm
+
+
+def workspace_bytes(inp: DSparkInputs) -> int:
+    p = problem_struct(inp)
+    return int(abi.dspark_workspace_size(ctypes.byref(p)))
+
+
+def new_workspace(inp: DSparkInputs) -> torch.Tensor:
+    n = workspace_bytes(inp)
+    return torch.empty(n + 256, dtype=torch.uint8, device=inp.draft_logits.device)
+
+
+def _aligned_ws(ws: torch.Tensor):
+    base = ws.data_ptr()
+    off = (-base) % 256
+    return ctypes.c_void_p(base + off), ws.numel() - off
+
+
+class Outputs:
+    """Device buffers one fused call writes (allocated once, reusable)."""
+
+    def __init__(self, inp: DSparkInputs, rows: bool = True, grads: bool = True):
+        dev = inp.draft_logits.device
+        R = inp.R
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.loss_num = torch.zeros(1, **f32)
+        self.num_tokens = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.report = torch.zeros(abi.DSPARK_REP_COUNT, 2, **f32)
+        self.ce_rows = torch.zeros(R, **f32) if rows else None
+        self.l1_rows = torch.zeros(R, **f32) if rows else None
+        self.accept_rows = torch.zeros(R, **f32) if rows else None
+        self.conf_rows = torch.zeros(R, **f32) if rows else None
+        self.grad_scale = torch.full((1,), float(inp.grad_scale), **f32)
+        self.dlogits = torch.empty_like(inp.draft_logits) if grads else None
+        self.dconf = torch.zeros(R, **f32) if grads else None
+        self.dW1 = self.dW2 = self.dconf_w = self.dconf_b = self.dhidden = None
+        if grads and inp.markov_w2 is not None:
+            self.dW1 = torch.zeros(inp.markov_w1.shape, **f32)
+            self.dW2 = torch.zeros(inp.markov_w2.shape, **f32)
+        if grads and inp.conf_w is not None:
+            self.dconf_w = torch.zeros(inp.conf_w.numel(), **f32)
+            self.dconf_b = torch.zeros(1, **f32)
+            self.dhidden = torch.zeros(inp.draft_hidden.shape, dtype=torch.bfloat16, device=dev)
+        self.ws = new_workspace(inp)
+
+    def fwd_struct(self) -> abi.dspark_fwd_out_t:
+        o = abi.dspark_fwd_out_t()
+        o.loss_num, o.num_tokens, o.report = _ptr(self.loss_num), _ptr(self.num_tokens), _ptr(self.report)
+        o.ce_rows, o.l1_rows = _ptr(self.ce_rows), _ptr(self.l1_rows)
+        o.accept_rows, o.conf_rows = _ptr(self.accept_rows), _ptr(self.conf_rows)
+        return o
+
+    def grads_struct(self, inp: DSparkInputs, accumulate: bool = False) -> abi.dspark_grads_t:
+        g = abi.dspark_grads_t()
+        g.grad_scale = _ptr(self.grad_scale)
+        g.dlogits, g.dlogits_ld = _ptr(self.dlogits), inp.V
+        g.dconf = _ptr(self.dconf)
+        g.dW1, g.dW2 = _ptr(self.dW1), _ptr(self.dW2)
+        g.dconf_w, g.dconf_b, g.dhidden = _ptr(self.dconf_w), _ptr(self.dconf_b), _ptr(self.dhidden)
+        g.accumulate = 1 if accumulate else 0
+        return g
+
+
+class Call:
+    """A prepared fused forward+backward call: structs built once, launched many times."""
+
+    def __init__(self, inp: DSparkInputs, out: Optional[Outputs] = None, grads: bool = True,
+                 rows: bool = True, invalid_row_mode: int = 0, accumulate: bool = False):
+        self.inp = inp
+        self.out = out if out is not None else Outputs(inp, rows=rows, grads=grads)
+        self.prob = problem_struct(inp)
+        self.prm = params_struct(inp, invalid_row_mode)
+        self.fwd = self.out.fwd_struct()
+        self.grads = self.out.grads_struct(inp, accumulate) if grads else None
+        self.ws_ptr, self.ws_len = _aligned_ws(self.out.ws)
+
+    def launch(self, stream=None) -> None:
+        s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        st = abi.dspark_loss_fwd(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.fwd),
+                                 ctypes.byref(self.grads) if self.grads is not None else None,
+                                 self.ws_ptr, self.ws_len, ctypes.c_void_p(s))
+        abi.check(st, "dspark_loss_fwd")
+
+    def backward(self, stream=None) -> None:
+        s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        st = abi.dspark_loss_bwd(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.grads),
+                                 self.ws_ptr, self.ws_len, ctypes.c_void_p(s))
+        abi.check(st, "dspark_loss_bwd")
+
+    def check_status(self, stream=None) -> int:
+        s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+        return int(abi.dspark_check_status(self.ws_ptr, ctypes.c_void_p(s)))
+
+
+def dspark_loss(inp: DSparkInputs, grads: bool = True, rows: bool = True, invalid_row_mode: int = 0):
+    """One fused call on the current stream; returns the Outputs (not synchronised)."""
+    c = Call(inp, grads=grads, rows=rows, invalid_row_mode=invalid_row_mode)
+    c.launch()
+    return c.out
+
+
+def acceptance(l1_rows: torch.Tensor, eval_mask: torch.Tensor, block_keep: Optional[torch.Tensor] = None):
+    """Standalone acceptance report: (accept_pair[2], tau_pair[2], accept_rows[R])."""
+    B, N, K = eval_mask.shape
+    dev = l1_rows.device
+    _need(l1_rows, torch.float32, "l1_rows")
+    _need(eval_mask, torch.uint8, "eval_mask")
+    _need(block_keep, torch.uint8, "block_keep")
+    ap = torch.zeros(2, dtype=torch.float32, device=dev)
+    tp = torch.zeros(2, dtype=torch.float32, device=dev)
+    ar = torch.zeros(B * N * K, dtype=torch.float32, device=dev)
+    st = abi.dspark_acceptance(B, N, K, _ptr(l1_rows), _ptr(eval_mask), _ptr(block_keep), _ptr(ap),
+                               _ptr(tp), _ptr(ar), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    abi.check(st, "dspark_acceptance")
+    return ap, tp, ar

@@ -1,0 +1,150 @@
+"""Host-side checks of the C-ABI library: it loads, exports every symbol include/dspark.h
+declares, its structs have the layout the ctypes binding assumes, and host validation
+returns the documented status codes before touching the GPU.  No CUDA call is made."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dspark.h")
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from speculative_decoding_draft_vocab_b200 import build
+    build.build()
+    from speculative_decoding_draft_vocab_b200 import abi as _abi
+    return _abi
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"DSPARK_API\s+[\w\s\*]+?\b(dspark_\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(abi):
+    names = _declared_functions()
+    assert len(names) >= 6
+    for n in names:
+        assert hasattr(abi.lib, n), n
+        assert hasattr(abi, n), f"binding lacks {n}"
+
+
+C_LAYOUT = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "dspark.h"
+#define F(T, f) printf(#T " " #f " %zu\n", offsetof(T, f));
+#define S(T) printf(#T " sizeof %zu\n", sizeof(T));
+int main(void) {
+BODY
+  return 0;
+}
+"""
+
+
+def test_struct_layout_matches_ctypes(abi):
+    lines = []
+    for cls in (abi.dspark_problem_t, abi.dspark_params_t, abi.dspark_fwd_out_t, abi.dspark_grads_t):
+        t = cls.__name__
+        lines.append(f"  S({t})")
+        for f, _ in cls._fields_:
+            lines.append(f"  F({t}, {f})")
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        with open(src, "w") as f:
+            f.write(C_LAYOUT.replace("BODY", "\n".join(lines)))
+        subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), src, "-o", exe], check=True)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    got = {}
+    for line in out.splitlines():
+        t, f, v = line.split()
+        got[(t, f)] = int(v)
+    for cls in (abi.dspark_problem_t, abi.dspark_params_t, abi.dspark_fwd_out_t, abi.dspark_grads_t):
+        t = cls.__name__
+        assert got[(t, "sizeof")] == ctypes.sizeof(cls), t
+        for f, _ in cls._fields_:
+            assert got[(t, f)] == getattr(cls, f).offset, (t, f)
+
+
+def _problem(abi, V=1024, dtype=None, target=True):
+    p = abi.dspark_problem_t()
+    p.B, p.N, p.K, p.V = 1, 2, 4, V
+    p.logits_dtype = abi.DSPARK_BF16 if dtype is None else dtype
+    p.draft_logits, p.draft_ld = ctypes.c_void_p(0x10000), V
+    if target:
+        p.target_logits, p.target_ld = ctypes.c_void_p(0x20000), V
+    p.target_ids = ctypes.c_void_p(0x30000)
+    p.eval_mask = ctypes.c_void_p(0x40000)
+    return p
+
+
+def _params(abi, l1=0.9):
+    prm = abi.dspark_params_t()
+    prm.ce_alpha, prm.l1_alpha, prm.conf_alpha, prm.gamma = 0.1, l1, 1.0, 4.0
+    prm.gamma_enabled = 1
+    return prm
+
+
+def _fwd(abi, p, prm, ws=0x100000, ws_bytes=1 << 30, grads=None):
+    out = abi.dspark_fwd_out_t()
+    return abi.dspark_loss_fwd(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(out),
+                               ctypes.byref(grads) if grads is not None else None,
+                               ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def test_host_validation_status_codes(abi):
+    prm = _params(abi)
+    # a teacher-dependent term without the teacher is refused before launch
+    assert _fwd(abi, _problem(abi, target=False), prm) == abi.DSPARK_ERR_MISSING_TARGET
+    # V * sizeof(bf16) not a multiple of 16 bytes
+    assert _fwd(abi, _problem(abi, V=1020), prm) == abi.DSPARK_ERR_ALIGNMENT
+    # misaligned row pointer
+    p = _problem(abi)
+    p.draft_logits = ctypes.c_void_p(0x10008)
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_ALIGNMENT
+    # short workspace, missing workspace, misaligned workspace
+    p = _problem(abi)
+    assert _fwd(abi, p, prm, ws_bytes=16) == abi.DSPARK_ERR_WORKSPACE
+    assert _fwd(abi, p, prm, ws=0) == abi.DSPARK_ERR_WORKSPACE
+    assert _fwd(abi, p, prm, ws=0x100010) == abi.DSPARK_ERR_ALIGNMENT
+    # bad sizes / dtype
+    p = _problem(abi)
+    p.K = 0
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    p = _problem(abi, dtype=7)
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    # both confidence sources at once
+    p = _problem(abi)
+    p.confidence_logits = ctypes.c_void_p(0x50000)
+    p.conf_w = ctypes.c_void_p(0x60000)
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    # gamma enabled but not positive
+    prm2 = _params(abi)
+    prm2.gamma = 0.0
+    assert _fwd(abi, _problem(abi), prm2) == abi.DSPARK_ERR_INVALID_ARG
+    # a misaligned dlogits stride
+    g = abi.dspark_grads_t()
+    g.dlogits, g.dlogits_ld = ctypes.c_void_p(0x70000), 1028
+    assert _fwd(abi, _problem(abi), prm, grads=g) == abi.DSPARK_ERR_ALIGNMENT
+    # acceptance with NULL inputs
+    assert abi.dspark_acceptance(1, 1, 1, None, None, None, None, None, None, None) == abi.DSPARK_ERR_INVALID_ARG
+    assert abi.dspark_check_status(None, None) == abi.DSPARK_ERR_WORKSPACE
+
+
+def test_status_strings_and_workspace_size(abi):
+    for s in range(9):
+        assert abi.dspark_status_string(s)
+    p = _problem(abi)
+    n1 = abi.dspark_workspace_size(ctypes.byref(p))
+    p.N = 200
+    n2 = abi.dspark_workspace_size(ctypes.byref(p))
+    assert 0 < n1 < n2 and n1 % 256 == 0
+    p.K = 0
+    assert abi.dspark_workspace_size(ctypes.byref(p)) == 0
