@@ -9,8 +9,9 @@ Tolerances (fixed for the whole suite):
     where ref_o is the FP64 value rounded to the output dtype (bf16's half-ulp is
     above 2e-3, so a 1-ulp rounding flip is allowed), skipping elements whose
     sign(p - q) is not decided at FP32 precision (either sign is a valid L1
-    sub-gradient there); plus a per-row relative L2 error <= 2e-3 against the
-    unrounded FP64 row.
+    sub-gradient there); plus a per-row relative L2 error <= 2e-3 against the same
+    rounded row ref_o.  (Against the unrounded row, bf16 rounding alone reaches
+    2.5e-3 on rows whose mass sits in a few elements: a half-ulp is 2^-9.)
 """
 
 from __future__ import annotations
@@ -85,9 +86,9 @@ def check_dlogit_row(gpu_row: np.ndarray, ref_row: np.ndarray, amb: np.ndarray, 
         raise AssertionError(f"{tag} dlogits: {int(bad.sum())} elements off; worst j={j} "
                              f"gpu={gpu_row[j]!r} ref={ref_row[j]!r} tol={tol[j]!r}")
     keep = ~amb
-    nref = np.linalg.norm(ref_row[keep])
+    nref = np.linalg.norm(ref_o[keep])
     if nref > 0:
-        rel = np.linalg.norm((gpu_row - ref_row)[keep]) / nref
+        rel = np.linalg.norm((gpu_row - ref_o)[keep]) / nref
         assert rel <= REL_DLOGIT, f"{tag} dlogits row relative L2 error {rel:.3e}"
     return int(amb.sum())
 
