@@ -109,7 +109,28 @@ __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
   return v;
 }
 
+// Named barrier over `nthreads` threads (a multiple of 32); id 0 is __syncthreads.
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Store 16 bytes into (possibly another CTA's) shared memory at cluster address
+// `addr`; completion is counted on the mbarrier at cluster address `bar` (same CTA
+// as `addr`).
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar) : "memory");
+}
+
 // ---------------------------------------------------------------- math
+// max of three floats in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x on the SFU (ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -57,46 +57,67 @@ template <> __device__ __forceinline__ float load_elem<__nv_bfloat16>(const uint
   return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t*>(p)) << 16);
 }
 
-// (max, sum 2^(x - max)) in base-2 units; max = -inf marks an empty partial.
-struct MS {
-  float m, s;
-};
-__device__ __forceinline__ MS ms_combine(MS a, MS b) {
-  const float m = fmaxf(a.m, b.m);
-  if (m == -INFINITY) return MS{m, 0.f};
-  const float sa = (a.m == -INFINITY) ? 0.f : a.s * ex2(a.m - m);
-  const float sb = (b.m == -INFINITY) ? 0.f : b.s * ex2(b.m - m);
-  return MS{m, sa + sb};
+// ------------------------------------------------------------ reductions
+// Partial of a logsumexp in base 2: (m, s) with s = sum 2^(x - m); m = -inf is empty.
+// Combining takes the maximum first and then one rescaled sum, so each thread
+// spends one ex2 per reduction level group rather than one per pairwise merge.
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
 }
-__device__ __forceinline__ MS ms_shfl(MS v, int off) {
-  return MS{__shfl_xor_sync(0xffffffffu, v.m, off), __shfl_xor_sync(0xffffffffu, v.s, off)};
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+// (m, s) of every lane -> the warp's (M, S), identical in all lanes.
+__device__ __forceinline__ void warp_lse_merge(float& m, float& s) {
+  const float M = warp_max(m);
+  const float t = (m == -INFINITY) ? 0.f : s * ex2(m - M);
+  s = warp_sum(t);
+  m = M;
 }
 
-struct Ctrl {
-  uint64_t mbar[2];
-  float4 slotA;     // this CTA's (max, sum) partials of draft and teacher
-  float4 slotB;     // this CTA's (L1, S) partials
-  float4 red[32];   // per-warp partials
-  float4 bcast[2];  // row scalars broadcast to the CTA
-  float ztid;       // raw draft logit at the target id (owner CTA only)
+// Per warp-group (row stream) control block in shared memory.
+struct WgCtrl {
+  uint64_t mbar_data[2];  // row segment landed (bulk copies)
+  uint64_t mbar_ga;       // all cluster ranks' logsumexp partials landed
+  uint64_t mbar_gb;       // all cluster ranks' (L1, S) partials landed
+  float4 ga[16];          // (m_z, s_z, m_t, s_t) from rank i
+  float4 gb[16];          // (L1, S, 0, 0) from rank i
+  float4 red[16];         // per-warp partials
+  float4 bcast;           // row logsumexps (base 2)
+  float ztid;             // raw draft logit at the target id (owner only)
+  float pad[3];
 };
 
-template <typename T, int CL, int NT, int NV, bool HAS_T>
-__global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
+// One thread-block cluster of CL CTAs streams rows; each CTA holds WGS independent
+// warp groups of NTW threads, and warp group w of every CTA in the cluster works on
+// the same row, so WGS rows are in flight per cluster and one group's reductions
+// overlap the other's arithmetic.  Each thread keeps NV 16-byte vectors of its
+// segment of the row (as FP32 exponentials) in registers.
+template <typename T, int CL, int WGS, int NTW, int NV, bool HAS_T>
+__global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) {
   constexpr int EPV = VecTraits<T>::EPV;
   constexpr int NE = NV * EPV;
-  constexpr int NW = NT / 32;
+  constexpr int NW = NTW / 32;
   constexpr int NTENS = HAS_T ? 2 : 1;
-  static_assert(NW <= 32, "one warp combines the per-warp partials");
+  static_assert(NW <= 16 && CL <= 16, "control block sizes");
+  static_assert(NE % 2 == 0, "pairs of elements");
   extern __shared__ __align__(128) uint8_t smem[];
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wg = threadIdx.x / NTW;
+  const int tid = threadIdx.x % NTW;
+  const int lane = tid & 31, warp = tid >> 5;
+  const uint32_t bar_id = 1 + wg;
   const uint32_t rank = cluster_ctarank();
   const uint32_t cid = cluster_id_x();
   const uint32_t G = nclusters_x();
   const uint32_t seg_bytes = uint32_t(a.seg_vec) * 16u;
   const int nbuf = a.nbuf;
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + size_t(nbuf) * NTENS * seg_bytes);
+  uint8_t* wg_bufs = smem + size_t(wg) * nbuf * NTENS * seg_bytes;
+  WgCtrl* ctrl = reinterpret_cast<WgCtrl*>(smem + size_t(WGS) * nbuf * NTENS * seg_bytes) + wg;
   WsHeader* hdr = a.ws.hdr;
 
   const int v0 = int(rank) * a.seg_vec;
@@ -104,23 +125,27 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t bytes = uint32_t(nvec) * 16u;
   const int n_sup = hdr->n_sup;
   const int n_zero = hdr->n_zero;
-  const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
+  const int sid = int(cid) * WGS + wg;     // this row stream
+  const int NS = int(G) * WGS;             // streams in the grid
+  const int my_n = (sid < n_sup) ? (n_sup - 1 - sid) / NS + 1 : 0;
   const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
   const uint8_t* target = static_cast<const uint8_t*>(a.target);
   const bool bwd = a.dlogits != nullptr;
   const float g = a.grad_scale ? *a.grad_scale : 1.f;
 
   auto buf = [&](int b, int tsel) -> uint8_t* {
-    return smem + (size_t(b) * NTENS + tsel) * seg_bytes;
+    return wg_bufs + (size_t(b) * NTENS + tsel) * seg_bytes;
   };
-  const uint32_t bar0 = smem_u32(&ctrl->mbar[0]);
-  const uint32_t bar1 = smem_u32(&ctrl->mbar[1]);
+  const uint32_t bar_data0 = smem_u32(&ctrl->mbar_data[0]);
+  const uint32_t bar_data1 = smem_u32(&ctrl->mbar_data[1]);
+  const uint32_t bar_ga = smem_u32(&ctrl->mbar_ga);
+  const uint32_t bar_gb = smem_u32(&ctrl->mbar_gb);
   uint64_t policy = 0;
 
-  auto issue = [&](int j) {  // thread 0: stream row j's segment into buffer j % nbuf
+  auto issue = [&](int j) {  // thread 0 of the group: stream row j's segment
     const int b = j % nbuf;
-    const uint32_t bar = b ? bar1 : bar0;
-    const int64_t row = a.ws.sup_list[cid + size_t(j) * G];
+    const uint32_t bar = b ? bar_data1 : bar_data0;
+    const int64_t row = a.ws.sup_list[sid + size_t(j) * NS];
     mbar_arrive_expect_tx(bar, NTENS * bytes);
     if (bytes) {
       bulk_g2s(smem_u32(buf(b, 0)), draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * sizeof(T),
@@ -131,34 +156,39 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
                  policy);
     }
   };
+  auto flag_timeout = [&]() { atomicOr(&hdr->status, kFlagTimeout); };
 
   if (tid == 0) {
     policy = l2_policy_evict_first();
-    mbar_init(bar0, 1);
-    mbar_init(bar1, 1);
+    mbar_init(bar_data0, 1);
+    mbar_init(bar_data1, 1);
+    mbar_init(bar_ga, 1);
+    mbar_init(bar_gb, 1);
     fence_mbar_init();
-    for (int j = 0; j < min(nbuf, my_n); ++j) issue(j);
   }
+  // every CTA's barriers exist before any peer signals them
   __syncthreads();
+  cluster_sync();
+  if (tid == 0)
+    for (int j = 0; j < min(nbuf, my_n); ++j) issue(j);
 
   for (int j = 0; j < my_n; ++j) {
     const int b = j % nbuf;
     const uint32_t phase = uint32_t(j / nbuf) & 1u;
-    const int64_t row = a.ws.sup_list[cid + size_t(j) * G];
+    const uint32_t gphase = uint32_t(j) & 1u;
+    const int64_t row = a.ws.sup_list[sid + size_t(j) * NS];
     const int64_t tok = a.tids[row];
     const int tv = int(tok / EPV) - v0;  // target id's vector inside this segment
     const int te = int(tok % EPV);
 
-    if (!mbar_wait_bounded(b ? bar1 : bar0, phase)) {
-      if (tid == 0) atomicOr(&hdr->status, kFlagTimeout);
-    }
+    if (!mbar_wait_bounded(b ? bar_data1 : bar_data0, phase) && tid == 0) flag_timeout();
 
     // ---- segment -> registers
     float xz[NE];
-    float xt[HAS_T ? NE : 1];
+    float xt[HAS_T ? NE : 2];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      const int v = tid + i * NT;
+      const int v = tid + i * NTW;
       if (v < nvec) {
         unpack16<T>(*reinterpret_cast<const uint4*>(buf(b, 0) + size_t(v) * 16), &xz[i * EPV]);
         if constexpr (HAS_T)
@@ -173,15 +203,15 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     }
     if (tid == 0 && tv >= 0 && tv < nvec)
       ctrl->ztid = load_elem<T>(buf(b, 0) + size_t(tv) * 16 + size_t(te) * sizeof(T));
-    __syncthreads();  // the buffer is free again
+    named_bar(bar_id, NTW);  // the buffer is free again
     if (tid == 0 && j + nbuf < my_n) issue(j + nbuf);
 
     // ---- pass 1: per-thread max, exponentials kept in registers, sums
     float mz = -INFINITY, mt = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < NE; ++e) {
-      mz = fmaxf(mz, xz[e]);
-      if constexpr (HAS_T) mt = fmaxf(mt, xt[e]);
+    for (int e = 0; e < NE; e += 2) {
+      mz = fmax3(mz, xz[e], xz[e + 1]);
+      if constexpr (HAS_T) mt = fmax3(mt, xt[e], xt[e + 1]);
     }
     const float oz = (mz == -INFINITY) ? 0.f : mz * kLog2e;
     const float ot = (mt == -INFINITY) ? 0.f : mt * kLog2e;
@@ -195,86 +225,75 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         st += xt[e];
       }
     }
-    MS pz{mz == -INFINITY ? -INFINITY : oz, sz};
-    MS pt{mt == -INFINITY ? -INFINITY : ot, st};
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      pz = ms_combine(pz, ms_shfl(pz, off));
-      if constexpr (HAS_T) pt = ms_combine(pt, ms_shfl(pt, off));
+    {
+      float m1 = (mz == -INFINITY) ? -INFINITY : oz, s1 = sz;
+      float m2 = (mt == -INFINITY) ? -INFINITY : ot, s2 = st;
+      warp_lse_merge(m1, s1);
+      if constexpr (HAS_T) warp_lse_merge(m2, s2);
+      if (lane == 0) ctrl->red[warp] = make_float4(m1, s1, m2, s2);
     }
-    if (lane == 0) ctrl->red[warp] = make_float4(pz.m, pz.s, pt.m, pt.s);
-    __syncthreads();
+    named_bar(bar_id, NTW);
     if (warp == 0) {
       const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-      MS qz{r4.x, r4.y}, qt{r4.z, r4.w};
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        qz = ms_combine(qz, ms_shfl(qz, off));
-        if constexpr (HAS_T) qt = ms_combine(qt, ms_shfl(qt, off));
+      float m1 = r4.x, s1 = r4.y, m2 = r4.z, s2 = r4.w;
+      warp_lse_merge(m1, s1);
+      if constexpr (HAS_T) warp_lse_merge(m2, s2);
+      if (lane == 0) mbar_arrive_expect_tx(bar_ga, CL * 16);
+      __syncwarp();
+      if (lane < CL) {  // all-gather of this CTA's partial into every rank
+        const uint32_t dst = dsmem_map(smem_u32(&ctrl->ga[rank]), uint32_t(lane));
+        st_async_f4(dst, make_float4(m1, s1, m2, s2), dsmem_map(bar_ga, uint32_t(lane)));
       }
-      if (lane == 0) ctrl->slotA = make_float4(qz.m, qz.s, qt.m, qt.s);
+      if (!mbar_wait_bounded(bar_ga, gphase) && lane == 0) flag_timeout();
+      const float4 q4 = lane < CL ? ctrl->ga[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      float n1 = q4.x, u1 = q4.y, n2 = q4.z, u2 = q4.w;
+      warp_lse_merge(n1, u1);
+      if constexpr (HAS_T) warp_lse_merge(n2, u2);
+      if (lane == 0) ctrl->bcast = make_float4(n1 + log2f(u1), HAS_T ? n2 + log2f(u2) : 0.f, 0.f, 0.f);
     }
-    cluster_sync();
-    if (warp == 0) {
-      float4 r4 = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-      if (lane < CL) r4 = dsmem_ld_f4(dsmem_map(smem_u32(&ctrl->slotA), uint32_t(lane)));
-      MS qz{r4.x, r4.y}, qt{r4.z, r4.w};
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        qz = ms_combine(qz, ms_shfl(qz, off));
-        if constexpr (HAS_T) qt = ms_combine(qt, ms_shfl(qt, off));
-      }
-      if (lane == 0)
-        ctrl->bcast[0] = make_float4(qz.m + log2f(qz.s), HAS_T ? qt.m + log2f(qt.s) : 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
-    const float lz2 = ctrl->bcast[0].x;  // lse_d in base-2 units
-    const float lt2 = ctrl->bcast[0].y;
+    named_bar(bar_id, NTW);
+    const float4 lse4 = ctrl->bcast;
+    const float lz2 = lse4.x;  // lse_d in base-2 units
+    const float lt2 = lse4.y;
     const float az = (mz == -INFINITY) ? 0.f : ex2(oz - lz2);  // p = e * az
     const float at = (!HAS_T || mt == -INFINITY) ? 0.f : ex2(ot - lt2);
 
-    // ---- pass 2: L1 and S
+    // ---- pass 2: L1 and S; keeps p in xz and u = p*sign(p - q) in xt
     float L1 = 0.f, S = 0.f;
     if constexpr (HAS_T) {
       float l1p = 0.f, sp = 0.f;
 #pragma unroll
       for (int e = 0; e < NE; ++e) {
-        const float p = xz[e] * az, q = xt[e] * at, d = p - q;
+        const float p = __fmul_rn(xz[e], az);
+        const float q = __fmul_rn(xt[e], at);
+        const float d = __fsub_rn(p, q);
+        const float u = d != 0.f ? copysignf(p, d) : 0.f;
         l1p += fabsf(d);
-        sp += d > 0.f ? p : (d < 0.f ? -p : 0.f);
+        sp += u;
+        xz[e] = p;
+        xt[e] = u;
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        l1p += __shfl_xor_sync(0xffffffffu, l1p, off);
-        sp += __shfl_xor_sync(0xffffffffu, sp, off);
-      }
+      l1p = warp_sum(l1p);
+      sp = warp_sum(sp);
       if (lane == 0) ctrl->red[warp] = make_float4(l1p, sp, 0.f, 0.f);
-      __syncthreads();
+      named_bar(bar_id, NTW);
       if (warp == 0) {
         const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-        float x = r4.x, y = r4.y;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          x += __shfl_xor_sync(0xffffffffu, x, off);
-          y += __shfl_xor_sync(0xffffffffu, y, off);
+        const float x = warp_sum(r4.x), y = warp_sum(r4.y);
+        if (lane == 0) mbar_arrive_expect_tx(bar_gb, CL * 16);
+        __syncwarp();
+        if (lane < CL) {
+          const uint32_t dst = dsmem_map(smem_u32(&ctrl->gb[rank]), uint32_t(lane));
+          st_async_f4(dst, make_float4(x, y, 0.f, 0.f), dsmem_map(bar_gb, uint32_t(lane)));
         }
-        if (lane == 0) ctrl->slotB = make_float4(x, y, 0.f, 0.f);
       }
-      cluster_sync();
-      if (warp == 0) {
-        float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lane < CL) r4 = dsmem_ld_f4(dsmem_map(smem_u32(&ctrl->slotB), uint32_t(lane)));
-        float x = r4.x, y = r4.y;
+      if (!mbar_wait_bounded(bar_gb, gphase) && tid == 0) flag_timeout();
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          x += __shfl_xor_sync(0xffffffffu, x, off);
-          y += __shfl_xor_sync(0xffffffffu, y, off);
-        }
-        if (lane == 0) ctrl->bcast[1] = make_float4(x, y, 0.f, 0.f);
+      for (int i = 0; i < CL; ++i) {  // same order in every CTA
+        const float4 q4 = ctrl->gb[i];
+        L1 += q4.x;
+        S += q4.y;
       }
-      __syncthreads();
-      L1 = ctrl->bcast[1].x;
-      S = ctrl->bcast[1].y;
     }
 
     // ---- per-row statistics
@@ -292,28 +311,21 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
       }
     }
 
-    // ---- pass 3: dlogits
+    // ---- pass 3: dlogits = p*(cce - cl1*S) + cl1*u, minus cce at the target id
     if (bwd) {
       const float gw = g * a.ws.w[row];
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
-      const float kpos = cce + cl1 * (1.f - S);
-      const float kneg = cce + cl1 * (-1.f - S);
-      const float kzero = cce - cl1 * S;
+      const float k0 = cce - cl1 * S;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
-        const int v = tid + i * NT;
+        const int v = tid + i * NTW;
         if (v < nvec) {
           float o[EPV];
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
-            const float p = xz[i * EPV + e] * az;
-            if constexpr (HAS_T) {
-              const float d = p - xt[i * EPV + e] * at;
-              o[e] = p * (d > 0.f ? kpos : (d < 0.f ? kneg : kzero));
-            } else {
-              o[e] = p * cce;
-            }
+            if constexpr (HAS_T) o[e] = fmaf(xt[i * EPV + e], cl1, xz[i * EPV + e] * k0);
+            else o[e] = (xz[i * EPV + e] * az) * cce;
           }
           if (v == tv) {
 #pragma unroll
@@ -328,15 +340,16 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
   // ---- rows outside the supervision mask: dlogits = 0
   if (bwd && n_zero > 0) {
-    const int first = ((int(cid) - n_sup) % int(G) + int(G)) % int(G);
+    const int first = ((sid - n_sup) % NS + NS) % NS;
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-    for (int zi = first; zi < n_zero; zi += int(G)) {
+    for (int zi = first; zi < n_zero; zi += NS) {
       const int64_t row = a.ws.zero_list[zi];
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
-      for (int v = tid; v < nvec; v += NT) *reinterpret_cast<uint4*>(out + size_t(v) * 16) = z4;
+      for (int v = tid; v < nvec; v += NTW) *reinterpret_cast<uint4*>(out + size_t(v) * 16) = z4;
     }
   }
-  // no CTA leaves while a peer may still read its shared memory
+  // no CTA leaves while a peer may still signal or read its shared memory
+  __syncthreads();
   cluster_sync();
 }
 
@@ -347,11 +360,10 @@ struct LaunchCache {
   std::mutex mu;
   int dev = -1;
   size_t smem = 0;
-  const void* fn = nullptr;
   int clusters = 0;
 };
 
-template <typename T, int CL, int NT, int NV, bool HAS_T>
+template <typename T, int CL, int WGS, int NTW, int NV, bool HAS_T>
 cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   constexpr int EPV = VecTraits<T>::EPV;
   constexpr int NTENS = HAS_T ? 2 : 1;
@@ -359,32 +371,36 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   a.vvec = int32_t(a.V / EPV);
   a.seg_vec = (a.vvec + CL - 1) / CL;
   const size_t per_buf = size_t(a.seg_vec) * 16 * NTENS;
-  const size_t ctrl = sizeof(Ctrl);
+  const size_t ctrl = sizeof(WgCtrl) * WGS;
   constexpr size_t kMaxSmem = 227 * 1024;
-  a.nbuf = (2 * per_buf + ctrl <= kMaxSmem) ? 2 : 1;
-  const size_t smem = a.nbuf * per_buf + ctrl;
+  a.nbuf = (2 * per_buf * WGS + ctrl <= kMaxSmem) ? 2 : 1;
+  const size_t smem = a.nbuf * per_buf * WGS + ctrl;
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
-  auto kern = sweep_kernel<T, CL, NT, NV, HAS_T>;
+  auto kern = sweep_kernel<T, CL, WGS, NTW, NV, HAS_T>;
   static LaunchCache cache;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CL;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
   int clusters = 0;
   {
     std::lock_guard<std::mutex> lk(cache.mu);
     if (cache.dev != dev || cache.smem != smem) {
       err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxSmem));
       if (err != cudaSuccess) return err;
+      if (CL > 8) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (err != cudaSuccess) return err;
+      }
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(CL, 1, 1);
-      q.blockDim = dim3(NT, 1, 1);
+      q.blockDim = dim3(WGS * NTW, 1, 1);
       q.dynamicSmemBytes = smem;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = CL;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
       q.attrs = at;
       q.numAttrs = 1;
       int n = 0;
@@ -403,50 +419,45 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(clusters * CL), 1, 1);
-  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.blockDim = dim3(WGS * NTW, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = CL;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// Capacity of a (CL, NT, NV) build = CL * NT * NV * elements-per-vector.
-struct Build {
-  int cl, nt, nv;
-};
-constexpr Build kBf16Builds[] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}};
-constexpr Build kF32Builds[] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 5}, {8, 512, 10}};
+// A build covers rows of up to CL * NTW * NV * (elements per vector) logits.
+constexpr int kNumBuilds = 5;
+constexpr int64_t kBf16Cap[kNumBuilds] = {1 * 128 * 1 * 8, 2 * 256 * 2 * 8, 4 * 256 * 4 * 8,
+                                          8 * 256 * 5 * 8, 16 * 256 * 5 * 8};
+constexpr int64_t kF32Cap[kNumBuilds] = {1 * 128 * 2 * 4, 2 * 256 * 4 * 4, 4 * 256 * 8 * 4,
+                                         8 * 256 * 10 * 4, 16 * 256 * 10 * 4};
 
 int pick_build(int dtype, int64_t V) {
-  const Build* b = dtype == DSPARK_BF16 ? kBf16Builds : kF32Builds;
-  const int epv = dtype == DSPARK_BF16 ? 8 : 4;
-  for (int i = 0; i < 4; ++i)
-    if (int64_t(b[i].cl) * b[i].nt * b[i].nv * epv >= V) return i;
+  const int64_t* cap = dtype == DSPARK_BF16 ? kBf16Cap : kF32Cap;
+  for (int i = 0; i < kNumBuilds; ++i)
+    if (cap[i] >= V) return i;
   return -1;
 }
 
 template <typename T, bool HT>
-cudaError_t dispatch(const Build* builds, int i, const SweepArgs& a, cudaStream_t s) {
-  (void)builds;
+cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
     switch (i) {
-      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<T, 4, 512, 4, HT>(a, s);
-      case 3: return launch_cfg<T, 8, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<T, 1, 2, 128, 1, HT>(a, s);
+      case 1: return launch_cfg<T, 2, 2, 256, 2, HT>(a, s);
+      case 2: return launch_cfg<T, 4, 2, 256, 4, HT>(a, s);
+      case 3: return launch_cfg<T, 8, 2, 256, 5, HT>(a, s);
+      case 4: return launch_cfg<T, 16, 2, 256, 5, HT>(a, s);
     }
   } else {
     switch (i) {
-      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<T, 4, 512, 5, HT>(a, s);
-      case 3: return launch_cfg<T, 8, 512, 10, HT>(a, s);
+      case 0: return launch_cfg<T, 1, 2, 128, 2, HT>(a, s);
+      case 1: return launch_cfg<T, 2, 2, 256, 4, HT>(a, s);
+      case 2: return launch_cfg<T, 4, 2, 256, 8, HT>(a, s);
+      case 3: return launch_cfg<T, 8, 2, 256, 10, HT>(a, s);
+      case 4: return launch_cfg<T, 16, 2, 256, 10, HT>(a, s);
     }
   }
   return cudaErrorInvalidValue;
@@ -460,10 +471,8 @@ cudaError_t launch_sweep(int dtype, bool has_target, const SweepArgs& a, cudaStr
   const int i = pick_build(dtype, a.V);
   if (i < 0) return cudaErrorInvalidValue;
   if (dtype == DSPARK_BF16)
-    return has_target ? dispatch<__nv_bfloat16, true>(kBf16Builds, i, a, s)
-                      : dispatch<__nv_bfloat16, false>(kBf16Builds, i, a, s);
-  return has_target ? dispatch<float, true>(kF32Builds, i, a, s)
-                    : dispatch<float, false>(kF32Builds, i, a, s);
+    return has_target ? dispatch<__nv_bfloat16, true>(i, a, s) : dispatch<__nv_bfloat16, false>(i, a, s);
+  return has_target ? dispatch<float, true>(i, a, s) : dispatch<float, false>(i, a, s);
 }
 
 // ------------------------------------------------------- backward-only stream
