@@ -79,45 +79,44 @@ __device__ __forceinline__ void warp_lse_merge(float& m, float& s) {
   m = M;
 }
 
-// Per warp-group (row stream) control block in shared memory.
-struct WgCtrl {
-  uint64_t mbar_data[2];  // row segment landed (bulk copies)
+// Control block in shared memory.
+struct Ctrl {
+  uint64_t mbar_data[2];  // row segment (draft + teacher) landed
   uint64_t mbar_ga;       // all cluster ranks' logsumexp partials landed
   uint64_t mbar_gb;       // all cluster ranks' (L1, S) partials landed
   float4 ga[16];          // (m_z, s_z, m_t, s_t) from rank i
   float4 gb[16];          // (L1, S, 0, 0) from rank i
-  float4 red[16];         // per-warp partials
+  float4 red[32];         // per-warp partials
   float4 bcast;           // row logsumexps (base 2)
   float ztid;             // raw draft logit at the target id (owner only)
   float pad[3];
 };
 
-// One thread-block cluster of CL CTAs streams rows; each CTA holds WGS independent
-// warp groups of NTW threads, and warp group w of every CTA in the cluster works on
-// the same row, so WGS rows are in flight per cluster and one group's reductions
-// overlap the other's arithmetic.  Each thread keeps NV 16-byte vectors of its
-// segment of the row (as FP32 exponentials) in registers.
-template <typename T, int CL, int WGS, int NTW, int NV, bool HAS_T>
-__global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) {
+// One cluster of CL CTAs owns one supervised row at a time; CTA `rank` owns the
+// rank-th contiguous segment of the vocabulary.  Draft values live in registers
+// (NV 16-byte vectors per thread, as FP32 exponentials); the teacher segment stays
+// in shared memory as loaded and is re-read, so a CTA holds 6 bytes per logit pair
+// on chip and a row fits in 4 SMs of a 148-SM part.  Shared memory holds one draft
+// landing buffer and two teacher buffers: the next row's copy is issued as soon as
+// the current draft segment is in registers, one full row ahead of its use.
+template <typename T, int CL, int NT, int NV, bool HAS_T>
+__global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   constexpr int EPV = VecTraits<T>::EPV;
   constexpr int NE = NV * EPV;
-  constexpr int NW = NTW / 32;
-  constexpr int NTENS = HAS_T ? 2 : 1;
-  static_assert(NW <= 16 && CL <= 16, "control block sizes");
+  constexpr int NW = NT / 32;
+  static_assert(NW <= 32 && CL <= 16, "control block sizes");
   static_assert(NE % 2 == 0, "pairs of elements");
   extern __shared__ __align__(128) uint8_t smem[];
 
-  const int wg = threadIdx.x / NTW;
-  const int tid = threadIdx.x % NTW;
-  const int lane = tid & 31, warp = tid >> 5;
-  const uint32_t bar_id = 1 + wg;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
   const uint32_t cid = cluster_id_x();
   const uint32_t G = nclusters_x();
   const uint32_t seg_bytes = uint32_t(a.seg_vec) * 16u;
-  const int nbuf = a.nbuf;
-  uint8_t* wg_bufs = smem + size_t(wg) * nbuf * NTENS * seg_bytes;
-  WgCtrl* ctrl = reinterpret_cast<WgCtrl*>(smem + size_t(WGS) * nbuf * NTENS * seg_bytes) + wg;
+  // buffers: HAS_T: [draft][teacher 0][teacher 1]; else [draft 0][draft 1]
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + size_t(3 - (HAS_T ? 0 : 1)) * seg_bytes);
+  auto zbuf = [&](int j) -> uint8_t* { return HAS_T ? smem : smem + size_t(j & 1) * seg_bytes; };
+  auto tbuf = [&](int j) -> uint8_t* { return smem + size_t(1 + (j & 1)) * seg_bytes; };
   WsHeader* hdr = a.ws.hdr;
 
   const int v0 = int(rank) * a.seg_vec;
@@ -125,43 +124,36 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
   const uint32_t bytes = uint32_t(nvec) * 16u;
   const int n_sup = hdr->n_sup;
   const int n_zero = hdr->n_zero;
-  const int sid = int(cid) * WGS + wg;     // this row stream
-  const int NS = int(G) * WGS;             // streams in the grid
-  const int my_n = (sid < n_sup) ? (n_sup - 1 - sid) / NS + 1 : 0;
+  const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
   const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
   const uint8_t* target = static_cast<const uint8_t*>(a.target);
   const bool bwd = a.dlogits != nullptr;
   const float g = a.grad_scale ? *a.grad_scale : 1.f;
 
-  auto buf = [&](int b, int tsel) -> uint8_t* {
-    return wg_bufs + (size_t(b) * NTENS + tsel) * seg_bytes;
-  };
-  const uint32_t bar_data0 = smem_u32(&ctrl->mbar_data[0]);
-  const uint32_t bar_data1 = smem_u32(&ctrl->mbar_data[1]);
+  const uint32_t bar_d0 = smem_u32(&ctrl->mbar_data[0]);
+  const uint32_t bar_d1 = smem_u32(&ctrl->mbar_data[1]);
   const uint32_t bar_ga = smem_u32(&ctrl->mbar_ga);
   const uint32_t bar_gb = smem_u32(&ctrl->mbar_gb);
   uint64_t policy = 0;
 
-  auto issue = [&](int j) {  // thread 0 of the group: stream row j's segment
-    const int b = j % nbuf;
-    const uint32_t bar = b ? bar_data1 : bar_data0;
-    const int64_t row = a.ws.sup_list[sid + size_t(j) * NS];
-    mbar_arrive_expect_tx(bar, NTENS * bytes);
+  auto issue = [&](int j) {  // thread 0: stream row j's segment (draft and teacher)
+    const uint32_t bar = (j & 1) ? bar_d1 : bar_d0;
+    const int64_t row = a.ws.sup_list[cid + size_t(j) * G];
+    mbar_arrive_expect_tx(bar, (HAS_T ? 2u : 1u) * bytes);
     if (bytes) {
-      bulk_g2s(smem_u32(buf(b, 0)), draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * sizeof(T),
+      bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * sizeof(T),
                bytes, bar, policy);
       if constexpr (HAS_T)
-        bulk_g2s(smem_u32(buf(b, 1)),
-                 target + (size_t(row) * a.ld_t + size_t(v0) * EPV) * sizeof(T), bytes, bar,
-                 policy);
+        bulk_g2s(smem_u32(tbuf(j)), target + (size_t(row) * a.ld_t + size_t(v0) * EPV) * sizeof(T),
+                 bytes, bar, policy);
     }
   };
   auto flag_timeout = [&]() { atomicOr(&hdr->status, kFlagTimeout); };
 
   if (tid == 0) {
     policy = l2_policy_evict_first();
-    mbar_init(bar_data0, 1);
-    mbar_init(bar_data1, 1);
+    mbar_init(bar_d0, 1);
+    mbar_init(bar_d1, 1);
     mbar_init(bar_ga, 1);
     mbar_init(bar_gb, 1);
     fence_mbar_init();
@@ -169,49 +161,70 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
   // every CTA's barriers exist before any peer signals them
   __syncthreads();
   cluster_sync();
-  if (tid == 0)
-    for (int j = 0; j < min(nbuf, my_n); ++j) issue(j);
+  if (tid == 0) {
+    if (my_n > 0) issue(0);
+    if (!HAS_T && my_n > 1) issue(1);
+  }
+
+  // per-row scalars, loaded one row ahead
+  int64_t row = my_n > 0 ? a.ws.sup_list[cid] : 0;
+  int64_t tok = my_n > 0 ? a.tids[row] : 0;
+  float wr = my_n > 0 ? a.ws.w[row] : 0.f;
 
   for (int j = 0; j < my_n; ++j) {
-    const int b = j % nbuf;
-    const uint32_t phase = uint32_t(j / nbuf) & 1u;
+    const uint32_t phase = uint32_t(j >> 1) & 1u;
     const uint32_t gphase = uint32_t(j) & 1u;
-    const int64_t row = a.ws.sup_list[sid + size_t(j) * NS];
-    const int64_t tok = a.tids[row];
     const int tv = int(tok / EPV) - v0;  // target id's vector inside this segment
     const int te = int(tok % EPV);
+    const uint8_t* zb = zbuf(j);
+    const uint8_t* tb = tbuf(j);
 
-    if (!mbar_wait_bounded(b ? bar_data1 : bar_data0, phase) && tid == 0) flag_timeout();
+    if (!mbar_wait_bounded((j & 1) ? bar_d1 : bar_d0, phase) && tid == 0) flag_timeout();
 
-    // ---- segment -> registers
+    // ---- draft segment -> registers
     float xz[NE];
-    float xt[HAS_T ? NE : 2];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      const int v = tid + i * NTW;
+      const int v = tid + i * NT;
       if (v < nvec) {
-        unpack16<T>(*reinterpret_cast<const uint4*>(buf(b, 0) + size_t(v) * 16), &xz[i * EPV]);
-        if constexpr (HAS_T)
-          unpack16<T>(*reinterpret_cast<const uint4*>(buf(b, 1) + size_t(v) * 16), &xt[i * EPV]);
+        unpack16<T>(*reinterpret_cast<const uint4*>(zb + size_t(v) * 16), &xz[i * EPV]);
       } else {
 #pragma unroll
-        for (int e = 0; e < EPV; ++e) {
-          xz[i * EPV + e] = -INFINITY;
-          if constexpr (HAS_T) xt[i * EPV + e] = -INFINITY;
-        }
+        for (int e = 0; e < EPV; ++e) xz[i * EPV + e] = -INFINITY;
       }
     }
     if (tid == 0 && tv >= 0 && tv < nvec)
-      ctrl->ztid = load_elem<T>(buf(b, 0) + size_t(tv) * 16 + size_t(te) * sizeof(T));
-    named_bar(bar_id, NTW);  // the buffer is free again
-    if (tid == 0 && j + nbuf < my_n) issue(j + nbuf);
+      ctrl->ztid = load_elem<T>(zb + size_t(tv) * 16 + size_t(te) * sizeof(T));
+    __syncthreads();  // the draft buffer is free again
+    if (tid == 0) {
+      // HAS_T: draft buffer + the teacher buffer of row j-1 (its pass 2 is done).
+      // Without a teacher the draft buffers alternate.
+      if (HAS_T && j + 1 < my_n) issue(j + 1);
+      if (!HAS_T && j + 2 < my_n) issue(j + 2);
+    }
+    int64_t nrow = 0, ntok = 0;
+    float nw = 0.f;
+    if (j + 1 < my_n) {
+      nrow = a.ws.sup_list[cid + size_t(j + 1) * G];
+      ntok = a.tids[nrow];
+      nw = a.ws.w[nrow];
+    }
 
-    // ---- pass 1: per-thread max, exponentials kept in registers, sums
+    // ---- pass 1: per-thread maxima, draft exponentials kept, sums
     float mz = -INFINITY, mt = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < NE; e += 2) {
-      mz = fmax3(mz, xz[e], xz[e + 1]);
-      if constexpr (HAS_T) mt = fmax3(mt, xt[e], xt[e + 1]);
+    for (int e = 0; e < NE; e += 2) mz = fmax3(mz, xz[e], xz[e + 1]);
+    if constexpr (HAS_T) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int v = tid + i * NT;
+        if (v < nvec) {
+          float t8[EPV];
+          unpack16<T>(*reinterpret_cast<const uint4*>(tb + size_t(v) * 16), t8);
+#pragma unroll
+          for (int e = 0; e < EPV; e += 2) mt = fmax3(mt, t8[e], t8[e + 1]);
+        }
+      }
     }
     const float oz = (mz == -INFINITY) ? 0.f : mz * kLog2e;
     const float ot = (mt == -INFINITY) ? 0.f : mt * kLog2e;
@@ -220,9 +233,17 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
     for (int e = 0; e < NE; ++e) {
       xz[e] = ex2(fmaf(xz[e], kLog2e, -oz));
       sz += xz[e];
-      if constexpr (HAS_T) {
-        xt[e] = ex2(fmaf(xt[e], kLog2e, -ot));
-        st += xt[e];
+    }
+    if constexpr (HAS_T) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int v = tid + i * NT;
+        if (v < nvec) {
+          float t8[EPV];
+          unpack16<T>(*reinterpret_cast<const uint4*>(tb + size_t(v) * 16), t8);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) st += ex2(fmaf(t8[e], kLog2e, -ot));
+        }
       }
     }
     {
@@ -232,7 +253,7 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
       if constexpr (HAS_T) warp_lse_merge(m2, s2);
       if (lane == 0) ctrl->red[warp] = make_float4(m1, s1, m2, s2);
     }
-    named_bar(bar_id, NTW);
+    __syncthreads();
     if (warp == 0) {
       const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
       float m1 = r4.x, s1 = r4.y, m2 = r4.z, s2 = r4.w;
@@ -251,32 +272,41 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
       if constexpr (HAS_T) warp_lse_merge(n2, u2);
       if (lane == 0) ctrl->bcast = make_float4(n1 + log2f(u1), HAS_T ? n2 + log2f(u2) : 0.f, 0.f, 0.f);
     }
-    named_bar(bar_id, NTW);
+    __syncthreads();
     const float4 lse4 = ctrl->bcast;
     const float lz2 = lse4.x;  // lse_d in base-2 units
     const float lt2 = lse4.y;
     const float az = (mz == -INFINITY) ? 0.f : ex2(oz - lz2);  // p = e * az
     const float at = (!HAS_T || mt == -INFINITY) ? 0.f : ex2(ot - lt2);
 
-    // ---- pass 2: L1 and S; keeps p in xz and u = p*sign(p - q) in xt
+    // ---- pass 2: L1 and S.  q is rebuilt exactly as pass 1 formed it, so equal
+    // draft and teacher rows give p == q bit for bit.  xz <- u = p * sign(p - q)
+    // (an exact tie takes the sub-gradient +p).
     float L1 = 0.f, S = 0.f;
     if constexpr (HAS_T) {
       float l1p = 0.f, sp = 0.f;
 #pragma unroll
-      for (int e = 0; e < NE; ++e) {
-        const float p = __fmul_rn(xz[e], az);
-        const float q = __fmul_rn(xt[e], at);
-        const float d = __fsub_rn(p, q);
-        const float u = d != 0.f ? copysignf(p, d) : 0.f;
-        l1p += fabsf(d);
-        sp += u;
-        xz[e] = p;
-        xt[e] = u;
+      for (int i = 0; i < NV; ++i) {
+        const int v = tid + i * NT;
+        if (v < nvec) {
+          float t8[EPV];
+          unpack16<T>(*reinterpret_cast<const uint4*>(tb + size_t(v) * 16), t8);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) {
+            const float q = __fmul_rn(ex2(fmaf(t8[e], kLog2e, -ot)), at);
+            const float p = __fmul_rn(xz[i * EPV + e], az);
+            const float d = __fsub_rn(p, q);
+            const float u = copysignf(p, d);
+            l1p += fabsf(d);
+            sp += u;
+            xz[i * EPV + e] = u;
+          }
+        }
       }
       l1p = warp_sum(l1p);
       sp = warp_sum(sp);
       if (lane == 0) ctrl->red[warp] = make_float4(l1p, sp, 0.f, 0.f);
-      named_bar(bar_id, NTW);
+      __syncthreads();
       if (warp == 0) {
         const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float x = warp_sum(r4.x), y = warp_sum(r4.y);
@@ -313,18 +343,18 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
 
     // ---- pass 3: dlogits = p*(cce - cl1*S) + cl1*u, minus cce at the target id
     if (bwd) {
-      const float gw = g * a.ws.w[row];
+      const float gw = g * wr;
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
       const float k0 = cce - cl1 * S;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
-        const int v = tid + i * NTW;
+        const int v = tid + i * NT;
         if (v < nvec) {
           float o[EPV];
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
-            if constexpr (HAS_T) o[e] = fmaf(xt[i * EPV + e], cl1, xz[i * EPV + e] * k0);
+            if constexpr (HAS_T) o[e] = fmaf(xz[i * EPV + e], cl1, fabsf(xz[i * EPV + e]) * k0);
             else o[e] = (xz[i * EPV + e] * az) * cce;
           }
           if (v == tv) {
@@ -336,16 +366,19 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
         }
       }
     }
+    row = nrow;
+    tok = ntok;
+    wr = nw;
   }
 
   // ---- rows outside the supervision mask: dlogits = 0
   if (bwd && n_zero > 0) {
-    const int first = ((sid - n_sup) % NS + NS) % NS;
+    const int first = ((int(cid) - n_sup) % int(G) + int(G)) % int(G);
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-    for (int zi = first; zi < n_zero; zi += NS) {
-      const int64_t row = a.ws.zero_list[zi];
-      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
-      for (int v = tid; v < nvec; v += NTW) *reinterpret_cast<uint4*>(out + size_t(v) * 16) = z4;
+    for (int zi = first; zi < n_zero; zi += int(G)) {
+      const int64_t zr = a.ws.zero_list[zi];
+      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(zr) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
+      for (int v = tid; v < nvec; v += NT) *reinterpret_cast<uint4*>(out + size_t(v) * 16) = z4;
     }
   }
   // no CTA leaves while a peer may still signal or read its shared memory
@@ -356,6 +389,8 @@ __global__ void __launch_bounds__(WGS * NTW, 1) sweep_kernel(const SweepArgs a) 
 // ------------------------------------------------------------------ host side
 namespace {
 
+constexpr size_t kMaxSmem = 227 * 1024;
+
 struct LaunchCache {
   std::mutex mu;
   int dev = -1;
@@ -363,21 +398,25 @@ struct LaunchCache {
   int clusters = 0;
 };
 
-template <typename T, int CL, int WGS, int NTW, int NV, bool HAS_T>
+template <typename T, int CL>
+size_t smem_bytes(int64_t V, bool has_t) {
+  constexpr int EPV = VecTraits<T>::EPV;
+  const int64_t vvec = V / EPV;
+  const int64_t seg_vec = (vvec + CL - 1) / CL;
+  return size_t(has_t ? 3 : 2) * size_t(seg_vec) * 16 + sizeof(Ctrl);
+}
+
+template <typename T, int CL, int NT, int NV, bool HAS_T>
 cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   constexpr int EPV = VecTraits<T>::EPV;
-  constexpr int NTENS = HAS_T ? 2 : 1;
   SweepArgs a = a0;
   a.vvec = int32_t(a.V / EPV);
   a.seg_vec = (a.vvec + CL - 1) / CL;
-  const size_t per_buf = size_t(a.seg_vec) * 16 * NTENS;
-  const size_t ctrl = sizeof(WgCtrl) * WGS;
-  constexpr size_t kMaxSmem = 227 * 1024;
-  a.nbuf = (2 * per_buf * WGS + ctrl <= kMaxSmem) ? 2 : 1;
-  const size_t smem = a.nbuf * per_buf * WGS + ctrl;
+  a.nbuf = 2;
+  const size_t smem = smem_bytes<T, CL>(a.V, HAS_T);
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
-  auto kern = sweep_kernel<T, CL, WGS, NTW, NV, HAS_T>;
+  auto kern = sweep_kernel<T, CL, NT, NV, HAS_T>;
   static LaunchCache cache;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -399,7 +438,7 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
       }
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(CL, 1, 1);
-      q.blockDim = dim3(WGS * NTW, 1, 1);
+      q.blockDim = dim3(NT, 1, 1);
       q.dynamicSmemBytes = smem;
       q.attrs = at;
       q.numAttrs = 1;
@@ -419,7 +458,7 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(clusters * CL), 1, 1);
-  cfg.blockDim = dim3(WGS * NTW, 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = at;
@@ -427,17 +466,35 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// A build covers rows of up to CL * NTW * NV * (elements per vector) logits.
+// Builds, smallest first.  A build covers rows of up to CL * NT * NV * (elements per
+// vector) logits when its shared-memory buffers fit.
+struct Build {
+  int cl, nt, nv;
+};
 constexpr int kNumBuilds = 5;
-constexpr int64_t kBf16Cap[kNumBuilds] = {1 * 128 * 1 * 8, 2 * 256 * 2 * 8, 4 * 256 * 4 * 8,
-                                          8 * 256 * 5 * 8, 16 * 256 * 5 * 8};
-constexpr int64_t kF32Cap[kNumBuilds] = {1 * 128 * 2 * 4, 2 * 256 * 4 * 4, 4 * 256 * 8 * 4,
-                                         8 * 256 * 10 * 4, 16 * 256 * 10 * 4};
+constexpr Build kBf16Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {4, 512, 10}, {8, 512, 5}};
+constexpr Build kF32Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 8}, {8, 512, 10}, {16, 512, 5}};
 
-int pick_build(int dtype, int64_t V) {
-  const int64_t* cap = dtype == DSPARK_BF16 ? kBf16Cap : kF32Cap;
-  for (int i = 0; i < kNumBuilds; ++i)
-    if (cap[i] >= V) return i;
+template <typename T>
+size_t smem_for(int cl, int64_t V, bool has_t) {
+  switch (cl) {
+    case 1: return smem_bytes<T, 1>(V, has_t);
+    case 2: return smem_bytes<T, 2>(V, has_t);
+    case 4: return smem_bytes<T, 4>(V, has_t);
+    case 8: return smem_bytes<T, 8>(V, has_t);
+    default: return smem_bytes<T, 16>(V, has_t);
+  }
+}
+
+int pick_build(int dtype, int64_t V, bool has_t) {
+  const Build* b = dtype == DSPARK_BF16 ? kBf16Builds : kF32Builds;
+  const int epv = dtype == DSPARK_BF16 ? 8 : 4;
+  for (int i = 0; i < kNumBuilds; ++i) {
+    if (int64_t(b[i].cl) * b[i].nt * b[i].nv * epv < V) continue;
+    const size_t sm = dtype == DSPARK_BF16 ? smem_for<__nv_bfloat16>(b[i].cl, V, has_t)
+                                           : smem_for<float>(b[i].cl, V, has_t);
+    if (sm <= kMaxSmem) return i;
+  }
   return -1;
 }
 
@@ -445,19 +502,19 @@ template <typename T, bool HT>
 cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
   if constexpr (sizeof(T) == 2) {
     switch (i) {
-      case 0: return launch_cfg<T, 1, 2, 128, 1, HT>(a, s);
-      case 1: return launch_cfg<T, 2, 2, 256, 2, HT>(a, s);
-      case 2: return launch_cfg<T, 4, 2, 256, 4, HT>(a, s);
-      case 3: return launch_cfg<T, 8, 2, 256, 5, HT>(a, s);
-      case 4: return launch_cfg<T, 16, 2, 256, 5, HT>(a, s);
+      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<T, 4, 512, 4, HT>(a, s);
+      case 3: return launch_cfg<T, 4, 512, 10, HT>(a, s);
+      case 4: return launch_cfg<T, 8, 512, 5, HT>(a, s);
     }
   } else {
     switch (i) {
-      case 0: return launch_cfg<T, 1, 2, 128, 2, HT>(a, s);
-      case 1: return launch_cfg<T, 2, 2, 256, 4, HT>(a, s);
-      case 2: return launch_cfg<T, 4, 2, 256, 8, HT>(a, s);
-      case 3: return launch_cfg<T, 8, 2, 256, 10, HT>(a, s);
-      case 4: return launch_cfg<T, 16, 2, 256, 10, HT>(a, s);
+      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<T, 4, 512, 8, HT>(a, s);
+      case 3: return launch_cfg<T, 8, 512, 10, HT>(a, s);
+      case 4: return launch_cfg<T, 16, 512, 5, HT>(a, s);
     }
   }
   return cudaErrorInvalidValue;
@@ -465,10 +522,12 @@ cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool sweep_supported(int dtype, int64_t V, bool /*has_target*/) { return pick_build(dtype, V) >= 0; }
+bool sweep_supported(int dtype, int64_t V, bool has_target) {
+  return pick_build(dtype, V, has_target) >= 0;
+}
 
 cudaError_t launch_sweep(int dtype, bool has_target, const SweepArgs& a, cudaStream_t s) {
-  const int i = pick_build(dtype, a.V);
+  const int i = pick_build(dtype, a.V, has_target);
   if (i < 0) return cudaErrorInvalidValue;
   if (dtype == DSPARK_BF16)
     return has_target ? dispatch<__nv_bfloat16, true>(i, a, s) : dispatch<__nv_bfloat16, false>(i, a, s);
