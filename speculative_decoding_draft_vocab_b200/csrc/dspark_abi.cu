@@ -149,10 +149,7 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   if (e != cudaSuccess) return cuda_status(e);
 
   SweepArgs sa = sweep_args(prob, params, v, grads);
-  e = launch_sweep(int(prob->logits_dtype), sh.has_target_rows, sa, s);
-  if (e != cudaSuccess) return cuda_status(e);
-
-  FinalizeArgs fa{};
+  FinalizeArgs& fa = sa.fin;
   fa.B = prob->B; fa.N = prob->N; fa.K = prob->K;
   fa.block_keep = prob->block_keep;
   fa.confidence_logits = prob->confidence_logits;
@@ -170,7 +167,7 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   fa.accept_rows = out->accept_rows;
   fa.conf_rows = out->conf_rows;
   fa.dconf = grads ? grads->dconf : nullptr;
-  return cuda_status(launch_finalize(fa, s));
+  return cuda_status(launch_sweep(int(prob->logits_dtype), sh.has_target_rows, sa, s));
 }
 
 dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_params_t* params,

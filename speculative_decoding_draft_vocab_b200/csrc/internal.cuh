@@ -5,7 +5,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/dspark.h"
+#include "dspark.h"
 
 namespace dspark {
 
@@ -97,23 +97,6 @@ struct PrologueArgs {
   WsView ws;
 };
 
-struct SweepArgs {
-  const void* draft;
-  int64_t ld_d;
-  const void* target;        // null: CE only
-  int64_t ld_t;
-  void* dlogits;             // null: forward only
-  int64_t ld_g;
-  const int64_t* tids;
-  const float* grad_scale;   // null: 1
-  WsView ws;
-  int64_t V;
-  int32_t vvec;              // V / elements per 16-byte vector
-  int32_t seg_vec;           // vectors per CTA segment
-  int32_t nbuf;              // prefetch depth (1 or 2)
-  float ce_alpha, l1_alpha;
-};
-
 struct FinalizeArgs {
   int64_t B, N, K;
   const uint8_t* block_keep;
@@ -133,12 +116,31 @@ struct FinalizeArgs {
   float* dconf;
 };
 
+struct SweepArgs {
+  const void* draft;
+  int64_t ld_d;
+  const void* target;        // null: CE only
+  int64_t ld_t;
+  void* dlogits;             // null: forward only
+  int64_t ld_g;
+  const int64_t* tids;
+  const float* grad_scale;   // null: 1
+  WsView ws;
+  int64_t V;
+  int32_t vvec;              // V / elements per 16-byte vector
+  int32_t seg_vec;           // vectors per CTA segment
+  int32_t nbuf;              // prefetch depth (1 or 2)
+  float ce_alpha, l1_alpha;
+  FinalizeArgs fin;          // the per-row epilogue the last CTA runs
+};
+
+
+
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s);
 // Sweep config chosen for (dtype, V); returns false if V exceeds every build.
 bool sweep_supported(int dtype, int64_t V, bool has_target);
 cudaError_t launch_sweep(int dtype, bool has_target, const SweepArgs& a, cudaStream_t s);
-cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
                               const uint8_t* eval_mask, const uint8_t* block_keep,
                               float* accept_pair, float* tau_pair, float* accept_rows,

@@ -14,6 +14,8 @@ namespace dspark {
 constexpr int kPrologueThreads = 1024;
 
 __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const PrologueArgs a) {
+  // the sweep may be scheduled now; it waits for this grid before reading anything
+  asm volatile("griddepcontrol.launch_dependents;");
   const int tid = threadIdx.x;
   const int64_t nblk = a.B * a.N;
   const int64_t R = nblk * a.K;
@@ -22,28 +24,27 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const Prolog
     hdr->status = 0;
     hdr->done = 0;
   }
-  __syncthreads();
 
-  // ---- masks and weights, one thread per block of K positions
+  // ---- masks and weights, one thread per row (the prefix is re-scanned per row)
   uint32_t flags = 0;
-  for (int64_t blk = tid; blk < nblk; blk += kPrologueThreads) {
+  for (int64_t r = tid; r < R; r += kPrologueThreads) {
+    const int64_t blk = r / a.K, k = r - blk * a.K;
+    // independent loads (no early exit) so they are in flight together
     bool run = a.block_keep == nullptr || a.block_keep[blk] != 0;
-    for (int64_t k = 0; k < a.K; ++k) {
-      const int64_t r = blk * a.K + k;
-      run = run && a.eval_mask[r] != 0;
-      bool mm = run;
-      if (mm) {
-        const int64_t t = a.target_ids[r];
-        if (t < 0 || t >= a.V) { flags |= kFlagIdOutOfRange; mm = false; }
-        if (a.prev_ids != nullptr && a.valid[r] != 0) {
-          const int64_t pv = a.prev_ids[r];
-          if (pv < 0 || pv >= a.Vt) { flags |= kFlagIdOutOfRange; mm = false; }
-        }
+    for (int64_t j = 0; j <= k; ++j) run &= a.eval_mask[blk * a.K + j] != 0;
+    bool mm = run;
+    if (mm) {
+      const int64_t t = a.target_ids[r];
+      if (t < 0 || t >= a.V) { flags |= kFlagIdOutOfRange; mm = false; }
+      if (a.prev_ids != nullptr && a.valid[r] != 0) {
+        const int64_t pv = a.prev_ids[r];
+        if (pv < 0 || pv >= a.Vt) { flags |= kFlagIdOutOfRange; mm = false; }
       }
-      a.ws.m[r] = mm ? 1 : 0;
-      a.ws.w[r] = !mm ? 0.f : (a.gamma_enabled ? expf(-float(k) / a.gamma) : 1.f);
     }
+    a.ws.m[r] = mm ? 1 : 0;
+    a.ws.w[r] = !mm ? 0.f : (a.gamma_enabled ? expf(-float(k) / a.gamma) : 1.f);
   }
+  __syncthreads();  // status cleared before any flag is raised
   if (flags) atomicOr(&hdr->status, flags);
   __syncthreads();
 

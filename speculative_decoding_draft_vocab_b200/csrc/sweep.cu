@@ -20,6 +20,7 @@
 #include <algorithm>
 #include <mutex>
 
+#include "finalize.cuh"
 #include "internal.cuh"
 #include "ptx.cuh"
 
@@ -89,7 +90,8 @@ struct Ctrl {
   float4 red[32];         // per-warp partials
   float4 bcast;           // row logsumexps (base 2)
   float ztid;             // raw draft logit at the target id (owner only)
-  float pad[3];
+  int last;               // this CTA finished last and writes the report
+  float pad[2];
 };
 
 // One cluster of CL CTAs owns one supervised row at a time; CTA `rank` owns the
@@ -122,13 +124,9 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const int v0 = int(rank) * a.seg_vec;
   const int nvec = max(0, min(a.seg_vec, a.vvec - v0));
   const uint32_t bytes = uint32_t(nvec) * 16u;
-  const int n_sup = hdr->n_sup;
-  const int n_zero = hdr->n_zero;
-  const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
   const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
   const uint8_t* target = static_cast<const uint8_t*>(a.target);
   const bool bwd = a.dlogits != nullptr;
-  const float g = a.grad_scale ? *a.grad_scale : 1.f;
 
   const uint32_t bar_d0 = smem_u32(&ctrl->mbar_data[0]);
   const uint32_t bar_d1 = smem_u32(&ctrl->mbar_data[1]);
@@ -161,6 +159,26 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   // every CTA's barriers exist before any peer signals them
   __syncthreads();
   cluster_sync();
+  // the mask prologue has finished and its writes are visible past this point
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int n_sup = hdr->n_sup;
+  const int n_zero = hdr->n_zero;
+  const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
+  const float g = a.grad_scale ? *a.grad_scale : 1.f;
+  // this cluster's share of zero rows, written a slice after each supervised row
+  const int zfirst = ((int(cid) - n_sup) % int(G) + int(G)) % int(G);
+  const int my_z = (bwd && zfirst < n_zero) ? (n_zero - 1 - zfirst) / int(G) + 1 : 0;
+  const int ztot = my_z * nvec;
+  const int zslice = my_n > 0 ? (ztot + my_n - 1) / my_n : ztot;
+  auto write_zeros = [&](int q0, int q1) {
+    for (int q = q0 + tid; q < q1; q += NT) {
+      const int rk = q / nvec;
+      const int v = q - rk * nvec;
+      const int64_t zr = a.ws.zero_list[zfirst + size_t(rk) * G];
+      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.dlogits) +
+                                (size_t(zr) * a.ld_g + size_t(v0 + v) * EPV) * sizeof(T)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
   if (tid == 0) {
     if (my_n > 0) issue(0);
     if (!HAS_T && my_n > 1) issue(1);
@@ -179,6 +197,9 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     const uint8_t* zb = zbuf(j);
     const uint8_t* tb = tbuf(j);
 
+    // a slice of the zero rows while this row's segment lands (nothing of the row
+    // is live in registers yet)
+    write_zeros(j * zslice, min(ztot, (j + 1) * zslice));
     if (!mbar_wait_bounded((j & 1) ? bar_d1 : bar_d0, phase) && tid == 0) flag_timeout();
 
     // ---- draft segment -> registers
@@ -371,19 +392,23 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     wr = nw;
   }
 
-  // ---- rows outside the supervision mask: dlogits = 0
-  if (bwd && n_zero > 0) {
-    const int first = ((int(cid) - n_sup) % int(G) + int(G)) % int(G);
-    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-    for (int zi = first; zi < n_zero; zi += int(G)) {
-      const int64_t zr = a.ws.zero_list[zi];
-      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(zr) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
-      for (int v = tid; v < nvec; v += NT) *reinterpret_cast<uint4*>(out + size_t(v) * 16) = z4;
-    }
-  }
+  // ---- what is left of this cluster's zero rows (all of them if it had no row)
+  write_zeros(my_n * zslice, ztot);
   // no CTA leaves while a peer may still signal or read its shared memory
   __syncthreads();
   cluster_sync();
+
+  // ---- the last CTA to finish writes the per-row epilogue and the report
+  if (tid == 0) {
+    __threadfence();
+    ctrl->last = atomicAdd(&hdr->done, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (ctrl->last) {
+    __threadfence();
+    finalize_rows(a.fin, reinterpret_cast<double*>(smem));
+    if (tid == 0) hdr->done = 0;
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -413,7 +438,8 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   a.vvec = int32_t(a.V / EPV);
   a.seg_vec = (a.vvec + CL - 1) / CL;
   a.nbuf = 2;
-  const size_t smem = smem_bytes<T, CL>(a.V, HAS_T);
+  // at least the report's reduction scratch (reused at the end)
+  const size_t smem = std::max<size_t>(smem_bytes<T, CL>(a.V, HAS_T), size_t(NT / 32) * kNAcc * sizeof(double));
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
   auto kern = sweep_kernel<T, CL, NT, NV, HAS_T>;
@@ -456,13 +482,19 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
     }
     clusters = cache.clusters;
   }
+  // programmatic dependent launch: the grid is scheduled while the mask prologue
+  // runs and waits for it (griddepcontrol.wait) before reading its results
+  cudaLaunchAttribute at2[2];
+  at2[0] = at[0];
+  at2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at2[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(clusters * CL), 1, 1);
   cfg.blockDim = dim3(NT, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.attrs = at2;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 

@@ -59,15 +59,19 @@ def test_gamma_none_and_grad_scale():
     _run_and_compare(inp)
 
 
-def test_identical_rows_give_exact_zero_l1():
-    """draft == teacher: L1 = 0 exactly, accept = 1, tau = K + 1 on full blocks."""
+def test_identical_rows_give_zero_l1():
+    """draft == teacher: L1 = 0 (the oracle gives exactly 0; the kernel forms the
+    draft and teacher exponentials at different program points, which agree to the
+    approximation bound of ex2 rather than bit for bit), accept = 1, tau = K + 1."""
     inp = make_inputs("recipe", device="cuda", B=1, N=3, K=7, V=16384, prefix=(7, 7), seed=6)
     inp.target_logits = inp.draft_logits.clone()
     call, ref, _ = _run_and_compare(inp)
-    l1 = call.out.l1_rows.cpu()
-    assert bool((l1 == 0).all())
-    assert bool((call.out.accept_rows.cpu() == 1).all())
-    assert call.out.report[5].tolist() == [3.0 * 8, 3.0]
+    assert np.all(ref["l1"] == 0.0)
+    l1 = call.out.l1_rows.cpu().numpy()
+    assert np.all(np.abs(l1) <= 1e-6)
+    assert np.allclose(call.out.accept_rows.cpu().numpy(), 1.0, atol=1e-6)
+    tau = call.out.report[5].tolist()
+    assert tau[1] == 3.0 and abs(tau[0] - 3.0 * 8) <= 1e-4 * 24
 
 
 def test_disjoint_rows_l1_two():
