@@ -194,6 +194,31 @@ DSPARK_API dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, co
                                   float* accept_pair, float* tau_pair, float* accept_rows,
                                   dspark_stream_t stream);
 
+/*
+ * dspark_loss_fwd without a caller workspace (no counterpart on the source pages; it is
+ * a service of this library).  For callers that cannot allocate device memory or pass
+ * a workspace, e.g. an operator plugin whose host framework owns all device memory, or
+ * a runtime that forbids cudaMalloc/cudaFree while serving because they synchronise the
+ * device: the workspace is a fixed __device__ array inside this library, 368,896 bytes,
+ * held on every GPU that loads the library until the process exits.  Same problem,
+ * params, outputs and gradients as dspark_loss_fwd; nothing is allocated.
+ *  - Serves micro-batches of at most 8192 rows (B*N*K); larger ones return
+ *    DSPARK_ERR_WORKSPACE before anything is enqueued.
+ *  - The first call on a device looks the array's device address up (once per device,
+ *    with that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents behind; the
+ *    next call clears what must start at zero.  Calls that overlap on the GPU (other
+ *    streams, other threads) race on the array: serialise them.
+ *  - Device-side error flags land in the shared array and are not reported back (there
+ *    is no workspace pointer to pass to dspark_check_status); rows with out-of-range ids
+ *    are still skipped.
+ */
+DSPARK_API dspark_status_t dspark_loss_fwd_noalloc(const dspark_problem_t* prob,
+                                                   const dspark_params_t* params,
+                                                   const dspark_fwd_out_t* out,
+                                                   const dspark_grads_t* grads,
+                                                   dspark_stream_t stream);
+
 /* Synchronises `stream` and returns the first device-side error recorded in `ws`
  * by the last call that used it (DSPARK_OK if none). */
 DSPARK_API dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream);

@@ -93,6 +93,9 @@ lib.dspark_loss_fwd.restype = ctypes.c_int
 lib.dspark_loss_bwd.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_grads_t),
                                 c_vp, ctypes.c_size_t, c_vp]
 lib.dspark_loss_bwd.restype = ctypes.c_int
+lib.dspark_loss_fwd_noalloc.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_fwd_out_t),
+                                        P(dspark_grads_t), c_vp]
+lib.dspark_loss_fwd_noalloc.restype = ctypes.c_int
 lib.dspark_acceptance.argtypes = [c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
 lib.dspark_acceptance.restype = ctypes.c_int
 lib.dspark_check_status.argtypes = [c_vp, c_vp]
@@ -104,6 +107,9 @@ lib.dspark_status_string.restype = ctypes.c_char_p
 dspark_workspace_size = lib.dspark_workspace_size
 dspark_loss_fwd = lib.dspark_loss_fwd
 dspark_loss_bwd = lib.dspark_loss_bwd
+dspark_loss_fwd_noalloc = lib.dspark_loss_fwd_noalloc
+# Rows (B*N*K) the fixed scratch of dspark_loss_fwd_noalloc serves.
+NOALLOC_MAX_ROWS = 8192
 dspark_acceptance = lib.dspark_acceptance
 dspark_check_status = lib.dspark_check_status
 dspark_status_string = lib.dspark_status_string

@@ -50,22 +50,27 @@ struct WsView {
   size_t bytes;        // total bytes used
 };
 
-inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsOffsets {
   size_t hdr, m, w, sup, zero, stats, bytes;
 };
 
-inline WsOffsets ws_offsets(int64_t R) {
+constexpr WsOffsets ws_offsets(int64_t R) {
   WsOffsets o{};
   size_t off = 0;
-  auto take = [&](size_t n) { size_t at = off; off = align256(off + n); return at; };
-  o.hdr = take(sizeof(WsHeader));
-  o.m = take(size_t(R));
-  o.w = take(sizeof(float) * R);
-  o.sup = take(sizeof(int32_t) * R);
-  o.zero = take(sizeof(int32_t) * R);
-  o.stats = take(sizeof(float) * kStride * R);
+  o.hdr = off;
+  off = align256(off + sizeof(WsHeader));
+  o.m = off;
+  off = align256(off + size_t(R));
+  o.w = off;
+  off = align256(off + sizeof(float) * size_t(R));
+  o.sup = off;
+  off = align256(off + sizeof(int32_t) * size_t(R));
+  o.zero = off;
+  off = align256(off + sizeof(int32_t) * size_t(R));
+  o.stats = off;
+  off = align256(off + sizeof(float) * kStride * size_t(R));
   o.bytes = off;
   return o;
 }
