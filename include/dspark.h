@@ -108,14 +108,18 @@ typedef struct {
   const void* target_hidden;   /* bf16 [R, target_hidden_size], already final-normed    */
   const void* lm_head;         /* bf16 [V, target_hidden_size]                          */
   int64_t target_hidden_size;
-  /* Markov head (all NULL / 0 when absent) */
+  /* Markov head (all NULL / 0 when absent).  Needs bf16 logits (the backward
+   * contracts the bf16 dlogits on the tensor cores), markov_rank a multiple of 8 and
+   * 16-byte aligned weights; otherwise DSPARK_ERR_UNSUPPORTED / DSPARK_ERR_ALIGNMENT. */
   const int64_t* prev_ids;     /* [R] previous token, in [0, target_vocab)              */
   const uint8_t* valid;        /* [R] nonzero = valid slot (also used by the conf head) */
   int64_t target_vocab;
   const void* markov_w1;       /* bf16 [target_vocab, markov_rank]                      */
   const void* markov_w2;       /* bf16 [V, markov_rank]                                 */
   int64_t markov_rank;
-  /* confidence head (NULL when absent; exclusive with confidence_logits) */
+  /* confidence head (NULL when absent; exclusive with confidence_logits).  Needs
+   * `valid`, hidden_size a multiple of 8 and 16-byte aligned draft_hidden / conf_w;
+   * conf_with_markov needs the Markov head. */
   const void* draft_hidden;    /* bf16 [R, hidden_size]                                 */
   int64_t hidden_size;
   const void* conf_w;          /* bf16 [hidden_size (+ markov_rank)]: proj.weight       */
@@ -159,7 +163,10 @@ typedef struct {
 } dspark_grads_t;
 
 /* Bytes of device workspace dspark_loss_fwd / dspark_loss_bwd need for `prob`
- * (0 on an invalid problem).  Independent of the pointers' values. */
+ * (0 on an invalid problem).  Depends on the sizes and on which optional parts are
+ * present (non-NULL), not on the addresses.  With the Markov head it includes the
+ * corrected rows, 4*V bytes per row (the Markov head's corrected logits are kept in
+ * FP32 between the forward and the backward). */
 DSPARK_API size_t dspark_workspace_size(const dspark_problem_t* prob);
 
 /*
@@ -175,11 +182,13 @@ DSPARK_API dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const d
 
 /*
  * Backward alone, after a dspark_loss_fwd(..., grads = NULL) on the same problem,
- * params and workspace: one more pass over the logits, recomputing the probabilities
- * from the per-row statistics saved in `ws`.
+ * params and workspace: one more pass over the logits (the corrected rows the forward
+ * left in `ws` when the Markov head is on), recomputing the probabilities from the
+ * per-row statistics saved in `ws`.  The statistics are kept; the backward writes its
+ * own scratch (dL/dc per row, the split partials of dL/de) into `ws`.
  */
 DSPARK_API dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_params_t* params,
-                                const dspark_grads_t* grads, const void* ws, size_t ws_bytes,
+                                const dspark_grads_t* grads, void* ws, size_t ws_bytes,
                                 dspark_stream_t stream);
 
 /*
@@ -199,11 +208,12 @@ DSPARK_API dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, co
  * a service of this library).  For callers that cannot allocate device memory or pass
  * a workspace, e.g. an operator plugin whose host framework owns all device memory, or
  * a runtime that forbids cudaMalloc/cudaFree while serving because they synchronise the
- * device: the workspace is a fixed __device__ array inside this library, 368,896 bytes,
+ * device: the workspace is a fixed __device__ array inside this library, 401,664 bytes,
  * held on every GPU that loads the library until the process exits.  Same problem,
  * params, outputs and gradients as dspark_loss_fwd; nothing is allocated.
- *  - Serves micro-batches of at most 8192 rows (B*N*K); larger ones return
- *    DSPARK_ERR_WORKSPACE before anything is enqueued.
+ *  - Serves micro-batches of at most 8192 rows (B*N*K) without the Markov head (whose
+ *    corrected rows need 4*V bytes per row); others return DSPARK_ERR_WORKSPACE before
+ *    anything is enqueued.
  *  - The first call on a device looks the array's device address up (once per device,
  *    with that device current); make that first call before any stream capture.
  *  - Every call on a device shares the one array and leaves its contents behind; the

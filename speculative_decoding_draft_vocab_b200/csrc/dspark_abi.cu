@@ -25,6 +25,22 @@ struct Shape {
   bool has_conf_head;
 };
 
+inline bool markov_present(const dspark_problem_t* p) {
+  return p->markov_w2 != nullptr || p->markov_w1 != nullptr || p->prev_ids != nullptr;
+}
+
+inline WsDims ws_dims(const dspark_problem_t* p) {
+  WsDims d{};
+  d.R = p->B * p->N * p->K;
+  d.markov = markov_present(p);
+  if (d.markov) {
+    d.V = p->V;
+    d.rank = p->markov_rank;
+    d.splits = heads_splits(d.R, p->V);
+  }
+  return d;
+}
+
 dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* prm, Shape* sh) {
   if (p == nullptr) return DSPARK_ERR_INVALID_ARG;
   if (p->B <= 0 || p->N <= 0 || p->K <= 0 || p->V <= 0) return DSPARK_ERR_INVALID_ARG;
@@ -41,7 +57,7 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
   s.has_target_rows = p->target_logits != nullptr;
   s.has_lm_head = p->lm_head != nullptr || p->target_hidden != nullptr;
   s.has_teacher = s.has_target_rows || s.has_lm_head;
-  s.has_markov = p->markov_w2 != nullptr || p->markov_w1 != nullptr || p->prev_ids != nullptr;
+  s.has_markov = markov_present(p);
   s.has_conf_given = p->confidence_logits != nullptr;
   s.has_conf_head = p->conf_w != nullptr || p->draft_hidden != nullptr;
   if (s.has_target_rows) {
@@ -56,10 +72,22 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
     if (prm->gamma_enabled && !(prm->gamma > 0.f)) return DSPARK_ERR_INVALID_ARG;
     if (prm->invalid_row_mode != 0 && prm->invalid_row_mode != 1) return DSPARK_ERR_INVALID_ARG;
   }
-  // The Markov head, the confidence head and the teacher-from-hidden path run in
-  // their own kernels; this build accepts them only once those are present.
-  if (s.has_markov || s.has_conf_head || s.has_lm_head) return DSPARK_ERR_UNSUPPORTED;
-  if (!sweep_supported(int(p->logits_dtype), p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
+  // The teacher-from-hidden path is not part of this build.
+  if (s.has_lm_head) return DSPARK_ERR_UNSUPPORTED;
+  if (s.has_markov) {
+    if (!p->markov_w1 || !p->markov_w2 || !p->prev_ids || !p->valid) return DSPARK_ERR_INVALID_ARG;
+    if (p->markov_rank <= 0 || p->target_vocab <= 0) return DSPARK_ERR_INVALID_ARG;
+    // the backward contracts the bf16 dlogits on the tensor cores
+    if (p->logits_dtype != DSPARK_BF16) return DSPARK_ERR_UNSUPPORTED;
+    if (p->markov_rank % 8 || !aligned16(p->markov_w1) || !aligned16(p->markov_w2)) return DSPARK_ERR_ALIGNMENT;
+  }
+  if (s.has_conf_head) {
+    if (!p->conf_w || !p->conf_b || !p->draft_hidden || !p->valid) return DSPARK_ERR_INVALID_ARG;
+    if (p->hidden_size <= 0) return DSPARK_ERR_INVALID_ARG;
+    if (p->conf_with_markov && !s.has_markov) return DSPARK_ERR_INVALID_ARG;
+    if (p->hidden_size % 8 || !aligned16(p->conf_w) || !aligned16(p->draft_hidden)) return DSPARK_ERR_ALIGNMENT;
+  }
+  if (!sweep_supported(int(p->logits_dtype), s.has_markov, p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
   *sh = s;
   return DSPARK_OK;
 }
@@ -69,7 +97,7 @@ inline dspark_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DS
 dspark_status_t check_ws(const dspark_problem_t* p, const void* ws, size_t ws_bytes) {
   if (ws == nullptr) return DSPARK_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DSPARK_ERR_ALIGNMENT;
-  if (ws_bytes < ws_offsets(p->B * p->N * p->K).bytes) return DSPARK_ERR_WORKSPACE;
+  if (ws_bytes < ws_offsets(ws_dims(p)).bytes) return DSPARK_ERR_WORKSPACE;
   return DSPARK_OK;
 }
 
@@ -96,7 +124,47 @@ SweepArgs sweep_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
   a.V = p->V;
   a.ce_alpha = prm->ce_alpha;
   a.l1_alpha = p->target_logits ? prm->l1_alpha : 0.f;
+  if (markov_present(p)) {  // the sweep reads the corrected rows, compact by supervised position
+    a.draft = ws.z;
+    a.ld_d = p->V;
+    a.draft_compact = 1;
+    a.valid = p->valid;
+    a.invalid_zero = prm->invalid_row_mode == 0;
+  }
   return a;
+}
+
+HeadsArgs heads_args(const dspark_problem_t* p, const dspark_params_t* prm, const WsView& ws,
+                     const dspark_grads_t* g) {
+  HeadsArgs h{};
+  h.R = p->B * p->N * p->K;
+  h.V = p->V;
+  h.Vt = p->target_vocab;
+  h.rank = markov_present(p) ? p->markov_rank : 0;
+  h.H = p->conf_w ? p->hidden_size : 0;
+  h.base = static_cast<const uint16_t*>(p->draft_logits);
+  h.ld_base = p->draft_ld;
+  h.prev_ids = p->prev_ids;
+  h.valid = p->valid;
+  h.w1 = markov_present(p) ? static_cast<const uint16_t*>(p->markov_w1) : nullptr;
+  h.w2 = static_cast<const uint16_t*>(p->markov_w2);
+  h.hidden = static_cast<const uint16_t*>(p->draft_hidden);
+  h.conf_w = static_cast<const uint16_t*>(p->conf_w);
+  h.conf_b = p->conf_b;
+  h.conf_with_markov = p->conf_w && p->conf_with_markov ? 1 : 0;
+  h.invalid_row_mode = prm->invalid_row_mode;
+  if (g) {
+    h.dlogits = static_cast<const uint16_t*>(g->dlogits);
+    h.ld_g = g->dlogits_ld;
+    h.dw1 = g->dW1;
+    h.dw2 = g->dW2;
+    h.dconf_w = g->dconf_w;
+    h.dconf_b = g->dconf_b;
+    h.dhidden = static_cast<uint16_t*>(g->dhidden);
+    h.accumulate = g->accumulate ? 1 : 0;
+  }
+  h.ws = ws;
+  return h;
 }
 
 }  // namespace
@@ -120,7 +188,8 @@ const char* dspark_status_string(dspark_status_t s) {
 
 size_t dspark_workspace_size(const dspark_problem_t* prob) {
   if (prob == nullptr || prob->B <= 0 || prob->N <= 0 || prob->K <= 0) return 0;
-  return ws_offsets(prob->B * prob->N * prob->K).bytes;
+  if (markov_present(prob) && (prob->V <= 0 || prob->markov_rank <= 0)) return 0;
+  return ws_offsets(ws_dims(prob)).bytes;
 }
 
 dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_params_t* params,
@@ -133,20 +202,28 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
   if (grads && (st = check_grads(prob, grads)) != DSPARK_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const WsView v = ws_layout(ws, sh.R);
+  const WsView v = ws_layout(ws, ws_dims(prob));
 
   PrologueArgs pa{};
   pa.B = prob->B; pa.N = prob->N; pa.K = prob->K; pa.V = prob->V; pa.Vt = prob->target_vocab;
   pa.eval_mask = prob->eval_mask;
   pa.block_keep = prob->block_keep;
   pa.target_ids = prob->target_ids;
-  pa.prev_ids = nullptr;
+  pa.prev_ids = sh.has_markov ? prob->prev_ids : nullptr;
   pa.valid = prob->valid;
   pa.gamma = params->gamma;
   pa.gamma_enabled = params->gamma_enabled;
   pa.ws = v;
   cudaError_t e = launch_prologue(pa, s);
   if (e != cudaSuccess) return cuda_status(e);
+
+  const HeadsArgs ha = heads_args(prob, params, v, grads);
+  if (sh.has_markov || sh.has_conf_head) {
+    if ((e = launch_heads_prep(ha, s)) != cudaSuccess) return cuda_status(e);
+  }
+  if (sh.has_markov) {
+    if ((e = launch_markov_bias(ha, s)) != cudaSuccess) return cuda_status(e);
+  }
 
   SweepArgs sa = sweep_args(prob, params, v, grads);
   FinalizeArgs& fa = sa.fin;
@@ -167,11 +244,14 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   fa.accept_rows = out->accept_rows;
   fa.conf_rows = out->conf_rows;
   fa.dconf = grads ? grads->dconf : nullptr;
-  return cuda_status(launch_sweep(int(prob->logits_dtype), sh.has_target_rows, sa, s));
+  e = launch_sweep(int(prob->logits_dtype), sh.has_markov, sh.has_target_rows, sa, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (grads && (sh.has_markov || sh.has_conf_head)) e = launch_heads_bwd(ha, s);
+  return cuda_status(e);
 }
 
 dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_params_t* params,
-                                const dspark_grads_t* grads, const void* ws, size_t ws_bytes,
+                                const dspark_grads_t* grads, void* ws, size_t ws_bytes,
                                 dspark_stream_t stream) {
   if (params == nullptr) return DSPARK_ERR_INVALID_ARG;
   Shape sh{};
@@ -180,18 +260,19 @@ dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_param
   if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
   if ((st = check_grads(prob, grads)) != DSPARK_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const WsView v = ws_layout(const_cast<void*>(ws), sh.R);
+  const WsView v = ws_layout(ws, ws_dims(prob));
   SweepArgs sa = sweep_args(prob, params, v, grads);
-  cudaError_t e = launch_bwd_stream(int(prob->logits_dtype), sh.has_target_rows, sa, sh.R, s);
+  cudaError_t e = launch_bwd_stream(int(prob->logits_dtype), sh.has_markov, sh.has_target_rows, sa, sh.R, s);
   if (e != cudaSuccess) return cuda_status(e);
-  if (grads->dconf) {
-    if (!(sh.has_conf_given || sh.has_conf_head)) {
-      e = cudaMemsetAsync(grads->dconf, 0, sizeof(float) * sh.R, s);
-    } else {
-      e = launch_conf_grad(sh.R, prob->confidence_logits, params->conf_alpha, grads->grad_scale, v,
-                           grads->dconf, s);
-    }
+  if (sh.has_conf_given || sh.has_conf_head) {
+    // dL/dc for this call's grad_scale, also saved for the confidence head's backward
+    e = launch_conf_grad(sh.R, prob->confidence_logits, params->conf_alpha, grads->grad_scale, v,
+                         grads->dconf, s);
+  } else if (grads->dconf) {
+    e = cudaMemsetAsync(grads->dconf, 0, sizeof(float) * sh.R, s);
   }
+  if (e != cudaSuccess) return cuda_status(e);
+  if (sh.has_markov || sh.has_conf_head) e = launch_heads_bwd(heads_args(prob, params, v, grads), s);
   return cuda_status(e);
 }
 

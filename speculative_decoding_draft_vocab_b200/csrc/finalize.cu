@@ -60,14 +60,15 @@ __global__ void conf_grad_kernel(int64_t R, const float* confidence_logits, floa
   const double g = grad_scale ? double(*grad_scale) : 1.0;
   for (int64_t r = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; r < R;
        r += int64_t(gridDim.x) * blockDim.x) {
-    if (ws.m[r] == 0) {
-      dconf[r] = 0.f;
-      continue;
+    float dc = 0.f;
+    if (ws.m[r] != 0) {
+      const float* st = ws.stats + r * kStride;
+      const double c = confidence_logits ? confidence_logits[r] : st[kStConf];
+      const double y = clamp01(1.0 - 0.5 * double(st[kStL1]));
+      dc = float(g * double(ws.w[r]) * double(conf_alpha) * (1.0 / (1.0 + exp(-c)) - y));
     }
-    const float* st = ws.stats + r * kStride;
-    const double c = confidence_logits ? confidence_logits[r] : st[kStConf];
-    const double y = clamp01(1.0 - 0.5 * double(st[kStL1]));
-    dconf[r] = float(g * double(ws.w[r]) * double(conf_alpha) * (1.0 / (1.0 + exp(-c)) - y));
+    ws.stats[r * kStride + kStDC] = dc;  // the confidence head's backward reads it
+    if (dconf) dconf[r] = dc;
   }
 }
 

@@ -69,13 +69,15 @@ __device__ inline void finalize_rows(const FinalizeArgs& a, double* scratch) {
       if (a.ce_rows) a.ce_rows[r] = float(ce);
       if (a.l1_rows) a.l1_rows[r] = float(l1);
       if (a.accept_rows) a.accept_rows[r] = float(y);
-      if (a.dconf)
-        a.dconf[r] = a.has_conf ? float(g * w * double(a.conf_alpha) * (1.0 / (1.0 + exp(-c)) - y)) : 0.f;
+      const float dc = a.has_conf ? float(g * w * double(a.conf_alpha) * (1.0 / (1.0 + exp(-c)) - y)) : 0.f;
+      if (a.dconf) a.dconf[r] = dc;
+      a.ws.stats[r * kStride + kStDC] = dc;
     } else {
       if (a.ce_rows) a.ce_rows[r] = 0.f;
       if (a.l1_rows) a.l1_rows[r] = 0.f;
       if (a.accept_rows) a.accept_rows[r] = 0.f;
       if (a.dconf) a.dconf[r] = 0.f;
+      a.ws.stats[r * kStride + kStDC] = 0.f;
     }
     if (a.conf_rows) a.conf_rows[r] = float(c);
   }

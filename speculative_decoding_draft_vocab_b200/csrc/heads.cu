@@ -1,0 +1,242 @@
+// The two DSpark auxiliary heads (NeMo RL design doc "DSpark Auxiliary Heads"):
+//   Markov head:      z = base + markov_w2 . e,  e = markov_w1[prev]   (valid slots)
+//                     an invalid slot's corrected row is all zero (mode 0) or its base
+//                     row (mode 1); prev ids are in the target vocabulary
+//   confidence head:  c = proj . [h ; e] + bias on valid slots, 0 on invalid ones
+// and their backward:
+//   dE_r  = W2^T dz_r + dc_r proj_e,  dW2 = sum_r dz_r (x) e_r,  dW1[prev_r] += dE_r
+//   dproj = sum_r dc_r [h_r ; e_r],  dbias = sum_r dc_r,  dh_r = dc_r proj_h
+// (TorchSpec pull request #132, test list: the Markov bias is W2 applied to the W1 row
+// of the previous token).  The two contractions against the vocabulary (bias,
+// dE, dW2) run on the tcgen05 GEMM; the rest are small row kernels.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "internal.cuh"
+#include "tc_host.cuh"
+
+namespace dspark {
+
+namespace {
+
+__device__ __forceinline__ float bf(uint16_t v) { return __uint_as_float(uint32_t(v) << 16); }
+
+// ---- gather of the Markov embeddings and the confidence logits (one warp per row)
+__global__ void __launch_bounds__(256) heads_prep_kernel(const HeadsArgs a) {
+  const int warps = blockDim.x / 32;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = int64_t(blockIdx.x) * warps + threadIdx.x / 32; r < a.R; r += int64_t(gridDim.x) * warps) {
+    const bool sup = a.ws.m[r] != 0;
+    const bool valid = a.valid[r] != 0;
+    const int64_t pv = a.prev_ids ? a.prev_ids[r] : -1;
+    const bool has_e = a.w1 != nullptr && valid && pv >= 0 && pv < a.Vt;
+    float edot = 0.f;
+    if (a.w1 != nullptr) {
+      const uint16_t* src = a.w1 + size_t(has_e ? pv : 0) * a.rank;
+      uint16_t* dall = a.ws.eall + size_t(r) * a.rank;
+      const int si = a.ws.sup_index[r];
+      uint16_t* dsup = sup ? a.ws.esup + size_t(si) * a.rank : nullptr;
+      for (int j = lane * 8; j < a.rank; j += 256) {  // 16-byte pieces
+        uint4 q = has_e ? *reinterpret_cast<const uint4*>(src + j) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(dall + j) = (sup && has_e) ? q : make_uint4(0u, 0u, 0u, 0u);
+        if (dsup) *reinterpret_cast<uint4*>(dsup + j) = q;
+        if (a.conf_w != nullptr && a.conf_with_markov && has_e) {
+          const uint16_t* e = reinterpret_cast<const uint16_t*>(&q);
+          const uint16_t* pw = a.conf_w + a.H + j;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) edot = fmaf(bf(e[t]), bf(pw[t]), edot);
+        }
+      }
+    }
+    if (a.conf_w != nullptr) {
+      float hdot = 0.f;
+      if (valid) {
+        const uint16_t* h = a.hidden + size_t(r) * a.H;
+        for (int j = lane * 8; j < a.H; j += 256) {
+          const uint4 q = *reinterpret_cast<const uint4*>(h + j);
+          const uint4 w = *reinterpret_cast<const uint4*>(a.conf_w + j);
+          const uint16_t* hv = reinterpret_cast<const uint16_t*>(&q);
+          const uint16_t* wv = reinterpret_cast<const uint16_t*>(&w);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) hdot = fmaf(bf(hv[t]), bf(wv[t]), hdot);
+        }
+      }
+      float c = hdot + edot;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+      if (lane == 0) a.ws.stats[r * kStride + kStConf] = valid ? c + *a.conf_b : 0.f;
+    }
+  }
+}
+
+// ---- epilogue of the bias GEMM: corrected row z = base + E.W2^T (compact rows)
+struct BiasEpi {
+  const int32_t* sup_list;
+  const WsHeader* hdr;
+  const uint16_t* base;
+  int64_t ld_base;
+  const uint8_t* valid;
+  int invalid_row_mode;
+  float* z;
+  int64_t ldz;
+  int V;
+  __device__ void operator()(int m, int n, int /*split*/, const float* v) const {
+    if (m >= hdr->n_sup) return;
+    const int64_t row = sup_list[m];
+    const bool ok = valid[row] != 0;
+    const uint16_t* b = base + size_t(row) * ld_base;
+    float* out = z + size_t(m) * ldz;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = n + i;
+      if (c < V) out[c] = ok ? bf(b[c]) + v[i] : (invalid_row_mode == 0 ? 0.f : bf(b[c]));
+    }
+  }
+};
+
+// ---- epilogue of the dE GEMM: one partial per K split
+struct PartialEpi {
+  float* dep;
+  int R, rank;
+  __device__ void operator()(int m, int n, int split, const float* v) const {
+    if (m >= R) return;
+    float* out = dep + (size_t(split) * R + m) * rank;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (n + i < rank) out[n + i] = v[i];
+  }
+};
+
+// ---- epilogue of the dW2 GEMM
+struct WeightEpi {
+  float* dw2;
+  int V, rank, accumulate;
+  __device__ void operator()(int m, int n, int /*split*/, const float* v) const {
+    if (m >= V) return;
+    float* out = dw2 + size_t(m) * rank;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (n + i < rank) out[n + i] = accumulate ? out[n + i] + v[i] : v[i];
+  }
+};
+
+// ---- dE = sum of the split partials (+ dc proj_e), then dW1[prev] += dE
+__global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const int splits) {
+  const int64_t n = a.R * a.rank;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / a.rank, j = i - r * a.rank;
+    const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
+    float acc = 0.f;
+    if (live) {
+      for (int s = 0; s < splits; ++s) acc += a.ws.dep[(size_t(s) * a.R + r) * a.rank + j];
+      if (a.conf_w != nullptr && a.conf_with_markov)
+        acc += a.ws.stats[r * kStride + kStDC] * bf(a.conf_w[a.H + j]);
+      const int64_t pv = a.prev_ids[r];
+      if (a.dw1 != nullptr) atomicAdd(a.dw1 + size_t(pv) * a.rank + j, acc);
+    }
+    a.ws.de[i] = acc;
+  }
+}
+
+// ---- dproj = sum_r dc_r [h_r ; e_r] and dbias = sum_r dc_r (fixed row order)
+__global__ void __launch_bounds__(256) dproj_kernel(const HeadsArgs a) {
+  const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
+  const int64_t j = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  if (j < cols) {
+    float acc = 0.f;
+    for (int64_t r = 0; r < a.R; ++r) {
+      if (a.ws.m[r] == 0 || a.valid[r] == 0) continue;
+      const float dc = a.ws.stats[r * kStride + kStDC];
+      const float x = j < a.H ? bf(a.hidden[size_t(r) * a.H + j]) : bf(a.ws.eall[size_t(r) * a.rank + (j - a.H)]);
+      acc = fmaf(dc, x, acc);
+    }
+    a.dconf_w[j] = a.accumulate ? a.dconf_w[j] + acc : acc;
+  }
+  if (blockIdx.x == 0) {
+    __shared__ float part[8];
+    float acc = 0.f;
+    for (int64_t r = threadIdx.x; r < a.R; r += blockDim.x)
+      if (a.ws.m[r] != 0 && a.valid[r] != 0) acc += a.ws.stats[r * kStride + kStDC];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.f;
+      for (int i = 0; i < int(blockDim.x / 32); ++i) t += part[i];
+      if (a.dconf_b) *a.dconf_b = a.accumulate ? *a.dconf_b + t : t;
+    }
+  }
+}
+
+// ---- dh_r = dc_r proj_h on supervised valid rows, 0 elsewhere (bf16)
+__global__ void __launch_bounds__(256) dhidden_kernel(const HeadsArgs a) {
+  const int64_t n = a.R * a.H;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / a.H, j = i - r * a.H;
+    const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
+    const float v = live ? a.ws.stats[r * kStride + kStDC] * bf(a.conf_w[j]) : 0.f;
+    a.dhidden[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+}
+
+inline int grid_for(int64_t n, int per_block) {
+  const int64_t g = (n + per_block - 1) / per_block;
+  return int(std::max<int64_t>(1, std::min<int64_t>(g, 4096)));
+}
+
+}  // namespace
+
+cudaError_t launch_heads_prep(const HeadsArgs& a, cudaStream_t s) {
+  heads_prep_kernel<<<grid_for(a.R, 8), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (!tc::make_map(&ma, a.ws.esup, a.R, a.rank, a.rank, 64, 128)) return cudaErrorInvalidValue;
+  if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 256)) return cudaErrorInvalidValue;
+  BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.base, a.ld_base, a.valid, a.invalid_row_mode, a.ws.z, a.V, int(a.V)};
+  return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s);
+}
+
+cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  if (a.w1 != nullptr) {
+    const int splits = heads_splits(a.R, a.V);
+    // dE partials: A = dlogits [R][V] (K-major), B = W2 as [V][rank] (MN-major)
+    CUtensorMap ma, mb;
+    if (!tc::make_map(&ma, a.dlogits, a.R, a.V, a.ld_g, 64, 128)) return cudaErrorInvalidValue;
+    if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
+    PartialEpi pe{a.ws.dep, int(a.R), int(a.rank)};
+    e = tc::gemm<256, false, true, 4>(ma, mb, int(a.R), int(a.rank), int(a.V), splits, pe, &a.ws.hdr->status, s);
+    if (e != cudaSuccess) return e;
+    // dW2 = dlogits^T . E: A = dlogits as [R][V] (MN-major, M = vocabulary),
+    // B = E by row [R][rank] (MN-major)
+    if (a.dw2 != nullptr) {
+      CUtensorMap ma2, mb2;
+      if (!tc::make_map(&ma2, a.dlogits, a.R, a.V, a.ld_g, 64, 64)) return cudaErrorInvalidValue;
+      if (!tc::make_map(&mb2, a.ws.eall, a.R, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
+      WeightEpi we{a.dw2, int(a.V), int(a.rank), a.accumulate};
+      e = tc::gemm<256, true, true, 4>(ma2, mb2, int(a.V), int(a.rank), int(a.R), 1, we, &a.ws.hdr->status, s);
+      if (e != cudaSuccess) return e;
+    }
+    de_reduce_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, splits);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.conf_w != nullptr) {
+    const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
+    if (a.dconf_w != nullptr) {
+      dproj_kernel<<<int((cols + 255) / 256), 256, 0, s>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (a.dhidden != nullptr) {
+      dhidden_kernel<<<grid_for(a.R * a.H, 256), 256, 0, s>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+  return cudaSuccess;
+}
+
+}  // namespace dspark

@@ -24,6 +24,7 @@ enum : int {
   kStS = 4,      // sum_j p_j * sign(p_j - q_j)
   kStConf = 5,   // confidence logit c
   kStZT = 6,     // corrected draft logit at the target id
+  kStDC = 7,     // dL/dc of the confidence logit
   kStride = 8,
 };
 
@@ -46,37 +47,70 @@ struct WsView {
   float* w;            // [R] loss weight m * exp(-k/gamma)
   int32_t* sup_list;   // [R] supervised rows in row order
   int32_t* zero_list;  // [R] unsupervised rows in row order
+  int32_t* sup_index;  // [R] position of a row in sup_list, -1 if unsupervised
   float* stats;        // [R][kStride]
+  // Markov head (present when the problem has it)
+  float* z;            // [R][V] corrected draft rows, compact by supervised position
+  uint16_t* esup;      // [R][rank] bf16 Markov embeddings, compact (0 on invalid slots)
+  uint16_t* eall;      // [R][rank] bf16 Markov embeddings by row (0 unless supervised+valid)
+  float* dep;          // [splits][R][rank] split-K partials of dE
+  float* de;           // [R][rank] dL/de
   size_t bytes;        // total bytes used
 };
 
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct WsOffsets {
-  size_t hdr, m, w, sup, zero, stats, bytes;
+// What a problem needs besides the per-row arrays.
+struct WsDims {
+  int64_t R = 0, V = 0, rank = 0, splits = 0;
+  bool markov = false;
 };
 
-constexpr WsOffsets ws_offsets(int64_t R) {
+struct WsOffsets {
+  size_t hdr, m, w, sup, zero, sidx, stats, z, esup, eall, dep, de, bytes;
+};
+
+constexpr WsOffsets ws_offsets(const WsDims& d) {
   WsOffsets o{};
   size_t off = 0;
+  const size_t R = size_t(d.R);
   o.hdr = off;
   off = align256(off + sizeof(WsHeader));
   o.m = off;
-  off = align256(off + size_t(R));
+  off = align256(off + R);
   o.w = off;
-  off = align256(off + sizeof(float) * size_t(R));
+  off = align256(off + sizeof(float) * R);
   o.sup = off;
-  off = align256(off + sizeof(int32_t) * size_t(R));
+  off = align256(off + sizeof(int32_t) * R);
   o.zero = off;
-  off = align256(off + sizeof(int32_t) * size_t(R));
+  off = align256(off + sizeof(int32_t) * R);
+  o.sidx = off;
+  off = align256(off + sizeof(int32_t) * R);
   o.stats = off;
-  off = align256(off + sizeof(float) * kStride * size_t(R));
+  off = align256(off + sizeof(float) * kStride * R);
+  const size_t zr = d.markov ? R : 0, er = d.markov ? R * size_t(d.rank) : 0;
+  o.z = off;
+  off = align256(off + sizeof(float) * zr * size_t(d.V));
+  o.esup = off;
+  off = align256(off + 2 * er);
+  o.eall = off;
+  off = align256(off + 2 * er);
+  o.dep = off;
+  off = align256(off + sizeof(float) * er * size_t(d.markov ? d.splits : 0));
+  o.de = off;
+  off = align256(off + sizeof(float) * er);
   o.bytes = off;
   return o;
 }
 
-inline WsView ws_layout(void* base, int64_t R) {
-  const WsOffsets o = ws_offsets(R);
+constexpr WsOffsets ws_offsets(int64_t R) {
+  WsDims d{};
+  d.R = R;
+  return ws_offsets(d);
+}
+
+inline WsView ws_layout(void* base, const WsDims& d) {
+  const WsOffsets o = ws_offsets(d);
   uint8_t* b = static_cast<uint8_t*>(base);
   WsView v{};
   v.hdr = reinterpret_cast<WsHeader*>(b + o.hdr);
@@ -84,9 +118,21 @@ inline WsView ws_layout(void* base, int64_t R) {
   v.w = reinterpret_cast<float*>(b + o.w);
   v.sup_list = reinterpret_cast<int32_t*>(b + o.sup);
   v.zero_list = reinterpret_cast<int32_t*>(b + o.zero);
+  v.sup_index = reinterpret_cast<int32_t*>(b + o.sidx);
   v.stats = reinterpret_cast<float*>(b + o.stats);
+  v.z = d.markov ? reinterpret_cast<float*>(b + o.z) : nullptr;
+  v.esup = d.markov ? reinterpret_cast<uint16_t*>(b + o.esup) : nullptr;
+  v.eall = d.markov ? reinterpret_cast<uint16_t*>(b + o.eall) : nullptr;
+  v.dep = d.markov ? reinterpret_cast<float*>(b + o.dep) : nullptr;
+  v.de = d.markov ? reinterpret_cast<float*>(b + o.de) : nullptr;
   v.bytes = o.bytes;
   return v;
+}
+
+inline WsView ws_layout(void* base, int64_t R) {
+  WsDims d{};
+  d.R = R;
+  return ws_layout(base, d);
 }
 
 // ------------------------------------------------------------- kernel arguments
@@ -135,25 +181,70 @@ struct SweepArgs {
   int32_t vvec;              // V / elements per 16-byte vector
   int32_t seg_vec;           // vectors per CTA segment
   int32_t nbuf;              // prefetch depth (1 or 2)
+  int32_t draft_compact;     // draft row of the i-th supervised row is i (corrected rows)
+  const uint8_t* valid;      // Markov valid-slot mask (with invalid_zero)
+  int32_t invalid_zero;      // invalid slots get zero dlogits (all-zero corrected row)
   float ce_alpha, l1_alpha;
   FinalizeArgs fin;          // the per-row epilogue the last CTA runs
 };
 
 
 
+// Markov head and confidence head (inputs, weight gradients and workspace).
+struct HeadsArgs {
+  int64_t R, V, Vt, rank, H;
+  const uint16_t* base;      // bf16 [R][ld_base] base draft logits
+  int64_t ld_base;
+  const int64_t* prev_ids;
+  const uint8_t* valid;
+  const uint16_t* w1;        // bf16 [Vt][rank], null without the Markov head
+  const uint16_t* w2;        // bf16 [V][rank]
+  const uint16_t* hidden;    // bf16 [R][H], null without the confidence head
+  const uint16_t* conf_w;    // bf16 [H (+ rank)]
+  const float* conf_b;
+  int32_t conf_with_markov;
+  int32_t invalid_row_mode;
+  const uint16_t* dlogits;   // bf16 [R][ld_g] (backward)
+  int64_t ld_g;
+  float* dw1;
+  float* dw2;
+  float* dconf_w;
+  float* dconf_b;
+  uint16_t* dhidden;         // bf16 [R][H]
+  int32_t accumulate;
+  WsView ws;
+};
+
+// K splits of the dE contraction (a fixed count for a given shape, so the workspace
+// size does not depend on the device).
+constexpr int kHeadsSlots = 148;
+constexpr int heads_splits(int64_t R, int64_t V) {
+  const int64_t m_tiles = (R + 127) / 128, kchunks = (V + 63) / 64;
+  const int64_t s = kHeadsSlots / m_tiles;
+  return int(s < 1 ? 1 : (s > kchunks ? kchunks : s));
+}
+
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s);
-// Sweep config chosen for (dtype, V); returns false if V exceeds every build.
-bool sweep_supported(int dtype, int64_t V, bool has_target);
-cudaError_t launch_sweep(int dtype, bool has_target, const SweepArgs& a, cudaStream_t s);
+// zf32: FP32 corrected draft rows (compact) with bf16 teacher and dlogits.  Returns
+// false if V exceeds every build of that combination.
+bool sweep_supported(int dtype, bool zf32, int64_t V, bool has_target);
+cudaError_t launch_sweep(int dtype, bool zf32, bool has_target, const SweepArgs& a, cudaStream_t s);
 cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
                               const uint8_t* eval_mask, const uint8_t* block_keep,
                               float* accept_pair, float* tau_pair, float* accept_rows,
                               cudaStream_t s);
+// dconf (if non-null) and the saved dL/dc of every row, for the given grad_scale
 cudaError_t launch_conf_grad(int64_t R, const float* confidence_logits, float conf_alpha,
                              const float* grad_scale, const WsView& ws, float* dconf,
                              cudaStream_t s);
-cudaError_t launch_bwd_stream(int dtype, bool has_target, const SweepArgs& a, int64_t R,
+cudaError_t launch_bwd_stream(int dtype, bool zf32, bool has_target, const SweepArgs& a, int64_t R,
                               cudaStream_t s);
+// Markov embeddings (both copies) and confidence logits
+cudaError_t launch_heads_prep(const HeadsArgs& a, cudaStream_t s);
+// corrected rows ws.z = base + E.W2^T (compact, FP32) on the tensor cores
+cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s);
+// dE, dW1, dW2, dconf_w, dconf_b, dhidden from dlogits and the saved dL/dc
+cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s);
 
 }  // namespace dspark

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kPrologueThreads) prologue_kernel(const Prolog
     if (r < R) {
       if (s) a.ws.sup_list[before] = int32_t(r);
       else a.ws.zero_list[r - before] = int32_t(r);
+      a.ws.sup_index[r] = s ? int32_t(before) : -1;
     }
     __syncthreads();
     if (tid == 0) {

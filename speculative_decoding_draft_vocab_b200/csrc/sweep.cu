@@ -80,6 +80,18 @@ __device__ __forceinline__ void warp_lse_merge(float& m, float& s) {
   m = M;
 }
 
+// One group of EPV draft values (16 bytes of T-sized teacher values) in the draft's own
+// type: 16 bytes, or 32 bytes when FP32 draft rows meet a 16-bit output type.
+template <typename TZ, int EPV>
+__device__ __forceinline__ void load_group(const uint8_t* p, float* f) {
+  if constexpr (sizeof(TZ) * EPV == 16) {
+    unpack16<TZ>(*reinterpret_cast<const uint4*>(p), f);
+  } else {
+    unpack16<float>(*reinterpret_cast<const uint4*>(p), f);
+    unpack16<float>(*reinterpret_cast<const uint4*>(p + 16), f + 4);
+  }
+}
+
 // Control block in shared memory.
 struct Ctrl {
   uint64_t mbar_data[2];  // row segment (draft + teacher) landed
@@ -101,9 +113,15 @@ struct Ctrl {
 // on chip and a row fits in 4 SMs of a 148-SM part.  Shared memory holds one draft
 // landing buffer and two teacher buffers: the next row's copy is issued as soon as
 // the current draft segment is in registers, one full row ahead of its use.
-template <typename T, int CL, int NT, int NV, bool HAS_T>
+// TZ is the draft rows' type (the logits type, or FP32 corrected rows of the Markov
+// head); T is the type of the teacher and of the dlogits.
+template <typename TZ, typename T, int CL, int NT, int NV, bool HAS_T>
 __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int ZB = EPV * int(sizeof(TZ));  // bytes of one draft group
+  // FP32 rows under 16-bit outputs only come from the Markov head (compact rows,
+  // valid-slot mask); the other builds carry none of that code
+  constexpr bool kMarkov = sizeof(TZ) == 4 && sizeof(T) == 2;
   constexpr int NE = NV * EPV;
   constexpr int NW = NT / 32;
   static_assert(NW <= 32 && CL <= 16, "control block sizes");
@@ -114,16 +132,22 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t rank = cluster_ctarank();
   const uint32_t cid = cluster_id_x();
   const uint32_t G = nclusters_x();
-  const uint32_t seg_bytes = uint32_t(a.seg_vec) * 16u;
+  const uint32_t seg_bytes = uint32_t(a.seg_vec) * 16u;          // teacher segment
+  const uint32_t zseg_bytes = uint32_t(a.seg_vec) * uint32_t(ZB);  // draft segment
   // buffers: HAS_T: [draft][teacher 0][teacher 1]; else [draft 0][draft 1]
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + size_t(3 - (HAS_T ? 0 : 1)) * seg_bytes);
-  auto zbuf = [&](int j) -> uint8_t* { return HAS_T ? smem : smem + size_t(j & 1) * seg_bytes; };
-  auto tbuf = [&](int j) -> uint8_t* { return smem + size_t(1 + (j & 1)) * seg_bytes; };
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + (HAS_T ? size_t(zseg_bytes) + 2 * size_t(seg_bytes)
+                                                      : 2 * size_t(zseg_bytes)));
+  auto zbuf = [&](int j) -> uint8_t* { return HAS_T ? smem : smem + size_t(j & 1) * zseg_bytes; };
+  auto tbuf = [&](int j) -> uint8_t* {
+    if constexpr (ZB == 16) return smem + size_t(1 + (j & 1)) * seg_bytes;  // zseg == seg
+    else return smem + zseg_bytes + size_t(j & 1) * seg_bytes;
+  };
   WsHeader* hdr = a.ws.hdr;
 
   const int v0 = int(rank) * a.seg_vec;
   const int nvec = max(0, min(a.seg_vec, a.vvec - v0));
   const uint32_t bytes = uint32_t(nvec) * 16u;
+  const uint32_t zbytes = uint32_t(nvec) * uint32_t(ZB);
   const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
   const uint8_t* target = static_cast<const uint8_t*>(a.target);
   const bool bwd = a.dlogits != nullptr;
@@ -136,11 +160,13 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
   auto issue = [&](int j) {  // thread 0: stream row j's segment (draft and teacher)
     const uint32_t bar = (j & 1) ? bar_d1 : bar_d0;
-    const int64_t row = a.ws.sup_list[cid + size_t(j) * G];
-    mbar_arrive_expect_tx(bar, (HAS_T ? 2u : 1u) * bytes);
+    const int64_t sidx = cid + int64_t(j) * G;
+    const int64_t row = a.ws.sup_list[sidx];
+    const int64_t drow = (kMarkov && a.draft_compact) ? sidx : row;  // compact corrected rows
+    mbar_arrive_expect_tx(bar, zbytes + (HAS_T ? bytes : 0u));
     if (bytes) {
-      bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * sizeof(T),
-               bytes, bar, policy);
+      bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(drow) * a.ld_d + size_t(v0) * EPV) * sizeof(TZ),
+               zbytes, bar, policy);
       if constexpr (HAS_T)
         bulk_g2s(smem_u32(tbuf(j)), target + (size_t(row) * a.ld_t + size_t(v0) * EPV) * sizeof(T),
                  bytes, bar, policy);
@@ -208,14 +234,14 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     for (int i = 0; i < NV; ++i) {
       const int v = tid + i * NT;
       if (v < nvec) {
-        unpack16<T>(*reinterpret_cast<const uint4*>(zb + size_t(v) * 16), &xz[i * EPV]);
+        load_group<TZ, EPV>(zb + size_t(v) * ZB, &xz[i * EPV]);
       } else {
 #pragma unroll
         for (int e = 0; e < EPV; ++e) xz[i * EPV + e] = -INFINITY;
       }
     }
     if (tid == 0 && tv >= 0 && tv < nvec)
-      ctrl->ztid = load_elem<T>(zb + size_t(tv) * 16 + size_t(te) * sizeof(T));
+      ctrl->ztid = load_elem<TZ>(zb + size_t(tv) * ZB + size_t(te) * sizeof(TZ));
     __syncthreads();  // the draft buffer is free again
     if (tid == 0) {
       // HAS_T: draft buffer + the teacher buffer of row j-1 (its pass 2 is done).
@@ -364,7 +390,9 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
     // ---- pass 3: dlogits = p*(cce - cl1*S) + cl1*u, minus cce at the target id
     if (bwd) {
-      const float gw = g * wr;
+      // an invalid Markov slot's corrected row is a constant: nothing flows to base
+      const bool zero_out = kMarkov && a.invalid_zero && a.valid[row] == 0;
+      const float gw = zero_out ? 0.f : g * wr;
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
       const float k0 = cce - cl1 * S;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
@@ -423,15 +451,16 @@ struct LaunchCache {
   int clusters = 0;
 };
 
-template <typename T, int CL>
+template <typename TZ, typename T, int CL>
 size_t smem_bytes(int64_t V, bool has_t) {
   constexpr int EPV = VecTraits<T>::EPV;
   const int64_t vvec = V / EPV;
   const int64_t seg_vec = (vvec + CL - 1) / CL;
-  return size_t(has_t ? 3 : 2) * size_t(seg_vec) * 16 + sizeof(Ctrl);
+  const size_t zseg = size_t(seg_vec) * EPV * sizeof(TZ), tseg = size_t(seg_vec) * 16;
+  return (has_t ? zseg + 2 * tseg : 2 * zseg) + sizeof(Ctrl);
 }
 
-template <typename T, int CL, int NT, int NV, bool HAS_T>
+template <typename TZ, typename T, int CL, int NT, int NV, bool HAS_T>
 cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   constexpr int EPV = VecTraits<T>::EPV;
   SweepArgs a = a0;
@@ -439,10 +468,10 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   a.seg_vec = (a.vvec + CL - 1) / CL;
   a.nbuf = 2;
   // at least the report's reduction scratch (reused at the end)
-  const size_t smem = std::max<size_t>(smem_bytes<T, CL>(a.V, HAS_T), size_t(NT / 32) * kNAcc * sizeof(double));
+  const size_t smem = std::max<size_t>(smem_bytes<TZ, T, CL>(a.V, HAS_T), size_t(NT / 32) * kNAcc * sizeof(double));
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
-  auto kern = sweep_kernel<T, CL, NT, NV, HAS_T>;
+  auto kern = sweep_kernel<TZ, T, CL, NT, NV, HAS_T>;
   static LaunchCache cache;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -482,7 +511,7 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
     }
     clusters = cache.clusters;
   }
-  // programmatic dependent launch: the grid is scheduled while the mask prologue
+  // programmatic dependent launch: the grid is scheduled while the kernel before it
   // runs and waits for it (griddepcontrol.wait) before reading its results
   cudaLaunchAttribute at2[2];
   at2[0] = at[0];
@@ -499,54 +528,66 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
 }
 
 // Builds, smallest first.  A build covers rows of up to CL * NT * NV * (elements per
-// vector) logits when its shared-memory buffers fit.
+// 16-byte output vector) logits when its shared-memory buffers fit.
 struct Build {
   int cl, nt, nv;
 };
 constexpr int kNumBuilds = 5;
 constexpr Build kBf16Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {4, 512, 10}, {8, 512, 5}};
 constexpr Build kF32Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 8}, {8, 512, 10}, {16, 512, 5}};
+// FP32 corrected draft rows with bf16 teacher and dlogits (Markov head)
+constexpr Build kZf32Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}, {8, 512, 5}};
 
-template <typename T>
+template <typename TZ, typename T>
 size_t smem_for(int cl, int64_t V, bool has_t) {
   switch (cl) {
-    case 1: return smem_bytes<T, 1>(V, has_t);
-    case 2: return smem_bytes<T, 2>(V, has_t);
-    case 4: return smem_bytes<T, 4>(V, has_t);
-    case 8: return smem_bytes<T, 8>(V, has_t);
-    default: return smem_bytes<T, 16>(V, has_t);
+    case 1: return smem_bytes<TZ, T, 1>(V, has_t);
+    case 2: return smem_bytes<TZ, T, 2>(V, has_t);
+    case 4: return smem_bytes<TZ, T, 4>(V, has_t);
+    case 8: return smem_bytes<TZ, T, 8>(V, has_t);
+    default: return smem_bytes<TZ, T, 16>(V, has_t);
   }
 }
 
-int pick_build(int dtype, int64_t V, bool has_t) {
-  const Build* b = dtype == DSPARK_BF16 ? kBf16Builds : kF32Builds;
+// zf32: FP32 draft rows (dtype then names the teacher / dlogits type, bf16 only)
+int pick_build(int dtype, bool zf32, int64_t V, bool has_t) {
+  if (zf32 && dtype != DSPARK_BF16) return -1;
+  const Build* b = zf32 ? kZf32Builds : (dtype == DSPARK_BF16 ? kBf16Builds : kF32Builds);
   const int epv = dtype == DSPARK_BF16 ? 8 : 4;
   for (int i = 0; i < kNumBuilds; ++i) {
     if (int64_t(b[i].cl) * b[i].nt * b[i].nv * epv < V) continue;
-    const size_t sm = dtype == DSPARK_BF16 ? smem_for<__nv_bfloat16>(b[i].cl, V, has_t)
-                                           : smem_for<float>(b[i].cl, V, has_t);
+    const size_t sm = zf32 ? smem_for<float, __nv_bfloat16>(b[i].cl, V, has_t)
+                           : (dtype == DSPARK_BF16 ? smem_for<__nv_bfloat16, __nv_bfloat16>(b[i].cl, V, has_t)
+                                                   : smem_for<float, float>(b[i].cl, V, has_t));
     if (sm <= kMaxSmem) return i;
   }
   return -1;
 }
 
-template <typename T, bool HT>
+template <typename TZ, typename T, bool HT>
 cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
-  if constexpr (sizeof(T) == 2) {
+  if constexpr (sizeof(TZ) == 4 && sizeof(T) == 2) {
     switch (i) {
-      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<T, 4, 512, 4, HT>(a, s);
-      case 3: return launch_cfg<T, 4, 512, 10, HT>(a, s);
-      case 4: return launch_cfg<T, 8, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<TZ, T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<TZ, T, 4, 512, 4, HT>(a, s);
+      default: return launch_cfg<TZ, T, 8, 512, 5, HT>(a, s);
+    }
+  } else if constexpr (sizeof(T) == 2) {
+    switch (i) {
+      case 0: return launch_cfg<TZ, T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<TZ, T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<TZ, T, 4, 512, 4, HT>(a, s);
+      case 3: return launch_cfg<TZ, T, 4, 512, 10, HT>(a, s);
+      case 4: return launch_cfg<TZ, T, 8, 512, 5, HT>(a, s);
     }
   } else {
     switch (i) {
-      case 0: return launch_cfg<T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<T, 4, 512, 8, HT>(a, s);
-      case 3: return launch_cfg<T, 8, 512, 10, HT>(a, s);
-      case 4: return launch_cfg<T, 16, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, T, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<TZ, T, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<TZ, T, 4, 512, 8, HT>(a, s);
+      case 3: return launch_cfg<TZ, T, 8, 512, 10, HT>(a, s);
+      case 4: return launch_cfg<TZ, T, 16, 512, 5, HT>(a, s);
     }
   }
   return cudaErrorInvalidValue;
@@ -554,74 +595,82 @@ cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool sweep_supported(int dtype, int64_t V, bool has_target) {
-  return pick_build(dtype, V, has_target) >= 0;
+bool sweep_supported(int dtype, bool zf32, int64_t V, bool has_target) {
+  return pick_build(dtype, zf32, V, has_target) >= 0;
 }
 
-cudaError_t launch_sweep(int dtype, bool has_target, const SweepArgs& a, cudaStream_t s) {
-  const int i = pick_build(dtype, a.V, has_target);
+cudaError_t launch_sweep(int dtype, bool zf32, bool has_target, const SweepArgs& a, cudaStream_t s) {
+  const int i = pick_build(dtype, zf32, a.V, has_target);
   if (i < 0) return cudaErrorInvalidValue;
+  if (zf32)
+    return has_target ? dispatch<float, __nv_bfloat16, true>(i, a, s) : dispatch<float, __nv_bfloat16, false>(i, a, s);
   if (dtype == DSPARK_BF16)
-    return has_target ? dispatch<__nv_bfloat16, true>(i, a, s) : dispatch<__nv_bfloat16, false>(i, a, s);
-  return has_target ? dispatch<float, true>(i, a, s) : dispatch<float, false>(i, a, s);
+    return has_target ? dispatch<__nv_bfloat16, __nv_bfloat16, true>(i, a, s)
+                      : dispatch<__nv_bfloat16, __nv_bfloat16, false>(i, a, s);
+  return has_target ? dispatch<float, float, true>(i, a, s) : dispatch<float, float, false>(i, a, s);
 }
 
 // ------------------------------------------------------- backward-only stream
 // dlogits from saved row statistics: one more read of the logits, no reductions.
-template <typename T, bool HAS_T>
+template <typename TZ, typename T, bool HAS_T>
 __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a, const int64_t R) {
   constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int ZB = EPV * int(sizeof(TZ));
   const int vvec = int(a.V / EPV);
   for (int64_t row = blockIdx.y; row < R; row += gridDim.y) {
-  uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * a.ld_g * sizeof(T);
-  const bool sup = a.ws.m[row] != 0;
-  if (!sup) {
-    for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x)
-      *reinterpret_cast<uint4*>(out + size_t(v) * 16) = make_uint4(0u, 0u, 0u, 0u);
-    continue;
-  }
-  const float* st = a.ws.stats + size_t(row) * kStride;
-  const float g = a.grad_scale ? *a.grad_scale : 1.f;
-  const float gw = g * a.ws.w[row];
-  const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
-  const float S = st[kStS];
-  const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S), kzero = cce - cl1 * S;
-  const float lz2 = st[kStLseD] * kLog2e, lt2 = st[kStLseT] * kLog2e;
-  const int64_t tok = a.tids[row];
-  const uint8_t* zr = static_cast<const uint8_t*>(a.draft) + size_t(row) * a.ld_d * sizeof(T);
-  const uint8_t* tr = static_cast<const uint8_t*>(a.target) + size_t(row) * a.ld_t * sizeof(T);
-  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x) {
-    float z[EPV], t[EPV], o[EPV];
-    unpack16<T>(*reinterpret_cast<const uint4*>(zr + size_t(v) * 16), z);
-    if constexpr (HAS_T) unpack16<T>(*reinterpret_cast<const uint4*>(tr + size_t(v) * 16), t);
-#pragma unroll
-    for (int e = 0; e < EPV; ++e) {
-      const float p = ex2(fmaf(z[e], kLog2e, -lz2));
-      if constexpr (HAS_T) {
-        const float d = p - ex2(fmaf(t[e], kLog2e, -lt2));
-        o[e] = p * (d > 0.f ? kpos : (d < 0.f ? kneg : kzero));
-      } else {
-        o[e] = p * cce;
-      }
-      if (int64_t(v) * EPV + e == tok) o[e] -= cce;
+    uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * a.ld_g * sizeof(T);
+    const bool zero_row = a.ws.m[row] == 0 || (a.invalid_zero && a.valid != nullptr && a.valid[row] == 0);
+    if (zero_row) {
+      for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x)
+        *reinterpret_cast<uint4*>(out + size_t(v) * 16) = make_uint4(0u, 0u, 0u, 0u);
+      continue;
     }
-    *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<T>(o);
-  }
+    const float* st = a.ws.stats + size_t(row) * kStride;
+    const float g = a.grad_scale ? *a.grad_scale : 1.f;
+    const float gw = g * a.ws.w[row];
+    const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
+    const float S = st[kStS];
+    const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S), kzero = cce - cl1 * S;
+    const float lz2 = st[kStLseD] * kLog2e, lt2 = st[kStLseT] * kLog2e;
+    const int64_t tok = a.tids[row];
+    const int64_t drow = a.draft_compact ? int64_t(a.ws.sup_index[row]) : row;
+    const uint8_t* zr = static_cast<const uint8_t*>(a.draft) + size_t(drow) * a.ld_d * sizeof(TZ);
+    const uint8_t* tr = static_cast<const uint8_t*>(a.target) + size_t(row) * a.ld_t * sizeof(T);
+    for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x) {
+      float z[EPV], t[EPV], o[EPV];
+      load_group<TZ, EPV>(zr + size_t(v) * ZB, z);
+      if constexpr (HAS_T) unpack16<T>(*reinterpret_cast<const uint4*>(tr + size_t(v) * 16), t);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) {
+        const float p = ex2(fmaf(z[e], kLog2e, -lz2));
+        if constexpr (HAS_T) {
+          const float d = p - ex2(fmaf(t[e], kLog2e, -lt2));
+          o[e] = p * (d > 0.f ? kpos : (d < 0.f ? kneg : kzero));
+        } else {
+          o[e] = p * cce;
+        }
+        if (int64_t(v) * EPV + e == tok) o[e] -= cce;
+      }
+      *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<T>(o);
+    }
   }
 }
 
-cudaError_t launch_bwd_stream(int dtype, bool has_target, const SweepArgs& a, int64_t R,
+cudaError_t launch_bwd_stream(int dtype, bool zf32, bool has_target, const SweepArgs& a, int64_t R,
                               cudaStream_t s) {
   const int epv = dtype == DSPARK_BF16 ? 8 : 4;
   const int64_t vvec = a.V / epv;
   const unsigned gx = unsigned(std::min<int64_t>((vvec + 1023) / 1024, 64));
   dim3 grid(gx > 0 ? gx : 1, unsigned(std::min<int64_t>(R, 65535)), 1);
-  if (dtype == DSPARK_BF16) {
-    if (has_target) bwd_stream_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(a, R);
-    else bwd_stream_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(a, R);
+  if (zf32) {
+    if (has_target) bwd_stream_kernel<float, __nv_bfloat16, true><<<grid, 256, 0, s>>>(a, R);
+    else bwd_stream_kernel<float, __nv_bfloat16, false><<<grid, 256, 0, s>>>(a, R);
+  } else if (dtype == DSPARK_BF16) {
+    if (has_target) bwd_stream_kernel<__nv_bfloat16, __nv_bfloat16, true><<<grid, 256, 0, s>>>(a, R);
+    else bwd_stream_kernel<__nv_bfloat16, __nv_bfloat16, false><<<grid, 256, 0, s>>>(a, R);
   } else {
-    if (has_target) bwd_stream_kernel<float, true><<<grid, 256, 0, s>>>(a, R);
-    else bwd_stream_kernel<float, false><<<grid, 256, 0, s>>>(a, R);
+    if (has_target) bwd_stream_kernel<float, float, true><<<grid, 256, 0, s>>>(a, R);
+    else bwd_stream_kernel<float, float, false><<<grid, 256, 0, s>>>(a, R);
   }
   return cudaGetLastError();
 }

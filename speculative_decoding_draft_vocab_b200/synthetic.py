@@ -126,13 +126,16 @@ def make_inputs(name: str = "recipe", device="cpu", seed: Optional[int] = None,
     hidden size), ``target_hidden_size``, ``rank``, ``target_vocab``,
     ``valid_p`` (probability a slot is Markov-valid), ``mask_holes`` (add stray
     ones after each prefix so the cumprod inside the loss has work to do),
-    ``no_target`` (CE-only), ``gamma``, ``grad_scale``, ``conf_with_markov``.
+    ``no_target`` (CE-only), ``gamma``, ``grad_scale``, ``conf_with_markov``,
+    ``markov_std`` (std of both Markov tables; 0.02 is the initialisation scale, a
+    larger one makes the correction visible in tests), ``conf_bias``.
     The default seed is 1234 + the configuration's index.
     """
     base = dict(CONFIGS[name])
     base.update(dict(hidden=HIDDEN, target_hidden_size=HIDDEN, rank=MARKOV_RANK,
                      target_vocab=None, valid_p=0.9, mask_holes=False, no_target=False,
-                     gamma=4.0, grad_scale=1.0, conf_with_markov=None))
+                     gamma=4.0, grad_scale=1.0, conf_with_markov=None, markov_std=0.02,
+                     conf_bias=0.0))
     unknown = set(overrides) - set(base)
     if unknown:
         raise TypeError(f"unknown overrides {sorted(unknown)}")
@@ -199,8 +202,8 @@ def make_inputs(name: str = "recipe", device="cpu", seed: Optional[int] = None,
         ids_in_t = target_ids.clamp(max=Vt - 1)
         inp.prev_ids = torch.cat([anchor, ids_in_t[..., :-1]], dim=-1).contiguous()
         inp.valid = (torch.rand((B, N, K), generator=gen, device=device) < c["valid_p"]).to(torch.uint8)
-        inp.markov_w1 = _normal(gen, (Vt, r), 0.02, device, torch.bfloat16)
-        inp.markov_w2 = _normal(gen, (V, r), 0.02, device, torch.bfloat16)
+        inp.markov_w1 = _normal(gen, (Vt, r), c["markov_std"], device, torch.bfloat16)
+        inp.markov_w2 = _normal(gen, (V, r), c["markov_std"], device, torch.bfloat16)
 
     # ---- confidence ----------------------------------------------------------
     if c["conf"] == "given":
@@ -213,7 +216,7 @@ def make_inputs(name: str = "recipe", device="cpu", seed: Optional[int] = None,
         inp.conf_with_markov = with_markov
         inp.draft_hidden = _normal(gen, (B, N, K, H), 1.0, device, torch.bfloat16)
         inp.conf_w = _normal(gen, (1, H + (r if with_markov else 0)), 0.02, device, torch.bfloat16)
-        inp.conf_b = torch.zeros(1, dtype=torch.float32, device=device)
+        inp.conf_b = torch.full((1,), float(c["conf_bias"]), dtype=torch.float32, device=device)
         if not c["markov"]:
             # a confidence head without a Markov head still needs the valid-slot mask
             inp.valid = (torch.rand((B, N, K), generator=gen, device=device) < c["valid_p"]).to(torch.uint8)

@@ -148,3 +148,61 @@ def test_status_strings_and_workspace_size(abi):
     assert 0 < n1 < n2 and n1 % 256 == 0
     p.K = 0
     assert abi.dspark_workspace_size(ctypes.byref(p)) == 0
+
+
+def _with_markov(abi, p, rank=64):
+    p.prev_ids = ctypes.c_void_p(0x80000)
+    p.valid = ctypes.c_void_p(0x90000)
+    p.target_vocab = 500
+    p.markov_w1 = ctypes.c_void_p(0xa0000)
+    p.markov_w2 = ctypes.c_void_p(0xb0000)
+    p.markov_rank = rank
+    return p
+
+
+def _with_conf_head(abi, p, H=256, with_markov=0):
+    p.valid = ctypes.c_void_p(0x90000)
+    p.draft_hidden = ctypes.c_void_p(0xc0000)
+    p.hidden_size = H
+    p.conf_w = ctypes.c_void_p(0xd0000)
+    p.conf_b = ctypes.c_void_p(0xe0000)
+    p.conf_with_markov = with_markov
+    return p
+
+
+def test_head_validation_status_codes(abi):
+    prm = _params(abi)
+    # the Markov head needs bf16 logits (its backward contracts bf16 dlogits)
+    assert _fwd(abi, _with_markov(abi, _problem(abi, dtype=abi.DSPARK_F32)), prm) == abi.DSPARK_ERR_UNSUPPORTED
+    # rank not a multiple of 8, misaligned table
+    assert _fwd(abi, _with_markov(abi, _problem(abi), rank=60), prm) == abi.DSPARK_ERR_ALIGNMENT
+    p = _with_markov(abi, _problem(abi))
+    p.markov_w2 = ctypes.c_void_p(0xb0008)
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_ALIGNMENT
+    # a partial Markov head (no valid mask / no W1) is refused
+    p = _with_markov(abi, _problem(abi))
+    p.valid = None
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    p = _with_markov(abi, _problem(abi))
+    p.markov_w1 = None
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    # confidence head: hidden size rule, a Markov input without the Markov head
+    assert _fwd(abi, _with_conf_head(abi, _problem(abi), H=100), prm) == abi.DSPARK_ERR_ALIGNMENT
+    assert _fwd(abi, _with_conf_head(abi, _problem(abi), with_markov=1), prm) == abi.DSPARK_ERR_INVALID_ARG
+    p = _with_conf_head(abi, _problem(abi))
+    p.conf_b = None
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    # the confidence head needs the teacher (its label is 1 - L1/2)
+    assert _fwd(abi, _with_conf_head(abi, _problem(abi, target=False)), _params(abi, l1=0.0)) == \
+        abi.DSPARK_ERR_MISSING_TARGET
+
+
+def test_markov_workspace_holds_corrected_rows(abi):
+    p = _problem(abi, V=4096)
+    p.B, p.N, p.K = 2, 3, 7
+    base = abi.dspark_workspace_size(ctypes.byref(p))
+    n = abi.dspark_workspace_size(ctypes.byref(_with_markov(abi, p, rank=64)))
+    R = 2 * 3 * 7
+    assert n >= base + R * 4096 * 4 + 2 * R * 64 * 2 + R * 64 * 4
+    # a workspace sized without the head is refused for a problem with it
+    assert _fwd(abi, p, _params(abi), ws_bytes=base) == abi.DSPARK_ERR_WORKSPACE
