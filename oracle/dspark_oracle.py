@@ -253,7 +253,10 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
     ``report`` (key -> (numerator, denominator); nothing divided), per-row
     ``ce``, ``l1``, ``S``, ``lse_d``, ``lse_t``, ``conf`` (c), ``bce``, ``accept``,
     masks ``m`` and ``w``, and with ``want_grads``: ``dlogits`` (row -> dL/dbase
-    row), ``sign_amb`` (row -> mask), ``dconf`` [R], and for the heads ``dW2``,
+    row), ``sign_amb`` (row -> mask), ``dlogit_swing`` (row -> width of the interval of
+    valid dz_j where sign(p_j - q_j) is undecided, 0 elsewhere), per-row sums over
+    every supervised row ``dz_norm2`` [R] (sum_j dlogits_j^2) and ``swing_sum`` [R],
+    ``dconf`` [R], and for the heads ``dW2``,
     ``dE`` (row -> dL/de), ``dW1`` (id -> row), ``dconf_w``, ``dconf_b``, ``dhidden``.
 
     The loss is sum_r w_r (ce_alpha*CE_r + l1_alpha*L1_r + conf_alpha*BCE_r) where
@@ -300,7 +303,8 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
     sup = np.nonzero(m_r)[0] if rows is None else np.asarray(rows, dtype=np.int64)
     keep = set(int(r) for r in (sup if keep_rows is None else keep_rows))
     ce = np.zeros(R); l1 = np.zeros(R); S = np.zeros(R); lse_d = np.zeros(R); lse_t = np.zeros(R)
-    dlogits, amb, dE = {}, {}, {}
+    dlogits, amb, swing, dE = {}, {}, {}, {}
+    dz_norm2, swing_sum = np.zeros(R), np.zeros(R)
     dW2 = np.zeros_like(w2) if (has_markov and want_grads) else None
 
     for c0 in range(0, len(sup), row_chunk):
@@ -333,10 +337,18 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
             row_grad = dz
             if has_markov and not markov_live and invalid_row_mode == 0:
                 row_grad = np.zeros(V)             # the corrected row is the constant 0
+            dz_norm2[r] = float(np.dot(row_grad, row_grad))
+            if rt["q"] is not None and row_grad is dz:
+                swing_sum[r] = float(np.sum(np.where(sign_ambiguity(rt["p"], rt["q"]),
+                                                     2.0 * grad_scale * w_r[r] * l1_alpha * rt["p"], 0.0)))
             if r in keep:
                 dlogits[r] = row_grad
                 amb[r] = (sign_ambiguity(rt["p"], rt["q"]) if rt["q"] is not None
                           else np.zeros(V, dtype=bool))
+                # where sign(p_j - q_j) is undecided, |p_j - q_j| has every sub-gradient in
+                # [-1, 1]: the valid values of dz_j span 2 g w l1_alpha p_j
+                swing[r] = (np.where(amb[r], 2.0 * grad_scale * w_r[r] * l1_alpha * rt["p"], 0.0)
+                            if row_grad is dz else np.zeros(V))
             if markov_live:
                 dz_live.append((r, dz))
         if dz_live:
@@ -372,7 +384,8 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
     dconf = np.zeros(R)
     if has_conf:
         dconf[sup] = grad_scale * w_r[sup] * conf_alpha * (sigmoid(c_rows[sup]) - y[sup])
-    res.update(dlogits=dlogits, sign_amb=amb, dconf=dconf)
+    res.update(dlogits=dlogits, sign_amb=amb, dlogit_swing=swing, dz_norm2=dz_norm2, swing_sum=swing_sum,
+               dconf=dconf)
     if conf_w is not None:
         hv = _as_rows(draft_hidden, R).astype(np.float64)
         H = hv.shape[1]

@@ -1,6 +1,7 @@
 // The C ABI of include/dspark.h: host-side validation, workspace carving and the
 // launch sequence of each entry point.  No allocation, no synchronisation (except
 // dspark_check_status, whose job it is).
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 
@@ -29,16 +30,30 @@ inline bool markov_present(const dspark_problem_t* p) {
   return p->markov_w2 != nullptr || p->markov_w1 != nullptr || p->prev_ids != nullptr;
 }
 
+inline bool lm_present(const dspark_problem_t* p) { return p->lm_head != nullptr || p->target_hidden != nullptr; }
+
 inline WsDims ws_dims(const dspark_problem_t* p) {
   WsDims d{};
   d.R = p->B * p->N * p->K;
+  d.V = p->V;
   d.markov = markov_present(p);
   if (d.markov) {
-    d.V = p->V;
     d.rank = p->markov_rank;
     d.splits = heads_splits(d.R, p->V);
   }
+  d.lm = lm_present(p) && p->target_logits == nullptr;
+  if (d.lm) {
+    d.Ht = p->target_hidden_size;
+    d.chunk = teacher_chunk_rows(d.R);
+  }
   return d;
+}
+
+// Row types the sweep reads and writes.
+inline int sweep_kind(const dspark_problem_t* p) {
+  if (p->logits_dtype == DSPARK_F32) return kSweepF32;
+  const bool z32 = markov_present(p), t32 = lm_present(p);
+  return z32 ? (t32 ? kSweepZT32 : kSweepZ32) : (t32 ? kSweepT32 : kSweepBf16);
 }
 
 dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* prm, Shape* sh) {
@@ -55,7 +70,7 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
   Shape s{};
   s.R = p->B * p->N * p->K;
   s.has_target_rows = p->target_logits != nullptr;
-  s.has_lm_head = p->lm_head != nullptr || p->target_hidden != nullptr;
+  s.has_lm_head = lm_present(p);
   s.has_teacher = s.has_target_rows || s.has_lm_head;
   s.has_markov = markov_present(p);
   s.has_conf_given = p->confidence_logits != nullptr;
@@ -72,8 +87,14 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
     if (prm->gamma_enabled && !(prm->gamma > 0.f)) return DSPARK_ERR_INVALID_ARG;
     if (prm->invalid_row_mode != 0 && prm->invalid_row_mode != 1) return DSPARK_ERR_INVALID_ARG;
   }
-  // The teacher-from-hidden path is not part of this build.
-  if (s.has_lm_head) return DSPARK_ERR_UNSUPPORTED;
+  if (s.has_lm_head) {
+    if (!p->lm_head || !p->target_hidden || p->target_hidden_size <= 0) return DSPARK_ERR_INVALID_ARG;
+    // the teacher rows come from the tensor cores in FP32; the sweep pairs them with
+    // bf16 logits
+    if (p->logits_dtype != DSPARK_BF16) return DSPARK_ERR_UNSUPPORTED;
+    if (p->target_hidden_size % 8 || !aligned16(p->lm_head) || !aligned16(p->target_hidden))
+      return DSPARK_ERR_ALIGNMENT;
+  }
   if (s.has_markov) {
     if (!p->markov_w1 || !p->markov_w2 || !p->prev_ids || !p->valid) return DSPARK_ERR_INVALID_ARG;
     if (p->markov_rank <= 0 || p->target_vocab <= 0) return DSPARK_ERR_INVALID_ARG;
@@ -87,7 +108,7 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
     if (p->conf_with_markov && !s.has_markov) return DSPARK_ERR_INVALID_ARG;
     if (p->hidden_size % 8 || !aligned16(p->conf_w) || !aligned16(p->draft_hidden)) return DSPARK_ERR_ALIGNMENT;
   }
-  if (!sweep_supported(int(p->logits_dtype), s.has_markov, p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
+  if (!sweep_supported(sweep_kind(p), p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
   *sh = s;
   return DSPARK_OK;
 }
@@ -123,7 +144,16 @@ SweepArgs sweep_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
   a.ws = ws;
   a.V = p->V;
   a.ce_alpha = prm->ce_alpha;
-  a.l1_alpha = p->target_logits ? prm->l1_alpha : 0.f;
+  a.l1_alpha = (p->target_logits || lm_present(p)) ? prm->l1_alpha : 0.f;
+  a.row0 = 0;
+  a.row1 = int32_t(p->B * p->N * p->K);
+  a.do_zero = 1;
+  a.do_final = 1;
+  if (lm_present(p)) {  // the teacher rows of the current chunk
+    a.target = ws.tchunk;
+    a.ld_t = p->V;
+    a.target_compact = 1;
+  }
   if (markov_present(p)) {  // the sweep reads the corrected rows, compact by supervised position
     a.draft = ws.z;
     a.ld_d = p->V;
@@ -132,6 +162,17 @@ SweepArgs sweep_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
     a.invalid_zero = prm->invalid_row_mode == 0;
   }
   return a;
+}
+
+TeacherArgs teacher_args(const dspark_problem_t* p, const WsView& ws) {
+  TeacherArgs t{};
+  t.R = p->B * p->N * p->K;
+  t.V = p->V;
+  t.Ht = p->target_hidden_size;
+  t.hidden = static_cast<const uint16_t*>(p->target_hidden);
+  t.lm_head = static_cast<const uint16_t*>(p->lm_head);
+  t.ws = ws;
+  return t;
 }
 
 HeadsArgs heads_args(const dspark_problem_t* p, const dspark_params_t* prm, const WsView& ws,
@@ -244,8 +285,24 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   fa.accept_rows = out->accept_rows;
   fa.conf_rows = out->conf_rows;
   fa.dconf = grads ? grads->dconf : nullptr;
-  e = launch_sweep(int(prob->logits_dtype), sh.has_markov, sh.has_target_rows, sa, s);
-  if (e != cudaSuccess) return cuda_status(e);
+  const int kind = sweep_kind(prob);
+  if (!sh.has_lm_head) {
+    e = launch_sweep(kind, sh.has_teacher, sa, s);
+    if (e != cudaSuccess) return cuda_status(e);
+  } else {
+    // teacher rows a chunk of supervised rows at a time, each chunk swept right after
+    const TeacherArgs ta = teacher_args(prob, v);
+    if ((e = launch_gather_hidden(ta, s)) != cudaSuccess) return cuda_status(e);
+    const int64_t C = teacher_chunk_rows(sh.R);
+    for (int64_t r0 = 0; r0 < sh.R; r0 += C) {
+      if ((e = launch_teacher_chunk(ta, r0, s)) != cudaSuccess) return cuda_status(e);
+      sa.row0 = int32_t(r0);
+      sa.row1 = int32_t(std::min<int64_t>(r0 + C, sh.R));
+      sa.do_zero = r0 == 0;
+      sa.do_final = r0 + C >= sh.R;
+      if ((e = launch_sweep(kind, true, sa, s)) != cudaSuccess) return cuda_status(e);
+    }
+  }
   if (grads && (sh.has_markov || sh.has_conf_head)) e = launch_heads_bwd(ha, s);
   return cuda_status(e);
 }
@@ -262,8 +319,23 @@ dspark_status_t dspark_loss_bwd(const dspark_problem_t* prob, const dspark_param
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WsView v = ws_layout(ws, ws_dims(prob));
   SweepArgs sa = sweep_args(prob, params, v, grads);
-  cudaError_t e = launch_bwd_stream(int(prob->logits_dtype), sh.has_markov, sh.has_target_rows, sa, sh.R, s);
-  if (e != cudaSuccess) return cuda_status(e);
+  const int kind = sweep_kind(prob);
+  cudaError_t e = cudaSuccess;
+  if (!sh.has_lm_head) {
+    e = launch_bwd_stream(kind, sh.has_teacher, sa, sh.R, s);
+    if (e != cudaSuccess) return cuda_status(e);
+  } else {
+    // a single chunk is still in the workspace from the forward; more are recomputed
+    const TeacherArgs ta = teacher_args(prob, v);
+    const int64_t C = teacher_chunk_rows(sh.R);
+    for (int64_t r0 = 0; r0 < sh.R; r0 += C) {
+      if (C < sh.R && (e = launch_teacher_chunk(ta, r0, s)) != cudaSuccess) return cuda_status(e);
+      sa.row0 = int32_t(r0);
+      sa.row1 = int32_t(std::min<int64_t>(r0 + C, sh.R));
+      sa.do_zero = r0 == 0;
+      if ((e = launch_bwd_stream(kind, true, sa, sh.R, s)) != cudaSuccess) return cuda_status(e);
+    }
+  }
   if (sh.has_conf_given || sh.has_conf_head) {
     // dL/dc for this call's grad_scale, also saved for the confidence head's backward
     e = launch_conf_grad(sh.R, prob->confidence_logits, params->conf_alpha, grads->grad_scale, v,

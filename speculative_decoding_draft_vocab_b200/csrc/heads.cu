@@ -7,7 +7,9 @@
 //   dE_r  = W2^T dz_r + dc_r proj_e,  dW2 = sum_r dz_r (x) e_r,  dW1[prev_r] += dE_r
 //   dproj = sum_r dc_r [h_r ; e_r],  dbias = sum_r dc_r,  dh_r = dc_r proj_h
 // (TorchSpec pull request #132, test list: the Markov bias is W2 applied to the W1 row
-// of the previous token).  The two contractions against the vocabulary (bias,
+// of the previous token), and the teacher computed from the target's final hidden
+// states, t = lm_head . h (TorchSpec pull request #132, scope list), one chunk of
+// supervised rows at a time.  The contractions against the vocabulary (bias, teacher,
 // dE, dW2) run on the tcgen05 GEMM; the rest are small row kernels.
 #include <cuda_bf16.h>
 
@@ -181,6 +183,35 @@ __global__ void __launch_bounds__(256) dhidden_kernel(const HeadsArgs a) {
   }
 }
 
+// ---- teacher from hidden states: gather, then t = lm_head . h per supervised row
+__global__ void __launch_bounds__(256) gather_hidden_kernel(const TeacherArgs a) {
+  const int warps = blockDim.x / 32;
+  const int lane = threadIdx.x & 31;
+  const int n_sup = a.ws.hdr->n_sup;
+  for (int64_t si = int64_t(blockIdx.x) * warps + threadIdx.x / 32; si < n_sup; si += int64_t(gridDim.x) * warps) {
+    const int64_t row = a.ws.sup_list[si];
+    const uint4* src = reinterpret_cast<const uint4*>(a.hidden + size_t(row) * a.Ht);
+    uint4* dst = reinterpret_cast<uint4*>(a.ws.hsup + size_t(si) * a.Ht);
+    for (int64_t j = lane; j < a.Ht / 8; j += 32) dst[j] = src[j];
+  }
+}
+
+// epilogue of the teacher GEMM: FP32 teacher rows of the chunk, row i of the chunk
+// being supervised-list position row0 + i
+struct TeacherEpi {
+  const WsHeader* hdr;
+  float* t;
+  int64_t V;
+  int row0, rows;
+  __device__ void operator()(int m, int n, int /*split*/, const float* v) const {
+    if (m >= rows || row0 + m >= hdr->n_sup) return;
+    float* out = t + size_t(m) * V;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (n + i < V) out[n + i] = v[i];
+  }
+};
+
 inline int grid_for(int64_t n, int per_block) {
   const int64_t g = (n + per_block - 1) / per_block;
   return int(std::max<int64_t>(1, std::min<int64_t>(g, 4096)));
@@ -193,12 +224,30 @@ cudaError_t launch_heads_prep(const HeadsArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_gather_hidden(const TeacherArgs& a, cudaStream_t s) {
+  gather_hidden_kernel<<<grid_for(a.R, 8), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_teacher_chunk(const TeacherArgs& a, int64_t row0, cudaStream_t s) {
+  const int64_t rows = std::min<int64_t>(teacher_chunk_rows(a.R), a.R - row0);
+  if (rows <= 0) return cudaSuccess;
+  // A = the chunk's hidden rows [rows][Ht] (K-major), B = lm_head [V][Ht] (K-major)
+  CUtensorMap ma, mb;
+  if (!tc::make_map(&ma, a.ws.hsup + size_t(row0) * a.Ht, rows, a.Ht, a.Ht, 64, 128)) return cudaErrorInvalidValue;
+  if (!tc::make_map(&mb, a.lm_head, a.V, a.Ht, a.Ht, 64, 256)) return cudaErrorInvalidValue;
+  TeacherEpi epi{a.ws.hdr, a.ws.tchunk, a.V, int(row0), int(rows)};
+  return tc::gemm<256, false, false, 4>(ma, mb, int(rows), int(a.V), int(a.Ht), 1, epi, &a.ws.hdr->status, s,
+                                        &a.ws.hdr->n_sup, int(row0));
+}
+
 cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   if (!tc::make_map(&ma, a.ws.esup, a.R, a.rank, a.rank, 64, 128)) return cudaErrorInvalidValue;
   if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 256)) return cudaErrorInvalidValue;
   BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.base, a.ld_base, a.valid, a.invalid_row_mode, a.ws.z, a.V, int(a.V)};
-  return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s);
+  return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s,
+                                        &a.ws.hdr->n_sup, 0);
 }
 
 cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {

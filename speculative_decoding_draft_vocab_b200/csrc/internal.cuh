@@ -55,6 +55,9 @@ struct WsView {
   uint16_t* eall;      // [R][rank] bf16 Markov embeddings by row (0 unless supervised+valid)
   float* dep;          // [splits][R][rank] split-K partials of dE
   float* de;           // [R][rank] dL/de
+  // teacher from hidden states (present when the problem has it)
+  uint16_t* hsup;      // [R][Ht] bf16 target hidden rows, compact by supervised position
+  float* tchunk;       // [chunk][V] FP32 teacher rows of one chunk of supervised rows
   size_t bytes;        // total bytes used
 };
 
@@ -64,10 +67,17 @@ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct WsDims {
   int64_t R = 0, V = 0, rank = 0, splits = 0;
   bool markov = false;
+  int64_t Ht = 0, chunk = 0;  // teacher from hidden states: hidden size, rows per chunk
+  bool lm = false;
 };
 
+// Supervised rows per teacher chunk (the FP32 teacher rows of a chunk are the only
+// vocabulary-wide teacher buffer; a multiple of the GEMM's 128-row tile).
+constexpr int64_t kTeacherChunk = 512;
+constexpr int64_t teacher_chunk_rows(int64_t R) { return R < kTeacherChunk ? R : kTeacherChunk; }
+
 struct WsOffsets {
-  size_t hdr, m, w, sup, zero, sidx, stats, z, esup, eall, dep, de, bytes;
+  size_t hdr, m, w, sup, zero, sidx, stats, z, esup, eall, dep, de, hsup, tchunk, bytes;
 };
 
 constexpr WsOffsets ws_offsets(const WsDims& d) {
@@ -99,6 +109,10 @@ constexpr WsOffsets ws_offsets(const WsDims& d) {
   off = align256(off + sizeof(float) * er * size_t(d.markov ? d.splits : 0));
   o.de = off;
   off = align256(off + sizeof(float) * er);
+  o.hsup = off;
+  off = align256(off + (d.lm ? 2 * R * size_t(d.Ht) : 0));
+  o.tchunk = off;
+  off = align256(off + (d.lm ? sizeof(float) * size_t(d.chunk) * size_t(d.V) : 0));
   o.bytes = off;
   return o;
 }
@@ -125,6 +139,8 @@ inline WsView ws_layout(void* base, const WsDims& d) {
   v.eall = d.markov ? reinterpret_cast<uint16_t*>(b + o.eall) : nullptr;
   v.dep = d.markov ? reinterpret_cast<float*>(b + o.dep) : nullptr;
   v.de = d.markov ? reinterpret_cast<float*>(b + o.de) : nullptr;
+  v.hsup = d.lm ? reinterpret_cast<uint16_t*>(b + o.hsup) : nullptr;
+  v.tchunk = d.lm ? reinterpret_cast<float*>(b + o.tchunk) : nullptr;
   v.bytes = o.bytes;
   return v;
 }
@@ -184,6 +200,10 @@ struct SweepArgs {
   int32_t draft_compact;     // draft row of the i-th supervised row is i (corrected rows)
   const uint8_t* valid;      // Markov valid-slot mask (with invalid_zero)
   int32_t invalid_zero;      // invalid slots get zero dlogits (all-zero corrected row)
+  int32_t target_compact;    // teacher row of list position i is i - row0 (teacher chunk)
+  int32_t row0, row1;        // supervised-list positions this launch covers
+  int32_t do_zero;           // this launch also zero-fills the unsupervised rows' dlogits
+  int32_t do_final;          // this launch ends with the per-row epilogue and report
   float ce_alpha, l1_alpha;
   FinalizeArgs fin;          // the per-row epilogue the last CTA runs
 };
@@ -226,10 +246,17 @@ constexpr int heads_splits(int64_t R, int64_t V) {
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s);
-// zf32: FP32 corrected draft rows (compact) with bf16 teacher and dlogits.  Returns
-// false if V exceeds every build of that combination.
-bool sweep_supported(int dtype, bool zf32, int64_t V, bool has_target);
-cudaError_t launch_sweep(int dtype, bool zf32, bool has_target, const SweepArgs& a, cudaStream_t s);
+// Row types of a sweep: draft / teacher / dlogits.
+enum : int {
+  kSweepBf16 = 0,  // bf16 / bf16 / bf16
+  kSweepF32 = 1,   // f32 / f32 / f32
+  kSweepZ32 = 2,   // f32 corrected rows (Markov head) / bf16 / bf16
+  kSweepT32 = 3,   // bf16 / f32 teacher chunk (teacher from hidden states) / bf16
+  kSweepZT32 = 4,  // f32 corrected rows / f32 teacher chunk / bf16
+};
+// False if V exceeds every build of that kind.
+bool sweep_supported(int kind, int64_t V, bool has_target);
+cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s);
 cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
                               const uint8_t* eval_mask, const uint8_t* block_keep,
                               float* accept_pair, float* tau_pair, float* accept_rows,
@@ -238,13 +265,22 @@ cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_r
 cudaError_t launch_conf_grad(int64_t R, const float* confidence_logits, float conf_alpha,
                              const float* grad_scale, const WsView& ws, float* dconf,
                              cudaStream_t s);
-cudaError_t launch_bwd_stream(int dtype, bool zf32, bool has_target, const SweepArgs& a, int64_t R,
-                              cudaStream_t s);
+cudaError_t launch_bwd_stream(int kind, bool has_target, const SweepArgs& a, int64_t R, cudaStream_t s);
 // Markov embeddings (both copies) and confidence logits
 cudaError_t launch_heads_prep(const HeadsArgs& a, cudaStream_t s);
 // corrected rows ws.z = base + E.W2^T (compact, FP32) on the tensor cores
 cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s);
 // dE, dW1, dW2, dconf_w, dconf_b, dhidden from dlogits and the saved dL/dc
 cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s);
+// Teacher from hidden states: gather of the supervised rows' hidden states, then the
+// FP32 teacher rows of supervised-list positions [row0, row0 + chunk rows).
+struct TeacherArgs {
+  int64_t R, V, Ht;
+  const uint16_t* hidden;    // bf16 [R][Ht]
+  const uint16_t* lm_head;   // bf16 [V][Ht]
+  WsView ws;
+};
+cudaError_t launch_gather_hidden(const TeacherArgs& a, cudaStream_t s);
+cudaError_t launch_teacher_chunk(const TeacherArgs& a, int64_t row0, cudaStream_t s);
 
 }  // namespace dspark

@@ -80,8 +80,8 @@ __device__ __forceinline__ void warp_lse_merge(float& m, float& s) {
   m = M;
 }
 
-// One group of EPV draft values (16 bytes of T-sized teacher values) in the draft's own
-// type: 16 bytes, or 32 bytes when FP32 draft rows meet a 16-bit output type.
+// One group of EPV values (one 16-byte vector of the output type) in the row's own
+// type: 16 bytes, or 32 bytes when FP32 rows meet a 16-bit output type.
 template <typename TZ, int EPV>
 __device__ __forceinline__ void load_group(const uint8_t* p, float* f) {
   if constexpr (sizeof(TZ) * EPV == 16) {
@@ -114,14 +114,19 @@ struct Ctrl {
 // landing buffer and two teacher buffers: the next row's copy is issued as soon as
 // the current draft segment is in registers, one full row ahead of its use.
 // TZ is the draft rows' type (the logits type, or FP32 corrected rows of the Markov
-// head); T is the type of the teacher and of the dlogits.
-template <typename TZ, typename T, int CL, int NT, int NV, bool HAS_T>
+// head); TT the teacher rows' type (the logits type, or FP32 rows of the teacher
+// computed from hidden states); TO the type of the dlogits.  A launch covers the
+// supervised rows of positions [row0, row1) in the supervised list.
+template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T>
 __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
-  constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int EPV = VecTraits<TO>::EPV;
   constexpr int ZB = EPV * int(sizeof(TZ));  // bytes of one draft group
-  // FP32 rows under 16-bit outputs only come from the Markov head (compact rows,
-  // valid-slot mask); the other builds carry none of that code
-  constexpr bool kMarkov = sizeof(TZ) == 4 && sizeof(T) == 2;
+  constexpr int TB = EPV * int(sizeof(TT));  // bytes of one teacher group
+  // FP32 rows under 16-bit outputs only come from the heads (compact corrected rows
+  // with their valid-slot mask; compact teacher chunks); the other builds carry none
+  // of that code
+  constexpr bool kMarkov = sizeof(TZ) == 4 && sizeof(TO) == 2;
+  constexpr bool kTChunk = sizeof(TT) == 4 && sizeof(TO) == 2;
   constexpr int NE = NV * EPV;
   constexpr int NW = NT / 32;
   static_assert(NW <= 32 && CL <= 16, "control block sizes");
@@ -132,21 +137,21 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t rank = cluster_ctarank();
   const uint32_t cid = cluster_id_x();
   const uint32_t G = nclusters_x();
-  const uint32_t seg_bytes = uint32_t(a.seg_vec) * 16u;          // teacher segment
+  const uint32_t seg_bytes = uint32_t(a.seg_vec) * uint32_t(TB);   // teacher segment
   const uint32_t zseg_bytes = uint32_t(a.seg_vec) * uint32_t(ZB);  // draft segment
   // buffers: HAS_T: [draft][teacher 0][teacher 1]; else [draft 0][draft 1]
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + (HAS_T ? size_t(zseg_bytes) + 2 * size_t(seg_bytes)
                                                       : 2 * size_t(zseg_bytes)));
   auto zbuf = [&](int j) -> uint8_t* { return HAS_T ? smem : smem + size_t(j & 1) * zseg_bytes; };
   auto tbuf = [&](int j) -> uint8_t* {
-    if constexpr (ZB == 16) return smem + size_t(1 + (j & 1)) * seg_bytes;  // zseg == seg
+    if constexpr (ZB == TB) return smem + size_t(1 + (j & 1)) * seg_bytes;  // zseg == seg
     else return smem + zseg_bytes + size_t(j & 1) * seg_bytes;
   };
   WsHeader* hdr = a.ws.hdr;
 
   const int v0 = int(rank) * a.seg_vec;
   const int nvec = max(0, min(a.seg_vec, a.vvec - v0));
-  const uint32_t bytes = uint32_t(nvec) * 16u;
+  const uint32_t bytes = uint32_t(nvec) * uint32_t(TB);
   const uint32_t zbytes = uint32_t(nvec) * uint32_t(ZB);
   const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
   const uint8_t* target = static_cast<const uint8_t*>(a.target);
@@ -160,15 +165,16 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
   auto issue = [&](int j) {  // thread 0: stream row j's segment (draft and teacher)
     const uint32_t bar = (j & 1) ? bar_d1 : bar_d0;
-    const int64_t sidx = cid + int64_t(j) * G;
+    const int64_t sidx = a.row0 + cid + int64_t(j) * G;
     const int64_t row = a.ws.sup_list[sidx];
     const int64_t drow = (kMarkov && a.draft_compact) ? sidx : row;  // compact corrected rows
+    const int64_t trow = (kTChunk && a.target_compact) ? sidx - a.row0 : row;  // teacher chunk
     mbar_arrive_expect_tx(bar, zbytes + (HAS_T ? bytes : 0u));
-    if (bytes) {
+    if (zbytes) {
       bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(drow) * a.ld_d + size_t(v0) * EPV) * sizeof(TZ),
                zbytes, bar, policy);
       if constexpr (HAS_T)
-        bulk_g2s(smem_u32(tbuf(j)), target + (size_t(row) * a.ld_t + size_t(v0) * EPV) * sizeof(T),
+        bulk_g2s(smem_u32(tbuf(j)), target + (size_t(trow) * a.ld_t + size_t(v0) * EPV) * sizeof(TT),
                  bytes, bar, policy);
     }
   };
@@ -187,8 +193,9 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   cluster_sync();
   // the mask prologue has finished and its writes are visible past this point
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int n_sup = hdr->n_sup;
-  const int n_zero = hdr->n_zero;
+  // this launch's supervised rows: list positions [row0, min(row1, n_sup))
+  const int n_sup = max(0, min(hdr->n_sup, a.row1) - a.row0);
+  const int n_zero = a.do_zero ? hdr->n_zero : 0;
   const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
   const float g = a.grad_scale ? *a.grad_scale : 1.f;
   // this cluster's share of zero rows, written a slice after each supervised row
@@ -202,7 +209,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
       const int v = q - rk * nvec;
       const int64_t zr = a.ws.zero_list[zfirst + size_t(rk) * G];
       *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.dlogits) +
-                                (size_t(zr) * a.ld_g + size_t(v0 + v) * EPV) * sizeof(T)) = make_uint4(0u, 0u, 0u, 0u);
+                                (size_t(zr) * a.ld_g + size_t(v0 + v) * EPV) * sizeof(TO)) = make_uint4(0u, 0u, 0u, 0u);
     }
   };
   if (tid == 0) {
@@ -211,7 +218,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   }
 
   // per-row scalars, loaded one row ahead
-  int64_t row = my_n > 0 ? a.ws.sup_list[cid] : 0;
+  int64_t row = my_n > 0 ? a.ws.sup_list[a.row0 + cid] : 0;
   int64_t tok = my_n > 0 ? a.tids[row] : 0;
   float wr = my_n > 0 ? a.ws.w[row] : 0.f;
 
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     int64_t nrow = 0, ntok = 0;
     float nw = 0.f;
     if (j + 1 < my_n) {
-      nrow = a.ws.sup_list[cid + size_t(j + 1) * G];
+      nrow = a.ws.sup_list[a.row0 + cid + size_t(j + 1) * G];
       ntok = a.tids[nrow];
       nw = a.ws.w[nrow];
     }
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         const int v = tid + i * NT;
         if (v < nvec) {
           float t8[EPV];
-          unpack16<T>(*reinterpret_cast<const uint4*>(tb + size_t(v) * 16), t8);
+          load_group<TT, EPV>(tb + size_t(v) * TB, t8);
 #pragma unroll
           for (int e = 0; e < EPV; e += 2) mt = fmax3(mt, t8[e], t8[e + 1]);
         }
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         const int v = tid + i * NT;
         if (v < nvec) {
           float t8[EPV];
-          unpack16<T>(*reinterpret_cast<const uint4*>(tb + size_t(v) * 16), t8);
+          load_group<TT, EPV>(tb + size_t(v) * TB, t8);
 #pragma unroll
           for (int e = 0; e < EPV; ++e) st += ex2(fmaf(t8[e], kLog2e, -ot));
         }
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         const int v = tid + i * NT;
         if (v < nvec) {
           float t8[EPV];
-          unpack16<T>(*reinterpret_cast<const uint4*>(tb + size_t(v) * 16), t8);
+          load_group<TT, EPV>(tb + size_t(v) * TB, t8);
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
             const float q = __fmul_rn(ex2(fmaf(t8[e], kLog2e, -ot)), at);
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
       const float gw = zero_out ? 0.f : g * wr;
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
       const float k0 = cce - cl1 * S;
-      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(T);
+      uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(TO);
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int v = tid + i * NT;
@@ -411,7 +418,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
             for (int e = 0; e < EPV; ++e)
               if (e == te) o[e] -= cce;
           }
-          *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<T>(o);
+          *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<TO>(o);
         }
       }
     }
@@ -426,7 +433,9 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   __syncthreads();
   cluster_sync();
 
-  // ---- the last CTA to finish writes the per-row epilogue and the report
+  // ---- the last CTA to finish writes the per-row epilogue and the report (in the
+  // launch that covers the last rows)
+  if (!a.do_final) return;
   if (tid == 0) {
     __threadfence();
     ctrl->last = atomicAdd(&hdr->done, 1u) == gridDim.x - 1;
@@ -451,27 +460,27 @@ struct LaunchCache {
   int clusters = 0;
 };
 
-template <typename TZ, typename T, int CL>
+template <typename TZ, typename TT, typename TO, int CL>
 size_t smem_bytes(int64_t V, bool has_t) {
-  constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int EPV = VecTraits<TO>::EPV;
   const int64_t vvec = V / EPV;
   const int64_t seg_vec = (vvec + CL - 1) / CL;
-  const size_t zseg = size_t(seg_vec) * EPV * sizeof(TZ), tseg = size_t(seg_vec) * 16;
+  const size_t zseg = size_t(seg_vec) * EPV * sizeof(TZ), tseg = size_t(seg_vec) * EPV * sizeof(TT);
   return (has_t ? zseg + 2 * tseg : 2 * zseg) + sizeof(Ctrl);
 }
 
-template <typename TZ, typename T, int CL, int NT, int NV, bool HAS_T>
+template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T>
 cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
-  constexpr int EPV = VecTraits<T>::EPV;
+  constexpr int EPV = VecTraits<TO>::EPV;
   SweepArgs a = a0;
   a.vvec = int32_t(a.V / EPV);
   a.seg_vec = (a.vvec + CL - 1) / CL;
   a.nbuf = 2;
   // at least the report's reduction scratch (reused at the end)
-  const size_t smem = std::max<size_t>(smem_bytes<TZ, T, CL>(a.V, HAS_T), size_t(NT / 32) * kNAcc * sizeof(double));
+  const size_t smem = std::max<size_t>(smem_bytes<TZ, TT, TO, CL>(a.V, HAS_T), size_t(NT / 32) * kNAcc * sizeof(double));
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
-  auto kern = sweep_kernel<TZ, T, CL, NT, NV, HAS_T>;
+  auto kern = sweep_kernel<TZ, TT, TO, CL, NT, NV, HAS_T>;
   static LaunchCache cache;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -535,59 +544,66 @@ struct Build {
 constexpr int kNumBuilds = 5;
 constexpr Build kBf16Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {4, 512, 10}, {8, 512, 5}};
 constexpr Build kF32Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 8}, {8, 512, 10}, {16, 512, 5}};
-// FP32 corrected draft rows with bf16 teacher and dlogits (Markov head)
-constexpr Build kZf32Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}, {8, 512, 5}};
+// FP32 draft or teacher rows of the heads with bf16 dlogits
+constexpr Build kHeadBuilds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}, {8, 512, 5}};
 
-template <typename TZ, typename T>
+using bf16 = __nv_bfloat16;
+
+template <typename TZ, typename TT, typename TO>
 size_t smem_for(int cl, int64_t V, bool has_t) {
   switch (cl) {
-    case 1: return smem_bytes<TZ, T, 1>(V, has_t);
-    case 2: return smem_bytes<TZ, T, 2>(V, has_t);
-    case 4: return smem_bytes<TZ, T, 4>(V, has_t);
-    case 8: return smem_bytes<TZ, T, 8>(V, has_t);
-    default: return smem_bytes<TZ, T, 16>(V, has_t);
+    case 1: return smem_bytes<TZ, TT, TO, 1>(V, has_t);
+    case 2: return smem_bytes<TZ, TT, TO, 2>(V, has_t);
+    case 4: return smem_bytes<TZ, TT, TO, 4>(V, has_t);
+    case 8: return smem_bytes<TZ, TT, TO, 8>(V, has_t);
+    default: return smem_bytes<TZ, TT, TO, 16>(V, has_t);
   }
 }
 
-// zf32: FP32 draft rows (dtype then names the teacher / dlogits type, bf16 only)
-int pick_build(int dtype, bool zf32, int64_t V, bool has_t) {
-  if (zf32 && dtype != DSPARK_BF16) return -1;
-  const Build* b = zf32 ? kZf32Builds : (dtype == DSPARK_BF16 ? kBf16Builds : kF32Builds);
-  const int epv = dtype == DSPARK_BF16 ? 8 : 4;
+size_t kind_smem(int kind, int cl, int64_t V, bool has_t) {
+  switch (kind) {
+    case kSweepBf16: return smem_for<bf16, bf16, bf16>(cl, V, has_t);
+    case kSweepF32: return smem_for<float, float, float>(cl, V, has_t);
+    case kSweepZ32: return smem_for<float, bf16, bf16>(cl, V, has_t);
+    case kSweepT32: return smem_for<bf16, float, bf16>(cl, V, has_t);
+    default: return smem_for<float, float, bf16>(cl, V, has_t);
+  }
+}
+
+int pick_build(int kind, int64_t V, bool has_t) {
+  const Build* b = kind == kSweepBf16 ? kBf16Builds : (kind == kSweepF32 ? kF32Builds : kHeadBuilds);
+  const int epv = kind == kSweepF32 ? 4 : 8;
   for (int i = 0; i < kNumBuilds; ++i) {
     if (int64_t(b[i].cl) * b[i].nt * b[i].nv * epv < V) continue;
-    const size_t sm = zf32 ? smem_for<float, __nv_bfloat16>(b[i].cl, V, has_t)
-                           : (dtype == DSPARK_BF16 ? smem_for<__nv_bfloat16, __nv_bfloat16>(b[i].cl, V, has_t)
-                                                   : smem_for<float, float>(b[i].cl, V, has_t));
-    if (sm <= kMaxSmem) return i;
+    if (kind_smem(kind, b[i].cl, V, has_t) <= kMaxSmem) return i;
   }
   return -1;
 }
 
-template <typename TZ, typename T, bool HT>
+template <typename TZ, typename TT, typename TO, bool HT>
 cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
-  if constexpr (sizeof(TZ) == 4 && sizeof(T) == 2) {
+  if constexpr (sizeof(TZ) == 4 && sizeof(TO) == 4) {
     switch (i) {
-      case 0: return launch_cfg<TZ, T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<TZ, T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<TZ, T, 4, 512, 4, HT>(a, s);
-      default: return launch_cfg<TZ, T, 8, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 8, HT>(a, s);
+      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 10, HT>(a, s);
+      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 5, HT>(a, s);
     }
-  } else if constexpr (sizeof(T) == 2) {
+  } else if constexpr (sizeof(TZ) == 2 && sizeof(TT) == 2) {
     switch (i) {
-      case 0: return launch_cfg<TZ, T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<TZ, T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<TZ, T, 4, 512, 4, HT>(a, s);
-      case 3: return launch_cfg<TZ, T, 4, 512, 10, HT>(a, s);
-      case 4: return launch_cfg<TZ, T, 8, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT>(a, s);
+      case 3: return launch_cfg<TZ, TT, TO, 4, 512, 10, HT>(a, s);
+      case 4: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT>(a, s);
     }
   } else {
     switch (i) {
-      case 0: return launch_cfg<TZ, T, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<TZ, T, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<TZ, T, 4, 512, 8, HT>(a, s);
-      case 3: return launch_cfg<TZ, T, 8, 512, 10, HT>(a, s);
-      case 4: return launch_cfg<TZ, T, 16, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT>(a, s);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT>(a, s);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT>(a, s);
+      default: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT>(a, s);
     }
   }
   return cudaErrorInvalidValue;
@@ -595,31 +611,46 @@ cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool sweep_supported(int dtype, bool zf32, int64_t V, bool has_target) {
-  return pick_build(dtype, zf32, V, has_target) >= 0;
-}
+bool sweep_supported(int kind, int64_t V, bool has_target) { return pick_build(kind, V, has_target) >= 0; }
 
-cudaError_t launch_sweep(int dtype, bool zf32, bool has_target, const SweepArgs& a, cudaStream_t s) {
-  const int i = pick_build(dtype, zf32, a.V, has_target);
+cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s) {
+  const int i = pick_build(kind, a.V, has_target);
   if (i < 0) return cudaErrorInvalidValue;
-  if (zf32)
-    return has_target ? dispatch<float, __nv_bfloat16, true>(i, a, s) : dispatch<float, __nv_bfloat16, false>(i, a, s);
-  if (dtype == DSPARK_BF16)
-    return has_target ? dispatch<__nv_bfloat16, __nv_bfloat16, true>(i, a, s)
-                      : dispatch<__nv_bfloat16, __nv_bfloat16, false>(i, a, s);
-  return has_target ? dispatch<float, float, true>(i, a, s) : dispatch<float, float, false>(i, a, s);
+  switch (kind) {
+    case kSweepBf16:
+      return has_target ? dispatch<bf16, bf16, bf16, true>(i, a, s) : dispatch<bf16, bf16, bf16, false>(i, a, s);
+    case kSweepF32:
+      return has_target ? dispatch<float, float, float, true>(i, a, s) : dispatch<float, float, float, false>(i, a, s);
+    case kSweepZ32:
+      return has_target ? dispatch<float, bf16, bf16, true>(i, a, s) : dispatch<float, bf16, bf16, false>(i, a, s);
+    case kSweepT32:
+      return dispatch<bf16, float, bf16, true>(i, a, s);
+    case kSweepZT32:
+      return dispatch<float, float, bf16, true>(i, a, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 // ------------------------------------------------------- backward-only stream
 // dlogits from saved row statistics: one more read of the logits, no reductions.
-template <typename TZ, typename T, bool HAS_T>
-__global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a, const int64_t R) {
-  constexpr int EPV = VecTraits<T>::EPV;
+// Covers the supervised rows of list positions [row0, row1) and, with do_zero, the
+// unsupervised rows.
+template <typename TZ, typename TT, typename TO, bool HAS_T>
+__global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a) {
+  constexpr int EPV = VecTraits<TO>::EPV;
   constexpr int ZB = EPV * int(sizeof(TZ));
+  constexpr int TB = EPV * int(sizeof(TT));
+  constexpr bool kMarkov = sizeof(TZ) == 4 && sizeof(TO) == 2;
+  constexpr bool kTChunk = sizeof(TT) == 4 && sizeof(TO) == 2;
   const int vvec = int(a.V / EPV);
-  for (int64_t row = blockIdx.y; row < R; row += gridDim.y) {
-    uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * a.ld_g * sizeof(T);
-    const bool zero_row = a.ws.m[row] == 0 || (a.invalid_zero && a.valid != nullptr && a.valid[row] == 0);
+  const int n_sup = max(0, min(a.ws.hdr->n_sup, a.row1) - a.row0);
+  const int n_zero = a.do_zero ? a.ws.hdr->n_zero : 0;
+  for (int idx = blockIdx.y; idx < n_sup + n_zero; idx += gridDim.y) {
+    const bool unsup = idx >= n_sup;
+    const int64_t sidx = int64_t(a.row0) + idx;
+    const int64_t row = unsup ? a.ws.zero_list[idx - n_sup] : a.ws.sup_list[sidx];
+    uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * a.ld_g * sizeof(TO);
+    const bool zero_row = unsup || (kMarkov && a.invalid_zero && a.valid[row] == 0);
     if (zero_row) {
       for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x)
         *reinterpret_cast<uint4*>(out + size_t(v) * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -633,13 +664,14 @@ __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a, cons
     const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S), kzero = cce - cl1 * S;
     const float lz2 = st[kStLseD] * kLog2e, lt2 = st[kStLseT] * kLog2e;
     const int64_t tok = a.tids[row];
-    const int64_t drow = a.draft_compact ? int64_t(a.ws.sup_index[row]) : row;
+    const int64_t drow = (kMarkov && a.draft_compact) ? sidx : row;
+    const int64_t trow = (kTChunk && a.target_compact) ? int64_t(idx) : row;
     const uint8_t* zr = static_cast<const uint8_t*>(a.draft) + size_t(drow) * a.ld_d * sizeof(TZ);
-    const uint8_t* tr = static_cast<const uint8_t*>(a.target) + size_t(row) * a.ld_t * sizeof(T);
+    const uint8_t* tr = static_cast<const uint8_t*>(a.target) + size_t(trow) * a.ld_t * sizeof(TT);
     for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x) {
       float z[EPV], t[EPV], o[EPV];
       load_group<TZ, EPV>(zr + size_t(v) * ZB, z);
-      if constexpr (HAS_T) unpack16<T>(*reinterpret_cast<const uint4*>(tr + size_t(v) * 16), t);
+      if constexpr (HAS_T) load_group<TT, EPV>(tr + size_t(v) * TB, t);
 #pragma unroll
       for (int e = 0; e < EPV; ++e) {
         const float p = ex2(fmaf(z[e], kLog2e, -lz2));
@@ -651,26 +683,37 @@ __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a, cons
         }
         if (int64_t(v) * EPV + e == tok) o[e] -= cce;
       }
-      *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<T>(o);
+      *reinterpret_cast<uint4*>(out + size_t(v) * 16) = pack16<TO>(o);
     }
   }
 }
 
-cudaError_t launch_bwd_stream(int dtype, bool zf32, bool has_target, const SweepArgs& a, int64_t R,
-                              cudaStream_t s) {
-  const int epv = dtype == DSPARK_BF16 ? 8 : 4;
+cudaError_t launch_bwd_stream(int kind, bool has_target, const SweepArgs& a, int64_t R, cudaStream_t s) {
+  const int epv = kind == kSweepF32 ? 4 : 8;
   const int64_t vvec = a.V / epv;
   const unsigned gx = unsigned(std::min<int64_t>((vvec + 1023) / 1024, 64));
-  dim3 grid(gx > 0 ? gx : 1, unsigned(std::min<int64_t>(R, 65535)), 1);
-  if (zf32) {
-    if (has_target) bwd_stream_kernel<float, __nv_bfloat16, true><<<grid, 256, 0, s>>>(a, R);
-    else bwd_stream_kernel<float, __nv_bfloat16, false><<<grid, 256, 0, s>>>(a, R);
-  } else if (dtype == DSPARK_BF16) {
-    if (has_target) bwd_stream_kernel<__nv_bfloat16, __nv_bfloat16, true><<<grid, 256, 0, s>>>(a, R);
-    else bwd_stream_kernel<__nv_bfloat16, __nv_bfloat16, false><<<grid, 256, 0, s>>>(a, R);
-  } else {
-    if (has_target) bwd_stream_kernel<float, float, true><<<grid, 256, 0, s>>>(a, R);
-    else bwd_stream_kernel<float, float, false><<<grid, 256, 0, s>>>(a, R);
+  dim3 grid(gx > 0 ? gx : 1, unsigned(std::max<int64_t>(1, std::min<int64_t>(R, 65535))), 1);
+  switch (kind) {
+    case kSweepBf16:
+      if (has_target) bwd_stream_kernel<bf16, bf16, bf16, true><<<grid, 256, 0, s>>>(a);
+      else bwd_stream_kernel<bf16, bf16, bf16, false><<<grid, 256, 0, s>>>(a);
+      break;
+    case kSweepF32:
+      if (has_target) bwd_stream_kernel<float, float, float, true><<<grid, 256, 0, s>>>(a);
+      else bwd_stream_kernel<float, float, float, false><<<grid, 256, 0, s>>>(a);
+      break;
+    case kSweepZ32:
+      if (has_target) bwd_stream_kernel<float, bf16, bf16, true><<<grid, 256, 0, s>>>(a);
+      else bwd_stream_kernel<float, bf16, bf16, false><<<grid, 256, 0, s>>>(a);
+      break;
+    case kSweepT32:
+      bwd_stream_kernel<bf16, float, bf16, true><<<grid, 256, 0, s>>>(a);
+      break;
+    case kSweepZT32:
+      bwd_stream_kernel<float, float, bf16, true><<<grid, 256, 0, s>>>(a);
+      break;
+    default:
+      return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }

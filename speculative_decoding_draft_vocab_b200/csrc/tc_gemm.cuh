@@ -104,9 +104,21 @@ constexpr size_t gemm_smem_bytes() {
   return size_t(STAGES) * (BM * BK * 2 + BN * BK * 2) + 1024 + 256;
 }
 
-// Work item w -> (m-tile, n-tile, k-split) and its range of 64-wide K chunks.
+// Work item w -> (m-tile, n-tile, k-split) and its range of 64-wide K chunks.  The
+// m-tile is the slowest index, so with a device-side row bound (rows m_base + m at or
+// past *m_bound are not needed) the needed items are exactly the first items().
 struct WorkMap {
   int m_tiles, n_tiles, ksplit, kchunks;
+  const int32_t* m_bound;
+  int m_base;
+  __device__ __forceinline__ int items() const {
+    int mt = m_tiles;
+    if (m_bound != nullptr) {
+      const int rem = *m_bound - m_base;
+      mt = rem <= 0 ? 0 : min(m_tiles, (rem + BM - 1) / BM);
+    }
+    return mt * n_tiles * ksplit;
+  }
   __device__ __forceinline__ void decode(int w, int& mt, int& nt, int& s, int& kc0, int& kc1) const {
     s = w % ksplit;
     const int t = w / ksplit;
@@ -137,7 +149,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int W = wm.m_tiles * wm.n_tiles * wm.ksplit;
+  const int W = wm.items();  // the same in every role
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

@@ -54,11 +54,15 @@ inline int sm_count() {
 }
 
 // D[M, N] = A . B^T over K (A is M x K, B is N x K in the math), operands as described
-// by their tensor maps; work split into `ksplit` slices of K.  Returns the launch error.
+// by their tensor maps; work split into `ksplit` slices of K.  With `m_bound`, rows m
+// with m_base + m >= *m_bound (a count the device holds) are skipped.  Returns the
+// launch error.
 template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi>
 cudaError_t gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int ksplit, const Epi& epi,
-                 uint32_t* status, cudaStream_t s) {
+                 uint32_t* status, cudaStream_t s, const int32_t* m_bound = nullptr, int m_base = 0) {
   WorkMap wm;
+  wm.m_bound = m_bound;
+  wm.m_base = m_base;
   wm.m_tiles = (M + BM - 1) / BM;
   wm.n_tiles = (N + BN - 1) / BN;
   wm.kchunks = (K + BK - 1) / BK;

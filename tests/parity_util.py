@@ -13,6 +13,15 @@ Tolerances (fixed for the whole suite):
     sub-gradient there); plus a per-row relative L2 error <= 2e-3 against the same
     rounded row ref_o.  (Against the unrounded row, bf16 rounding alone reaches
     2.5e-3 on rows whose mass sits in a few elements: a half-ulp is 2^-9.)
+Head weight gradients (dW2 = sum_r dz_r (x) e_r, dE_r = W2^T dz_r, hence dW1) are
+contracted on the tensor cores from the bf16 dlogits, so they carry the bf16 rounding
+of dz (unit roundoff u = 2^-8, one rounding per element, independent across elements):
+the error of a sum of rounded products has standard deviation at most
+u/sqrt(3) * sqrt(sum_k (dz_k x_k)^2), and check_heads allows 4u times that root-sum-
+square (about seven standard deviations) plus 1e-5 of the magnitude for FP32
+accumulation.  Where some row's sign(p_j - q_j) is undecided at FP32 precision, every
+sub-gradient of |p_j - q_j| is valid: the oracle reports the width of that interval of dz
+(``dlogit_swing``), and the bounds add its contraction with |e| (or |W2|).
 """
 
 from __future__ import annotations
@@ -133,3 +142,118 @@ def compare(inp, call, ref, dlogit_rows=None, check_rows=True):
         if bool(msk.any()):
             assert bool((g[msk] == 0).all())
     return n_amb
+
+
+U_BF16 = 2.0 ** -8
+
+
+def _live_rows(inp, ref):
+    valid = np32(inp.valid).reshape(-1)
+    sup = ref["rows"]
+    return np.array([int(r) for r in sup if valid[r] != 0], dtype=np.int64)
+
+
+def check_heads(inp, call, ref, mode, elementwise=True):
+    """Confidence logits, dL/dc and the head weight gradients of a finished call.
+
+    dW2 and dW1 are checked element-wise against the bound derived in the module
+    docstring when the oracle returned every supervised row's dlogits, and in every case
+    in Frobenius norm against the aggregate of that bound (the same sum of independent
+    rounding errors: its Frobenius norm is about u/sqrt(3) times that of the
+    root-sum-squares; u times it is allowed), plus the width of the valid sub-gradients
+    where sign(p - q) is undecided (``dlogit_swing``; changing one s_j also moves S, so
+    every other element can move by up to p_k times the same width: a second term of
+    the same size)."""
+    out = call.out
+    R = inp.R
+    u = U_BF16
+    valid = np32(inp.valid).reshape(-1)
+    # confidence logits of every row (0 on invalid slots)
+    if inp.conf_w is not None:
+        c = out.conf_rows.cpu().double().numpy()
+        np.testing.assert_allclose(c, ref["conf"], rtol=1e-4, atol=1e-5)
+    np.testing.assert_allclose(out.dconf.cpu().double().numpy(), ref["dconf"], rtol=1e-4, atol=2e-6)
+    live = _live_rows(inp, ref)
+    stats = {}
+    if inp.markov_w2 is not None:
+        w2 = np32(inp.markov_w2).astype(np.float64)
+        rank = w2.shape[1]
+        prev = np32(inp.prev_ids).reshape(-1).astype(np.int64)
+        e_live = O.markov_embedding(prev[live], np32(inp.markov_w1)) if len(live) else np.zeros((0, rank))
+        e_norm = np.linalg.norm(e_live, axis=1)
+        w2_colmax = np.abs(w2).max(0)                  # [rank]
+        w2_rowmax = np.linalg.norm(w2, axis=1).max()   # max_j ||W2_j||
+        nz2, swt = ref["dz_norm2"][live], ref["swing_sum"][live]
+        proj_e = None
+        if inp.conf_w is not None and inp.conf_with_markov:
+            proj_e = np32(inp.conf_w).reshape(-1).astype(np.float64)[inp.draft_hidden.shape[-1]:]
+        # ---- dW2 = sum_r dz_r (x) e_r
+        got = out.dW2.cpu().double().numpy()
+        want = ref["dW2"]
+        agg = u * np.sqrt(np.sum(nz2 * e_norm ** 2)) + 2 * np.sum(swt * e_norm) + 1e-5 * np.linalg.norm(want)
+        err_f = np.linalg.norm(got - want)
+        assert err_f <= agg, f"dW2 Frobenius error {err_f:.3e} > {agg:.3e}"
+        stats["dW2_frob_err"] = err_f / max(agg, 1e-30)
+        if elementwise:
+            Dz = np.stack([ref["dlogits"][int(r)] for r in live]) if len(live) else np.zeros((0, inp.V))
+            Sw = np.stack([ref["dlogit_swing"][int(r)] for r in live]) if len(live) else np.zeros((0, inp.V))
+            bound = (4 * u * np.sqrt((Dz ** 2).T @ (e_live ** 2)) + Sw.T @ np.abs(e_live)
+                     + (swt[:, None] * np.abs(e_live)).sum(0)[None, :] + 1e-5 * np.abs(want)
+                     + 1e-7 * np.abs(want).max())
+            bad = np.abs(got - want) > bound
+            assert not bad.any(), f"dW2: {int(bad.sum())} entries off; worst {np.max(np.abs(got - want) - bound)}"
+        # ---- dW1[id] = sum over rows with that previous id of dE_r = W2^T dz_r + dc_r proj_e
+        gotw1 = out.dW1.cpu().double().numpy()
+        ids = sorted(ref["dW1"])
+        touched = np.zeros(gotw1.shape[0], dtype=bool)
+        touched[ids] = True
+        assert np.all(gotw1[~touched] == 0.0), "dW1 rows of untouched ids must stay zero"
+        if ids:
+            want1 = np.stack([ref["dW1"][i] for i in ids])
+            conf_part = 0.0
+            if proj_e is not None:
+                conf_part = 1e-5 * np.sum(np.abs(ref["dconf"][live])) * np.linalg.norm(proj_e)
+            agg1 = (u * w2_rowmax * np.sqrt(np.sum(nz2)) + 2 * w2_rowmax * np.sum(swt) + conf_part
+                    + 1e-5 * np.linalg.norm(want1))
+            err1 = np.linalg.norm(gotw1[ids] - want1)
+            assert err1 <= agg1, f"dW1 Frobenius error {err1:.3e} > {agg1:.3e}"
+            stats["dW1_frob_err"] = err1 / max(agg1, 1e-30)
+        if elementwise and ids:
+            var, extra = {}, {}
+            for i, r in enumerate(live):
+                dz, sw = ref["dlogits"][int(r)], ref["dlogit_swing"][int(r)]
+                pid = int(prev[r])
+                var[pid] = var.get(pid, 0.0) + (dz ** 2) @ (w2 ** 2)
+                x = sw @ np.abs(w2) + swt[i] * w2_colmax
+                if proj_e is not None:
+                    x = x + 1e-5 * np.abs(ref["dconf"][r] * proj_e)
+                extra[pid] = extra.get(pid, 0.0) + x
+            for pid in ids:
+                want_row = ref["dW1"][pid]
+                err = np.abs(gotw1[pid] - want_row)
+                tol = 4 * u * np.sqrt(var[pid]) + extra[pid] + 1e-5 * np.abs(want_row) + 1e-9
+                assert np.all(err <= tol), f"dW1[{pid}]: worst {np.max(err - tol)}"
+    if inp.conf_w is not None:
+        H = inp.draft_hidden.shape[-1]
+        h = np32(inp.draft_hidden).reshape(R, H).astype(np.float64)
+        sup = np.zeros(R, dtype=bool)
+        sup[ref["rows"]] = True
+        dcl = np.where(sup & (valid != 0), ref["dconf"], 0.0)
+        x = h
+        if inp.conf_with_markov:
+            prev = np32(inp.prev_ids).reshape(-1).astype(np.int64)
+            e_all = np.zeros((R, inp.markov_w1.shape[1]))
+            lv = np.nonzero(sup & (valid != 0))[0]
+            e_all[lv] = O.markov_embedding(prev[lv], np32(inp.markov_w1))
+            x = np.concatenate([h, e_all], axis=1)
+        got = out.dconf_w.cpu().double().numpy()
+        tol = 1e-4 * (np.abs(dcl) @ np.abs(x)) + 1e-9
+        assert np.all(np.abs(got - ref["dconf_w"]) <= tol), np.max(np.abs(got - ref["dconf_w"]) - tol)
+        gb = float(out.dconf_b.item())
+        assert abs(gb - ref["dconf_b"]) <= 1e-4 * np.sum(np.abs(dcl)) + 1e-9
+        dh = out.dhidden.float().cpu().double().numpy().reshape(R, H)
+        want = ref["dhidden"]
+        want_o = round_to(want, "bf16")
+        tol = np.maximum(1e-4 * np.abs(want_o), bf16_ulp(want_o)) + 1e-12
+        assert np.all(np.abs(dh - want_o) <= tol)
+    return stats

@@ -206,3 +206,34 @@ def test_markov_workspace_holds_corrected_rows(abi):
     assert n >= base + R * 4096 * 4 + 2 * R * 64 * 2 + R * 64 * 4
     # a workspace sized without the head is refused for a problem with it
     assert _fwd(abi, p, _params(abi), ws_bytes=base) == abi.DSPARK_ERR_WORKSPACE
+
+
+def _with_lm_head(abi, p, Ht=256):
+    p.target_logits = None
+    p.target_hidden = ctypes.c_void_p(0xf0000)
+    p.lm_head = ctypes.c_void_p(0x100000)
+    p.target_hidden_size = Ht
+    return p
+
+
+def test_teacher_from_hidden_validation_and_workspace(abi):
+    prm = _params(abi)
+    # FP32 logits are not paired with the tensor-core teacher
+    assert _fwd(abi, _with_lm_head(abi, _problem(abi, dtype=abi.DSPARK_F32)), prm) == abi.DSPARK_ERR_UNSUPPORTED
+    assert _fwd(abi, _with_lm_head(abi, _problem(abi), Ht=100), prm) == abi.DSPARK_ERR_ALIGNMENT
+    p = _with_lm_head(abi, _problem(abi))
+    p.lm_head = None
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    # teacher logits and teacher hidden states together are ambiguous
+    p = _with_lm_head(abi, _problem(abi))
+    p.target_logits, p.target_ld = ctypes.c_void_p(0x20000), p.V
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    # the workspace holds the gathered hidden rows and one FP32 chunk of teacher rows
+    for B, N, K in ((1, 2, 4), (8, 16, 8)):
+        p = _problem(abi, V=4096)
+        p.B, p.N, p.K = B, N, K
+        base = abi.dspark_workspace_size(ctypes.byref(p))
+        n = abi.dspark_workspace_size(ctypes.byref(_with_lm_head(abi, p, Ht=256)))
+        R = B * N * K
+        assert n >= base + R * 256 * 2 + min(R, 512) * 4096 * 4
+        assert n < base + R * 256 * 2 + min(R, 512) * 4096 * 4 + 4096

@@ -12,6 +12,7 @@ import math
 import os
 
 import numpy as np
+import scipy.special
 import pytest
 
 from oracle import dspark_oracle as O
@@ -441,3 +442,26 @@ def test_planted_mistakes(monkeypatch, target, mutant, pins):
         except AssertionError:
             failed += 1
     assert failed >= 1
+
+
+def test_subgradient_swing_on_ties_and_none_elsewhere():
+    """Identical draft and teacher rows tie on every element: each |p_j - q_j| takes any
+    sub-gradient in [-1, 1], so the valid dz_j span 2 g w l1_alpha p_j with p the plain
+    softmax; rows far from ties have no such interval, and the per-row sums agree."""
+    rng = np.random.default_rng(21)
+    B, N, K, V = 1, 2, 3, 50
+    d = rng.normal(0, 2, (B, N, K, V))
+    ev = np.ones((B, N, K), dtype=np.int64)
+    ids = rng.integers(0, V, (B, N, K))
+    res = O.dspark_loss(d, ids, ev, target_logits=d.copy(), grad_scale=0.6, l1_alpha=0.9, gamma=4.0)
+    for r, sw in res["dlogit_swing"].items():
+        k = r % K
+        p = scipy.special.softmax(d.reshape(-1, V)[r])
+        np.testing.assert_allclose(sw, 2 * 0.6 * np.exp(-k / 4.0) * 0.9 * p, rtol=1e-12)
+        assert abs(res["swing_sum"][r] - sw.sum()) < 1e-12
+        assert abs(res["dz_norm2"][r] - np.dot(res["dlogits"][r], res["dlogits"][r])) < 1e-15
+    # a teacher far from the draft: no undecided signs
+    t = d + rng.normal(0, 1, d.shape)
+    res = O.dspark_loss(d, ids, ev, target_logits=t)
+    assert all(not sw.any() for sw in res["dlogit_swing"].values())
+    assert np.all(res["swing_sum"] == 0.0)
