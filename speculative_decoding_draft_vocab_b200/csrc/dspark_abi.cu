@@ -41,6 +41,8 @@ inline WsDims ws_dims(const dspark_problem_t* p) {
     d.rank = p->markov_rank;
     d.splits = heads_splits(d.R, p->V);
   }
+  if (p->conf_w != nullptr || p->draft_hidden != nullptr)
+    d.conf_cols = p->hidden_size + (p->conf_with_markov && d.markov ? p->markov_rank : 0);
   d.lm = lm_present(p) && p->target_logits == nullptr;
   if (d.lm) {
     d.Ht = p->target_hidden_size;

@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(256) heads_prep_kernel(const HeadsArgs a) {
       float hdot = 0.f;
       if (valid) {
         const uint16_t* h = a.hidden + size_t(r) * a.H;
+#pragma unroll 4
         for (int j = lane * 8; j < a.H; j += 256) {
           const uint4 q = *reinterpret_cast<const uint4*>(h + j);
           const uint4 w = *reinterpret_cast<const uint4*>(a.conf_w + j);
@@ -73,6 +74,8 @@ __global__ void __launch_bounds__(256) heads_prep_kernel(const HeadsArgs a) {
 }
 
 // ---- epilogue of the bias GEMM: corrected row z = base + E.W2^T (compact rows)
+// (epilogue functors get a 32 x 32 block of the accumulator, rows m0.., columns n0..,
+// element (r, j) at t[r * tc::kTileLd + j]; lane j handles column n0 + j of every row)
 struct BiasEpi {
   const int32_t* sup_list;
   const WsHeader* hdr;
@@ -83,16 +86,32 @@ struct BiasEpi {
   float* z;
   int64_t ldz;
   int V;
-  __device__ void operator()(int m, int n, int /*split*/, const float* v) const {
-    if (m >= hdr->n_sup) return;
-    const int64_t row = sup_list[m];
-    const bool ok = valid[row] != 0;
-    const uint16_t* b = base + size_t(row) * ld_base;
-    float* out = z + size_t(m) * ldz;
+  // lane l: the id of row m0 + l (low 32 bits) and its valid flag (bit 32); bit 33
+  // set past the last supervised row
+  __device__ uint64_t row_state(int m0, int lane) const {
+    const int m = m0 + lane;
+    if (m >= hdr->n_sup) return uint64_t(1) << 33;
+    const int32_t row = sup_list[m];
+    return uint64_t(uint32_t(row)) | (uint64_t(valid[row] != 0) << 32);
+  }
+  __device__ void operator()(int m0, int n0, int /*split*/, const float* t, int lane, uint64_t rs) const {
+    const int c = n0 + lane;
+    const bool col = c < V;
+    // every load of the block before any store (base and z may not alias, but the
+    // compiler cannot know that)
+    float bv[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int c = n + i;
-      if (c < V) out[c] = ok ? bf(b[c]) + v[i] : (invalid_row_mode == 0 ? 0.f : bf(b[c]));
+    for (int r = 0; r < 32; ++r) {
+      const uint64_t q = __shfl_sync(0xffffffffu, rs, r);
+      bv[r] = (col && !(q >> 33)) ? bf(base[size_t(uint32_t(q)) * ld_base + c]) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const uint64_t q = __shfl_sync(0xffffffffu, rs, r);
+      if (col && !(q >> 33)) {
+        const bool ok = (q >> 32) & 1u;
+        z[size_t(m0 + r) * ldz + c] = ok ? bv[r] + t[r * tc::kTileLd + lane] : (invalid_row_mode == 0 ? 0.f : bv[r]);
+      }
     }
   }
 };
@@ -101,12 +120,12 @@ struct BiasEpi {
 struct PartialEpi {
   float* dep;
   int R, rank;
-  __device__ void operator()(int m, int n, int split, const float* v) const {
-    if (m >= R) return;
-    float* out = dep + (size_t(split) * R + m) * rank;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (n + i < rank) out[n + i] = v[i];
+  __device__ uint64_t row_state(int, int) const { return 0; }
+  __device__ void operator()(int m0, int n0, int split, const float* t, int lane, uint64_t) const {
+    const int c = n0 + lane;
+    const int rows = min(32, R - m0);
+    if (c >= rank) return;
+    for (int r = 0; r < rows; ++r) dep[(size_t(split) * R + m0 + r) * rank + c] = t[r * tc::kTileLd + lane];
   }
 };
 
@@ -114,12 +133,19 @@ struct PartialEpi {
 struct WeightEpi {
   float* dw2;
   int V, rank, accumulate;
-  __device__ void operator()(int m, int n, int /*split*/, const float* v) const {
-    if (m >= V) return;
-    float* out = dw2 + size_t(m) * rank;
+  __device__ uint64_t row_state(int, int) const { return 0; }
+  __device__ void operator()(int m0, int n0, int /*split*/, const float* t, int lane, uint64_t) const {
+    const int c = n0 + lane;
+    const int rows = min(32, V - m0);
+    if (c >= rank) return;
+    float prev[32];
+    if (accumulate) {  // every load before any store
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (n + i < rank) out[n + i] = accumulate ? out[n + i] + v[i] : v[i];
+      for (int r = 0; r < 32; ++r) prev[r] = r < rows ? dw2[size_t(m0 + r) * rank + c] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 32; ++r)
+      if (r < rows) dw2[size_t(m0 + r) * rank + c] = (accumulate ? prev[r] : 0.f) + t[r * tc::kTileLd + lane];
   }
 };
 
@@ -141,18 +167,30 @@ __global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const
   }
 }
 
-// ---- dproj = sum_r dc_r [h_r ; e_r] and dbias = sum_r dc_r (fixed row order)
-__global__ void __launch_bounds__(256) dproj_kernel(const HeadsArgs a) {
+// ---- dproj = sum_r dc_r [h_r ; e_r] and dbias = sum_r dc_r: partial sums over blocks
+// of kDprojRows rows, then the partials in order (a fixed summation order)
+__global__ void __launch_bounds__(256) dproj_part_kernel(const HeadsArgs a) {
   const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
+  const int64_t j = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  const int64_t r0 = int64_t(blockIdx.y) * kDprojRows, r1 = min(a.R, r0 + kDprojRows);
+  if (j >= cols) return;
+  float acc = 0.f;
+  for (int64_t r = r0; r < r1; ++r) {
+    if (a.ws.m[r] == 0 || a.valid[r] == 0) continue;  // the same r in every thread
+    const float dc = a.ws.stats[r * kStride + kStDC];
+    const float x = j < a.H ? bf(a.hidden[size_t(r) * a.H + j]) : bf(a.ws.eall[size_t(r) * a.rank + (j - a.H)]);
+    acc = fmaf(dc, x, acc);
+  }
+  a.ws.dpp[size_t(blockIdx.y) * cols + j] = acc;
+}
+
+__global__ void __launch_bounds__(256) dproj_final_kernel(const HeadsArgs a) {
+  const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
+  const int64_t nchunks = (a.R + kDprojRows - 1) / kDprojRows;
   const int64_t j = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
   if (j < cols) {
     float acc = 0.f;
-    for (int64_t r = 0; r < a.R; ++r) {
-      if (a.ws.m[r] == 0 || a.valid[r] == 0) continue;
-      const float dc = a.ws.stats[r * kStride + kStDC];
-      const float x = j < a.H ? bf(a.hidden[size_t(r) * a.H + j]) : bf(a.ws.eall[size_t(r) * a.rank + (j - a.H)]);
-      acc = fmaf(dc, x, acc);
-    }
+    for (int64_t c = 0; c < nchunks; ++c) acc += a.ws.dpp[size_t(c) * cols + j];
     a.dconf_w[j] = a.accumulate ? a.dconf_w[j] + acc : acc;
   }
   if (blockIdx.x == 0) {
@@ -203,12 +241,12 @@ struct TeacherEpi {
   float* t;
   int64_t V;
   int row0, rows;
-  __device__ void operator()(int m, int n, int /*split*/, const float* v) const {
-    if (m >= rows || row0 + m >= hdr->n_sup) return;
-    float* out = t + size_t(m) * V;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (n + i < V) out[n + i] = v[i];
+  __device__ uint64_t row_state(int, int) const { return 0; }
+  __device__ void operator()(int m0, int n0, int /*split*/, const float* tile, int lane, uint64_t) const {
+    const int64_t c = n0 + lane;
+    const int nr = min(min(32, rows - m0), hdr->n_sup - row0 - m0);
+    if (c >= V) return;
+    for (int r = 0; r < nr; ++r) t[size_t(m0 + r) * V + c] = tile[r * tc::kTileLd + lane];
   }
 };
 
@@ -277,7 +315,9 @@ cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
   if (a.conf_w != nullptr) {
     const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
     if (a.dconf_w != nullptr) {
-      dproj_kernel<<<int((cols + 255) / 256), 256, 0, s>>>(a);
+      const dim3 grid(unsigned((cols + 255) / 256), unsigned((a.R + kDprojRows - 1) / kDprojRows));
+      dproj_part_kernel<<<grid, 256, 0, s>>>(a);
+      dproj_final_kernel<<<unsigned((cols + 255) / 256), 256, 0, s>>>(a);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.dhidden != nullptr) {

@@ -58,6 +58,8 @@ struct WsView {
   // teacher from hidden states (present when the problem has it)
   uint16_t* hsup;      // [R][Ht] bf16 target hidden rows, compact by supervised position
   float* tchunk;       // [chunk][V] FP32 teacher rows of one chunk of supervised rows
+  // confidence head (present when the problem has it)
+  float* dpp;          // [ceil(R / kDprojRows)][conf_cols] partial sums of dL/dproj
   size_t bytes;        // total bytes used
 };
 
@@ -69,7 +71,11 @@ struct WsDims {
   bool markov = false;
   int64_t Ht = 0, chunk = 0;  // teacher from hidden states: hidden size, rows per chunk
   bool lm = false;
+  int64_t conf_cols = 0;      // confidence head: length of proj (0 without the head)
 };
+
+// Rows per partial sum of the confidence head's weight gradient.
+constexpr int64_t kDprojRows = 64;
 
 // Supervised rows per teacher chunk (the FP32 teacher rows of a chunk are the only
 // vocabulary-wide teacher buffer; a multiple of the GEMM's 128-row tile).
@@ -77,7 +83,7 @@ constexpr int64_t kTeacherChunk = 512;
 constexpr int64_t teacher_chunk_rows(int64_t R) { return R < kTeacherChunk ? R : kTeacherChunk; }
 
 struct WsOffsets {
-  size_t hdr, m, w, sup, zero, sidx, stats, z, esup, eall, dep, de, hsup, tchunk, bytes;
+  size_t hdr, m, w, sup, zero, sidx, stats, z, esup, eall, dep, de, hsup, tchunk, dpp, bytes;
 };
 
 constexpr WsOffsets ws_offsets(const WsDims& d) {
@@ -113,6 +119,8 @@ constexpr WsOffsets ws_offsets(const WsDims& d) {
   off = align256(off + (d.lm ? 2 * R * size_t(d.Ht) : 0));
   o.tchunk = off;
   off = align256(off + (d.lm ? sizeof(float) * size_t(d.chunk) * size_t(d.V) : 0));
+  o.dpp = off;
+  off = align256(off + sizeof(float) * size_t((d.R + kDprojRows - 1) / kDprojRows) * size_t(d.conf_cols));
   o.bytes = off;
   return o;
 }
@@ -141,6 +149,7 @@ inline WsView ws_layout(void* base, const WsDims& d) {
   v.de = d.markov ? reinterpret_cast<float*>(b + o.de) : nullptr;
   v.hsup = d.lm ? reinterpret_cast<uint16_t*>(b + o.hsup) : nullptr;
   v.tchunk = d.lm ? reinterpret_cast<float*>(b + o.tchunk) : nullptr;
+  v.dpp = d.conf_cols ? reinterpret_cast<float*>(b + o.dpp) : nullptr;
   v.bytes = o.bytes;
   return v;
 }

@@ -92,19 +92,48 @@ __device__ __forceinline__ void load_group(const uint8_t* p, float* f) {
   }
 }
 
-// Control block in shared memory.
+// Warp maximum of an FP32 value (one instruction on sm_100a; -inf is the identity).
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// Control block in shared memory.  NP = cluster size x warps per CTA: every warp of
+// every CTA of the cluster pushes its partial of a row reduction into every CTA.
+template <int NP>
 struct Ctrl {
   uint64_t mbar_data[2];  // row segment (draft + teacher) landed
-  uint64_t mbar_ga;       // all cluster ranks' logsumexp partials landed
-  uint64_t mbar_gb;       // all cluster ranks' (L1, S) partials landed
-  float4 ga[16];          // (m_z, s_z, m_t, s_t) from rank i
-  float4 gb[16];          // (L1, S, 0, 0) from rank i
+  uint64_t mbar_ga;       // every warp's logsumexp partials landed
+  uint64_t mbar_gb;       // every CTA's (L1, S) partials landed
+  float4 ga[NP];          // (m_z, s_z, m_t, s_t) of warp w of rank i at [i * NW + w]
+  float4 gb[16];          // (L1, S, 0, 0) of rank i
   float4 red[32];         // per-warp partials
   float4 bcast;           // row logsumexps (base 2)
   float ztid;             // raw draft logit at the target id (owner only)
   int last;               // this CTA finished last and writes the report
   float pad[2];
+  // ring of the cluster's upcoming rows: row id, target id, loss weight
+  int32_t rrow[64];
+  int32_t rtok[64];
+  float rw[64];
 };
+
+constexpr int kRing = 64;       // ring entries
+constexpr int kRingFill = 32;   // entries loaded at a time
+
+// (m, s) partials of a base-2 logsumexp: the maximum first, then one rescaled sum.
+__device__ __forceinline__ void lse_pair_merge(float& m1, float& s1, float& m2, float& s2) {
+  const float M1 = warp_max_f32(m1), M2 = warp_max_f32(m2);
+  float t1 = (m1 == -INFINITY) ? 0.f : s1 * ex2(m1 - M1);
+  float t2 = (m2 == -INFINITY) ? 0.f : s2 * ex2(m2 - M2);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    t1 += __shfl_xor_sync(0xffffffffu, t1, off);
+    t2 += __shfl_xor_sync(0xffffffffu, t2, off);
+  }
+  m1 = M1, s1 = t1, m2 = M2, s2 = t2;
+}
 
 // One cluster of CL CTAs owns one supervised row at a time; CTA `rank` owns the
 // rank-th contiguous segment of the vocabulary.  Draft values live in registers
@@ -117,6 +146,8 @@ struct Ctrl {
 // head); TT the teacher rows' type (the logits type, or FP32 rows of the teacher
 // computed from hidden states); TO the type of the dlogits.  A launch covers the
 // supervised rows of positions [row0, row1) in the supervised list.
+// The row scalars come from a shared ring filled 64 rows ahead; the partials of the
+// row logsumexps go from every warp straight to every CTA of the cluster.
 template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T>
 __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   constexpr int EPV = VecTraits<TO>::EPV;
@@ -129,8 +160,10 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   constexpr bool kTChunk = sizeof(TT) == 4 && sizeof(TO) == 2;
   constexpr int NE = NV * EPV;
   constexpr int NW = NT / 32;
+  constexpr int NP = CL * NW;
   static_assert(NW <= 32 && CL <= 16, "control block sizes");
-  static_assert(NE % 2 == 0, "pairs of elements");
+  static_assert(NE % 4 == 0, "whole groups of four elements");
+  using CtrlT = Ctrl<NP>;
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -140,8 +173,8 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t seg_bytes = uint32_t(a.seg_vec) * uint32_t(TB);   // teacher segment
   const uint32_t zseg_bytes = uint32_t(a.seg_vec) * uint32_t(ZB);  // draft segment
   // buffers: HAS_T: [draft][teacher 0][teacher 1]; else [draft 0][draft 1]
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + (HAS_T ? size_t(zseg_bytes) + 2 * size_t(seg_bytes)
-                                                      : 2 * size_t(zseg_bytes)));
+  CtrlT* ctrl = reinterpret_cast<CtrlT*>(smem + (HAS_T ? size_t(zseg_bytes) + 2 * size_t(seg_bytes)
+                                                        : 2 * size_t(zseg_bytes)));
   auto zbuf = [&](int j) -> uint8_t* { return HAS_T ? smem : smem + size_t(j & 1) * zseg_bytes; };
   auto tbuf = [&](int j) -> uint8_t* {
     if constexpr (ZB == TB) return smem + size_t(1 + (j & 1)) * seg_bytes;  // zseg == seg
@@ -161,15 +194,14 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t bar_d1 = smem_u32(&ctrl->mbar_data[1]);
   const uint32_t bar_ga = smem_u32(&ctrl->mbar_ga);
   const uint32_t bar_gb = smem_u32(&ctrl->mbar_gb);
-  uint64_t policy = 0;
 
-  auto issue = [&](int j) {  // thread 0: stream row j's segment (draft and teacher)
+  // thread 0: stream the segment of the row at list position sidx (draft and teacher)
+  auto issue = [&](int j, int64_t sidx, int64_t row) {
     const uint32_t bar = (j & 1) ? bar_d1 : bar_d0;
-    const int64_t sidx = a.row0 + cid + int64_t(j) * G;
-    const int64_t row = a.ws.sup_list[sidx];
     const int64_t drow = (kMarkov && a.draft_compact) ? sidx : row;  // compact corrected rows
     const int64_t trow = (kTChunk && a.target_compact) ? sidx - a.row0 : row;  // teacher chunk
     mbar_arrive_expect_tx(bar, zbytes + (HAS_T ? bytes : 0u));
+    const uint64_t policy = l2_policy_evict_first();
     if (zbytes) {
       bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(drow) * a.ld_d + size_t(v0) * EPV) * sizeof(TZ),
                zbytes, bar, policy);
@@ -181,7 +213,6 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   auto flag_timeout = [&]() { atomicOr(&hdr->status, kFlagTimeout); };
 
   if (tid == 0) {
-    policy = l2_policy_evict_first();
     mbar_init(bar_d0, 1);
     mbar_init(bar_d1, 1);
     mbar_init(bar_ga, 1);
@@ -195,44 +226,65 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // this launch's supervised rows: list positions [row0, min(row1, n_sup))
   const int n_sup = max(0, min(hdr->n_sup, a.row1) - a.row0);
-  const int n_zero = a.do_zero ? hdr->n_zero : 0;
   const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
-  const float g = a.grad_scale ? *a.grad_scale : 1.f;
-  // this cluster's share of zero rows, written a slice after each supervised row
+  auto sidx_of = [&](int j) -> int64_t { return int64_t(a.row0) + cid + int64_t(j) * G; };
+
+  // this cluster's share of zero rows: a slice per supervised row, stored by warps
+  // 1 .. NW-1 while warp 0 merges the row's logsumexp partials; the id of the next
+  // slice's first row is loaded a slice ahead
+  const int n_zero = a.do_zero ? hdr->n_zero : 0;
   const int zfirst = ((int(cid) - n_sup) % int(G) + int(G)) % int(G);
   const int my_z = (bwd && zfirst < n_zero) ? (n_zero - 1 - zfirst) / int(G) + 1 : 0;
   const int ztot = my_z * nvec;
   const int zslice = my_n > 0 ? (ztot + my_n - 1) / my_n : ztot;
+  auto zrow_id = [&](int rk) -> int32_t { return rk < my_z ? a.ws.zero_list[zfirst + size_t(rk) * G] : 0; };
+  int32_t zr_pref = (my_z > 0 && warp != 0) ? zrow_id(0) : 0;
   auto write_zeros = [&](int q0, int q1) {
-    for (int q = q0 + tid; q < q1; q += NT) {
-      const int rk = q / nvec;
-      const int v = q - rk * nvec;
-      const int64_t zr = a.ws.zero_list[zfirst + size_t(rk) * G];
-      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.dlogits) +
-                                (size_t(zr) * a.ld_g + size_t(v0 + v) * EPV) * sizeof(TO)) = make_uint4(0u, 0u, 0u, 0u);
+    if (warp == 0 || q0 >= q1) return;
+    int rk = q0 / nvec;
+    const int rk_end = (q1 - 1) / nvec;
+    int32_t zr = zr_pref;
+    for (; rk <= rk_end; ++rk) {
+      const int32_t zr_next = zrow_id(rk + 1);  // in flight while this row is stored
+      const int lo = max(q0 - rk * nvec, 0), hi = min(q1 - rk * nvec, nvec);
+      uint8_t* base = static_cast<uint8_t*>(a.dlogits) + (size_t(zr) * a.ld_g + size_t(v0) * EPV) * sizeof(TO);
+      for (int v = lo + tid - 32; v < hi; v += NT - 32)
+        *reinterpret_cast<uint4*>(base + size_t(v) * 16) = make_uint4(0u, 0u, 0u, 0u);
+      zr_pref = (hi == nvec) ? zr_next : zr;  // where the next slice starts
+      zr = zr_next;
     }
   };
-  if (tid == 0) {
-    if (my_n > 0) issue(0);
-    if (!HAS_T && my_n > 1) issue(1);
-  }
 
-  // per-row scalars, loaded one row ahead
-  int64_t row = my_n > 0 ? a.ws.sup_list[a.row0 + cid] : 0;
-  int64_t tok = my_n > 0 ? a.tids[row] : 0;
-  float wr = my_n > 0 ? a.ws.w[row] : 0.f;
+  // per-row scalars (row and target id fit 32 bits: R < 2^31, V <= 2^30) of the rows
+  // j .. j + kRingFill - 1 in a shared ring, refilled kRingFill rows ahead
+  auto fill_ring = [&](int j0, int cnt) {
+    if (tid < cnt && j0 + tid < my_n) {
+      const int32_t r = a.ws.sup_list[sidx_of(j0 + tid)];
+      ctrl->rrow[(j0 + tid) % kRing] = r;
+      ctrl->rtok[(j0 + tid) % kRing] = int32_t(a.tids[r]);
+      ctrl->rw[(j0 + tid) % kRing] = a.ws.w[r];
+    }
+  };
+  fill_ring(0, kRing);
+  __syncthreads();
+  if (tid == 0) {
+    if (my_n > 0) issue(0, sidx_of(0), ctrl->rrow[0]);
+    if (!HAS_T && my_n > 1) issue(1, sidx_of(1), ctrl->rrow[1]);
+  }
 
   for (int j = 0; j < my_n; ++j) {
     const uint32_t phase = uint32_t(j >> 1) & 1u;
     const uint32_t gphase = uint32_t(j) & 1u;
-    const int tv = int(tok / EPV) - v0;  // target id's vector inside this segment
-    const int te = int(tok % EPV);
+    const int32_t row = ctrl->rrow[j % kRing];
+    const int32_t tok = ctrl->rtok[j % kRing];
+    const int tv = tok / EPV - v0;  // target id's vector inside this segment
+    const int te = tok % EPV;
     const uint8_t* zb = zbuf(j);
     const uint8_t* tb = tbuf(j);
+    // rows j + kRingFill .. j + kRing - 1 into the half of the ring that row j is not in
+    // (read from row j + kRingFill - 1 on, many barriers later)
+    if (j >= kRingFill && j % kRingFill == 0) fill_ring(j + kRingFill, kRingFill);
 
-    // a slice of the zero rows while this row's segment lands (nothing of the row
-    // is live in registers yet)
-    write_zeros(j * zslice, min(ztot, (j + 1) * zslice));
     if (!mbar_wait_bounded((j & 1) ? bar_d1 : bar_d0, phase) && tid == 0) flag_timeout();
 
     // ---- draft segment -> registers
@@ -253,18 +305,12 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     if (tid == 0) {
       // HAS_T: draft buffer + the teacher buffer of row j-1 (its pass 2 is done).
       // Without a teacher the draft buffers alternate.
-      if (HAS_T && j + 1 < my_n) issue(j + 1);
-      if (!HAS_T && j + 2 < my_n) issue(j + 2);
-    }
-    int64_t nrow = 0, ntok = 0;
-    float nw = 0.f;
-    if (j + 1 < my_n) {
-      nrow = a.ws.sup_list[a.row0 + cid + size_t(j + 1) * G];
-      ntok = a.tids[nrow];
-      nw = a.ws.w[nrow];
+      if (HAS_T && j + 1 < my_n) issue(j + 1, sidx_of(j + 1), ctrl->rrow[(j + 1) % kRing]);
+      if (!HAS_T && j + 2 < my_n) issue(j + 2, sidx_of(j + 2), ctrl->rrow[(j + 2) % kRing]);
     }
 
-    // ---- pass 1: per-thread maxima, draft exponentials kept, sums
+    // ---- pass 1: per-thread maxima, draft exponentials kept, sums (in this phase the
+    // MUFU pipe, not the add chains, sets the pace)
     float mz = -INFINITY, mt = -INFINITY;
 #pragma unroll
     for (int e = 0; e < NE; e += 2) mz = fmax3(mz, xz[e], xz[e + 1]);
@@ -300,31 +346,33 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         }
       }
     }
+
+    // ---- exchange A: every warp's (max, sum) pair into every CTA of the cluster
     {
       float m1 = (mz == -INFINITY) ? -INFINITY : oz, s1 = sz;
       float m2 = (mt == -INFINITY) ? -INFINITY : ot, s2 = st;
-      warp_lse_merge(m1, s1);
-      if constexpr (HAS_T) warp_lse_merge(m2, s2);
-      if (lane == 0) ctrl->red[warp] = make_float4(m1, s1, m2, s2);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-      float m1 = r4.x, s1 = r4.y, m2 = r4.z, s2 = r4.w;
-      warp_lse_merge(m1, s1);
-      if constexpr (HAS_T) warp_lse_merge(m2, s2);
-      if (lane == 0) mbar_arrive_expect_tx(bar_ga, CL * 16);
-      __syncwarp();
-      if (lane < CL) {  // all-gather of this CTA's partial into every rank
-        const uint32_t dst = dsmem_map(smem_u32(&ctrl->ga[rank]), uint32_t(lane));
+      lse_pair_merge(m1, s1, m2, s2);
+      if (warp == 0 && lane == 0) mbar_arrive_expect_tx(bar_ga, NP * 16);
+      if (lane < CL) {
+        const uint32_t dst = dsmem_map(smem_u32(&ctrl->ga[int(rank) * NW + warp]), uint32_t(lane));
         st_async_f4(dst, make_float4(m1, s1, m2, s2), dsmem_map(bar_ga, uint32_t(lane)));
       }
+    }
+    write_zeros(j * zslice, min(ztot, (j + 1) * zslice));
+    if (warp == 0) {
       if (!mbar_wait_bounded(bar_ga, gphase) && lane == 0) flag_timeout();
-      const float4 q4 = lane < CL ? ctrl->ga[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-      float n1 = q4.x, u1 = q4.y, n2 = q4.z, u2 = q4.w;
-      warp_lse_merge(n1, u1);
-      if constexpr (HAS_T) warp_lse_merge(n2, u2);
-      if (lane == 0) ctrl->bcast = make_float4(n1 + log2f(u1), HAS_T ? n2 + log2f(u2) : 0.f, 0.f, 0.f);
+      // NP partials, in the same order in every CTA: lane l merges l, l + 32, ...
+      float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
+#pragma unroll
+      for (int k = lane; k < NP; k += 32) {
+        const float4 q4 = ctrl->ga[k];
+        const float n1 = fmaxf(m1, q4.x), n2 = fmaxf(m2, q4.z);
+        s1 = (n1 == -INFINITY) ? 0.f : s1 * ex2(m1 - n1) + (q4.x == -INFINITY ? 0.f : q4.y * ex2(q4.x - n1));
+        s2 = (n2 == -INFINITY) ? 0.f : s2 * ex2(m2 - n2) + (q4.z == -INFINITY ? 0.f : q4.w * ex2(q4.z - n2));
+        m1 = n1, m2 = n2;
+      }
+      lse_pair_merge(m1, s1, m2, s2);
+      if (lane == 0) ctrl->bcast = make_float4(m1 + log2f(s1), HAS_T ? m2 + log2f(s2) : 0.f, 0.f, 0.f);
     }
     __syncthreads();
     const float4 lse4 = ctrl->bcast;
@@ -338,7 +386,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     // (an exact tie takes the sub-gradient +p).
     float L1 = 0.f, S = 0.f;
     if constexpr (HAS_T) {
-      float l1p = 0.f, sp = 0.f;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int v = tid + i * NT;
@@ -351,19 +399,29 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
             const float p = __fmul_rn(xz[i * EPV + e], az);
             const float d = __fsub_rn(p, q);
             const float u = copysignf(p, d);
-            l1p += fabsf(d);
-            sp += u;
+            l4[e & 3] += fabsf(d);
+            s4[e & 3] += u;
             xz[i * EPV + e] = u;
           }
         }
       }
-      l1p = warp_sum(l1p);
-      sp = warp_sum(sp);
+      float l1p = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      float sp = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        l1p += __shfl_xor_sync(0xffffffffu, l1p, off);
+        sp += __shfl_xor_sync(0xffffffffu, sp, off);
+      }
       if (lane == 0) ctrl->red[warp] = make_float4(l1p, sp, 0.f, 0.f);
       __syncthreads();
       if (warp == 0) {
         const float4 r4 = lane < NW ? ctrl->red[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float x = warp_sum(r4.x), y = warp_sum(r4.y);
+        float x = r4.x, y = r4.y;
+#pragma unroll
+        for (int off = NW / 2; off > 0; off >>= 1) {  // NW partials in lanes 0 .. NW-1
+          x += __shfl_xor_sync(0xffffffffu, x, off);
+          y += __shfl_xor_sync(0xffffffffu, y, off);
+        }
         if (lane == 0) mbar_arrive_expect_tx(bar_gb, CL * 16);
         __syncwarp();
         if (lane < CL) {
@@ -399,7 +457,8 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     if (bwd) {
       // an invalid Markov slot's corrected row is a constant: nothing flows to base
       const bool zero_out = kMarkov && a.invalid_zero && a.valid[row] == 0;
-      const float gw = zero_out ? 0.f : g * wr;
+      const float g = a.grad_scale ? *a.grad_scale : 1.f;
+      const float gw = zero_out ? 0.f : g * ctrl->rw[j % kRing];
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
       const float k0 = cce - cl1 * S;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(row) * a.ld_g + size_t(v0) * EPV) * sizeof(TO);
@@ -422,9 +481,6 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         }
       }
     }
-    row = nrow;
-    tok = ntok;
-    wr = nw;
   }
 
   // ---- what is left of this cluster's zero rows (all of them if it had no row)
@@ -466,7 +522,7 @@ size_t smem_bytes(int64_t V, bool has_t) {
   const int64_t vvec = V / EPV;
   const int64_t seg_vec = (vvec + CL - 1) / CL;
   const size_t zseg = size_t(seg_vec) * EPV * sizeof(TZ), tseg = size_t(seg_vec) * EPV * sizeof(TT);
-  return (has_t ? zseg + 2 * tseg : 2 * zseg) + sizeof(Ctrl);
+  return (has_t ? zseg + 2 * tseg : 2 * zseg) + sizeof(Ctrl<CL * 16>);
 }
 
 template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T>

@@ -6,7 +6,11 @@
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16
 //               per instruction, 4 per 64-wide stage) and tcgen05.commit
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator, one TMEM lane (= one tile
-//               row) per thread, handed to the epilogue functor 32 columns at a time
+//               row) per thread, 32 columns at a time, transposed through a padded
+//               32 x 33 shared tile so the epilogue functor can have the warp's lanes
+//               walk the columns of one row at a time (coalesced global accesses);
+//               the functor's row_state(m0, lane) is taken once per tile and handed
+//               to every 32-column block
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue of one
 // tile overlaps the MMAs of the next.  Operands are 128-byte-swizzled tiles, either
 // K-major (rows of 64 K values) or MN-major (rows of 64 M/N values per K index).
@@ -98,32 +102,36 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Epilogue staging: one 32 x 33 fp32 tile per epilogue warp.
+constexpr int kTileLd = 33;
+constexpr size_t kStageBytes = 4 * 32 * kTileLd * sizeof(float);
+
 // Shared memory a configuration needs (dynamic; the base is aligned to 1024 inside).
 template <int BN, int STAGES>
 constexpr size_t gemm_smem_bytes() {
-  return size_t(STAGES) * (BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+  return size_t(STAGES) * (BM * BK * 2 + BN * BK * 2) + 1024 + 256 + kStageBytes;
 }
 
 // Work item w -> (m-tile, n-tile, k-split) and its range of 64-wide K chunks.  The
-// m-tile is the slowest index, so with a device-side row bound (rows m_base + m at or
-// past *m_bound are not needed) the needed items are exactly the first items().
+// m-tile is the fastest index: CTAs running at the same time share their B tiles (the
+// large operand of the row-skinny products) through L2 instead of each m-tile
+// streaming all of B from HBM again.  With a device-side row bound (rows m_base + m
+// at or past *m_bound are not needed) only the first m_eff() m-tiles take part.
 struct WorkMap {
   int m_tiles, n_tiles, ksplit, kchunks;
   const int32_t* m_bound;
   int m_base;
-  __device__ __forceinline__ int items() const {
-    int mt = m_tiles;
-    if (m_bound != nullptr) {
-      const int rem = *m_bound - m_base;
-      mt = rem <= 0 ? 0 : min(m_tiles, (rem + BM - 1) / BM);
-    }
-    return mt * n_tiles * ksplit;
+  __device__ __forceinline__ int m_eff() const {
+    if (m_bound == nullptr) return m_tiles;
+    const int rem = *m_bound - m_base;
+    return rem <= 0 ? 0 : min(m_tiles, (rem + BM - 1) / BM);
   }
-  __device__ __forceinline__ void decode(int w, int& mt, int& nt, int& s, int& kc0, int& kc1) const {
-    s = w % ksplit;
-    const int t = w / ksplit;
-    nt = t % n_tiles;
-    mt = t / n_tiles;
+  __device__ __forceinline__ int items(int me) const { return me * n_tiles * ksplit; }
+  __device__ __forceinline__ void decode(int w, int me, int& mt, int& nt, int& s, int& kc0, int& kc1) const {
+    mt = w % me;
+    const int t = w / me;
+    s = t % ksplit;
+    nt = t / ksplit;
     kc0 = int((int64_t(s) * kchunks) / ksplit);
     kc1 = int((int64_t(s + 1) * kchunks) / ksplit);
   }
@@ -147,9 +155,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t accf0 = empty0 + 8 * STAGES;
   const uint32_t acce0 = accf0 + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  float* stage = reinterpret_cast<float*>(smem + size_t(STAGES) * SS + 256);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int W = wm.items();  // the same in every role
+  const int ME = wm.m_eff();  // the same in every role
+  const int W = wm.items(ME);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -174,7 +184,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     int it = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x) {
       int mt, nt, s, kc0, kc1;
-      wm.decode(w, mt, nt, s, kc0, kc1);
+      wm.decode(w, ME, mt, nt, s, kc0, kc1);
       for (int kc = kc0; kc < kc1; ++kc, ++it) {
         const int st = it % STAGES;
         const uint32_t round = uint32_t(it / STAGES);
@@ -202,7 +212,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     int it = 0, tl = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x, ++tl) {
       int mt, nt, s, kc0, kc1;
-      wm.decode(w, mt, nt, s, kc0, kc1);
+      wm.decode(w, ME, mt, nt, s, kc0, kc1);
       const int b = tl & 1;
       const uint32_t use = uint32_t(tl >> 1);
       if (!mbar_wait_bounded(acce0 + 8 * b, (use & 1u) ^ 1u)) timed_out = true;
@@ -229,21 +239,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else if (warp >= 2) {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
     const int q = warp & 3;
-    const int row_in_tile = q * 32 + lane;
+    float* tile = stage + q * 32 * kTileLd;
     int tl = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x, ++tl) {
       int mt, nt, s, kc0, kc1;
-      wm.decode(w, mt, nt, s, kc0, kc1);
+      wm.decode(w, ME, mt, nt, s, kc0, kc1);
       const int b = tl & 1;
       const uint32_t use = uint32_t(tl >> 1);
       if (!mbar_wait_bounded(accf0 + 8 * b, use & 1u)) timed_out = true;
       fence_after_sync();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(b * BN);
+      // per-row state of the functor (e.g. gathered row ids), fetched once per tile
+      const uint64_t rs = epi.row_state(mt * BM + q * 32, lane);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + uint32_t(c * 32), v);
-        epi(mt * BM + row_in_tile, nt * BN + c * 32, s, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) tile[lane * kTileLd + i] = v[i];  // row lane, column i
+        __syncwarp();
+        // rows m0 .. m0 + 31, columns n0 .. n0 + 31: element (r, j) at tile[r * kTileLd + j]
+        epi(mt * BM + q * 32, nt * BN + c * 32, s, static_cast<const float*>(tile), lane, rs);
+        __syncwarp();
       }
       fence_before_sync();
       __syncwarp();

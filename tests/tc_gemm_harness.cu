@@ -6,15 +6,14 @@
 
 using namespace dspark;
 
-struct SplitStoreEpi {  // partial of K split s at d[s][m][n]
+struct SplitStoreEpi {  // partial of K split s at d[s][m][n]; the block is rows m0.., columns n0..
   float* d;
   int M, N;
-  __device__ void operator()(int m, int n, int split, const float* v) const {
-    if (m >= M) return;
-    float* row = d + (int64_t(split) * M + m) * N;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (n + i < N) row[n + i] = v[i];
+  __device__ uint64_t row_state(int, int) const { return 0; }
+  __device__ void operator()(int m0, int n0, int split, const float* t, int lane, uint64_t) const {
+    const int n = n0 + lane;
+    if (n >= N) return;
+    for (int r = 0; r < 32 && m0 + r < M; ++r) d[(int64_t(split) * M + m0 + r) * N + n] = t[r * tc::kTileLd + lane];
   }
 };
 
