@@ -37,6 +37,7 @@ from speculative_decoding_draft_vocab_b200.synthetic import CONFIGS, make_inputs
 METRIC = "supervised rows/s, DSpark loss fwd+bwd @V=151936; achieved HBM GB/s vs peak"
 PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sweep_recipe_traffic.md")
 KERNEL_SOURCES = ["speculative_decoding_draft_vocab_b200/csrc/sweep.cu",
                   "speculative_decoding_draft_vocab_b200/csrc/prologue.cu",
@@ -59,12 +60,67 @@ def workload_desc(name: str, inp) -> str:
     return ", ".join(parts)
 
 
+WEIGHTS = ("markov_w1", "markov_w2", "conf_w", "conf_b", "lm_head")  # resident across steps
+
+
 def algorithmic_bytes(inp, n_sup: int) -> int:
-    """Logits read once per supervised row (draft + teacher), dlogits written for every
-    row: the bytes a perfect single-pass kernel must move."""
+    """The bytes a perfect single-pass implementation must move: the base draft and the
+    teacher logits of every supervised row read once, dlogits written for every row;
+    with the heads, the Markov tables read and their gradients written once, the
+    hidden states read once and their gradient written once; with the teacher from
+    hidden states, lm_head and the target hidden states read once instead of teacher
+    logits.  Corrected rows, teacher chunks and re-reads of dlogits by the weight
+    gradients are not counted: they are this implementation's overhead."""
     es = 2 if inp.dtype == "bf16" else 4
-    per_sup = inp.V * es * (3 if inp.target_logits is not None else 2)
-    return n_sup * per_sup + (inp.R - n_sup) * inp.V * es
+    b = n_sup * inp.V * es + inp.R * inp.V * es
+    if inp.target_logits is not None:
+        b += n_sup * inp.V * es
+    if inp.lm_head is not None:
+        b += inp.lm_head.numel() * 2 + n_sup * inp.lm_head.shape[1] * 2
+    if inp.markov_w2 is not None:
+        r = inp.markov_w2.shape[1]
+        b += inp.V * r * (2 + 4) + n_sup * r * (2 + 4)
+    if inp.conf_w is not None:
+        b += inp.draft_hidden.numel() * 2 * 2
+    return b
+
+
+def algorithmic_flops(inp, n_sup: int) -> int:
+    """Tensor-core work a perfect implementation must do: the Markov bias, dE and dW2
+    contractions (2 * rows * V * rank each) and the teacher product (2 * rows * V * Ht)."""
+    f = 0
+    if inp.markov_w2 is not None:
+        f += 3 * 2 * n_sup * inp.V * inp.markov_w2.shape[1]
+    if inp.lm_head is not None:
+        f += 2 * n_sup * inp.V * inp.lm_head.shape[1]
+    return f
+
+
+def launches_per_call(inp) -> int:
+    """Kernels one fused call launches (the launch sequence of dspark_loss_fwd)."""
+    n = 2  # mask prologue, sweep
+    markov, conf_head, lm = inp.markov_w2 is not None, inp.conf_w is not None, inp.lm_head is not None
+    if markov or conf_head:
+        n += 1  # gather of embeddings and confidence logits
+    if markov:
+        n += 1 + 3  # bias GEMM; dE GEMM, dW2 GEMM, dE reduction and dW1 scatter
+    if conf_head:
+        n += 3  # dproj partials, dproj final, dhidden
+    if lm:
+        chunks = (inp.R + 511) // 512
+        n += 1 + chunks + (chunks - 1)  # hidden gather, teacher GEMM per chunk, sweep per chunk
+    return n
+
+
+def oracle_kwargs(inp):
+    """The oracle's keyword arguments for a CPU copy of the inputs."""
+    def a(t):
+        return None if t is None else t.float().numpy()
+    return dict(target_logits=a(inp.target_logits), block_keep=a(inp.block_keep),
+                confidence_logits=a(inp.confidence_logits), prev_ids=a(inp.prev_ids), valid=a(inp.valid),
+                markov_w1=a(inp.markov_w1), markov_w2=a(inp.markov_w2), draft_hidden=a(inp.draft_hidden),
+                conf_w=a(inp.conf_w), conf_b=a(inp.conf_b), conf_with_markov=inp.conf_with_markov,
+                target_hidden=a(inp.target_hidden), lm_head=a(inp.lm_head), gamma=inp.gamma)
 
 
 def sources_sha() -> str:
@@ -101,6 +157,15 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s, burst figure (the GEMMs of one call are timed inside it)."""
+    try:
+        with open(PEAKS) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 class ClockSampler:
@@ -159,15 +224,21 @@ class ClockSampler:
 
 
 def run_cpu_baseline(name: str, budget_s: float, seed: int = None):
-    """Time the FP64 oracle on a bounded sample of supervised rows of the workload."""
+    """Time the FP64 oracle on a bounded sample of supervised rows of the workload, with
+    numpy's BLAS held to one thread (so `cores` is exactly 1)."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        return _cpu_baseline(name, budget_s, seed)
+
+
+def _cpu_baseline(name: str, budget_s: float, seed: int = None):
     import numpy as np
     from oracle import dspark_oracle as O
     inp = make_inputs(name, device="cpu", seed=seed)
     m = O.prefix_supervision_mask(inp.eval_mask.numpy(), inp.block_keep.numpy()).reshape(-1)
     sup = np.nonzero(m)[0]
     draft = inp.draft_logits.float().numpy()
-    target = inp.target_logits.float().numpy() if inp.target_logits is not None else None
-    kw = dict(target_logits=target, block_keep=inp.block_keep.numpy())
+    kw = oracle_kwargs(inp)
     # calibrate on 2 rows, then take as many rows as the budget allows
     t0 = time.perf_counter()
     O.dspark_loss(draft, inp.target_ids.numpy(), inp.eval_mask.numpy(), rows=sup[:2], **kw)
@@ -254,16 +325,29 @@ def main():
     ms_per_step = total_ms / args.steps
     value = rows_all * args.steps / (total_ms / 1e3)
 
-    # ---- roofline of the hot path (one call: mask prologue + sweep)
+    # ---- roofline of the call: HBM bytes and tensor FLOPs a perfect implementation
+    # needs; the bound is whichever takes longer at its measured peak
     alg = algorithmic_bytes(inp, n_sup)
+    flops = algorithmic_flops(inp, n_sup)
     peak, peak_kind = hbm_peak()
+    tpeak, tpeak_kind = tensor_peak()
     mean_ms = statistics.mean(per_step)
-    achieved = alg / (mean_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                "traffic": recorded_traffic(), "algorithmic_bytes": alg,
-                "timed": "dspark_loss_fwd with fused backward (mask prologue + sweep kernel), "
-                         "mean CUDA-event duration per call"}
+    t_hbm, t_tc = alg / (peak * 1e9), flops / (tpeak * 1e12)
+    n_launch = launches_per_call(inp)
+    timed = (f"dspark_loss_fwd with fused backward ({n_launch} kernels: "
+             + ("mask prologue + sweep" if n_launch == 2 else "prologue, heads, sweep, head gradients")
+             + "), mean CUDA-event duration per call")
+    if t_hbm >= t_tc:
+        achieved = alg / (mean_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                    "traffic": recorded_traffic() if n_launch == 2 else None, "algorithmic_bytes": alg,
+                    "algorithmic_flops": flops, "timed": timed}
+    else:
+        achieved = flops / (mean_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": round(achieved / tpeak, 4), "peak_kind": tpeak_kind, "traffic": None,
+                    "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
 
     # ---- end to end from pinned host buffers
     e2e = run_e2e(inp, args.e2e_steps, torch_api)
@@ -287,7 +371,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 1), "unit": "rows/s", "h2d_bytes_per_step": e2e["h2d"],
                     "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"], 4)},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": n_launch * args.steps,
             "clocks": clk.summary(),
             "wall_s_timed_region": round(wall, 3),
         }
@@ -298,9 +382,10 @@ def main():
 
 
 def run_e2e(inp, steps: int, torch_api):
-    """Per step: pinned host -> device copy of the micro-batch, the call, and a device ->
-    host read of the loss, token count and report."""
-    dev_tensors = {k: v for k, v in inp.tensors().items()}
+    """Per step: pinned host -> device copy of the micro-batch (logits, ids, masks, hidden
+    states; the head weights stay resident like model parameters), the call, and a
+    device -> host read of the loss, token count and report."""
+    dev_tensors = {k: v for k, v in inp.tensors().items() if k not in WEIGHTS}
     host = {k: v.cpu().pin_memory() for k, v in dev_tensors.items()}
     call = torch_api.Call(inp, grads=True, rows=False)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -326,17 +411,23 @@ def run_e2e(inp, steps: int, torch_api):
 
 
 def run_reference(args, world, rank):
-    """The oracle arm: rank 0 times the FP64 CPU oracle on a bounded sample per step."""
+    """The oracle arm: rank 0 times the FP64 CPU oracle on a bounded sample per step
+    (numpy's BLAS held to one thread)."""
     if rank != 0:
         return
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        _run_reference(args, world)
+
+
+def _run_reference(args, world):
     import numpy as np
     from oracle import dspark_oracle as O
     inp = make_inputs(args.workload, device="cpu")
     m = O.prefix_supervision_mask(inp.eval_mask.numpy(), inp.block_keep.numpy()).reshape(-1)
     sup = np.nonzero(m)[0]
     draft = inp.draft_logits.float().numpy()
-    target = inp.target_logits.float().numpy() if inp.target_logits is not None else None
-    kw = dict(target_logits=target, block_keep=inp.block_keep.numpy())
+    kw = oracle_kwargs(inp)
     t0 = time.perf_counter()
     O.dspark_loss(draft, inp.target_ids.numpy(), inp.eval_mask.numpy(), rows=sup[:1], **kw)
     per_row = time.perf_counter() - t0

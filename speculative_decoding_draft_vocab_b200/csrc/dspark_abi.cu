@@ -156,10 +156,9 @@ SweepArgs sweep_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
     a.ld_t = p->V;
     a.target_compact = 1;
   }
-  if (markov_present(p)) {  // the sweep reads the corrected rows, compact by supervised position
-    a.draft = ws.z;
-    a.ld_d = p->V;
-    a.draft_compact = 1;
+  if (markov_present(p)) {  // the sweep adds the head's bias rows (compact by supervised position)
+    a.bias = ws.bias;
+    a.ld_b = p->V;
     a.valid = p->valid;
     a.invalid_zero = prm->invalid_row_mode == 0;
   }
@@ -185,8 +184,6 @@ HeadsArgs heads_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
   h.Vt = p->target_vocab;
   h.rank = markov_present(p) ? p->markov_rank : 0;
   h.H = p->conf_w ? p->hidden_size : 0;
-  h.base = static_cast<const uint16_t*>(p->draft_logits);
-  h.ld_base = p->draft_ld;
   h.prev_ids = p->prev_ids;
   h.valid = p->valid;
   h.w1 = markov_present(p) ? static_cast<const uint16_t*>(p->markov_w1) : nullptr;

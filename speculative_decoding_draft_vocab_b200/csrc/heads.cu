@@ -1,5 +1,6 @@
 // The two DSpark auxiliary heads (NeMo RL design doc "DSpark Auxiliary Heads"):
-//   Markov head:      z = base + markov_w2 . e,  e = markov_w1[prev]   (valid slots)
+//   Markov head:      z = base + markov_w2 . e,  e = markov_w1[prev]   (valid slots;
+//                     the bias rows are written here, the sweep adds the base rows)
 //                     an invalid slot's corrected row is all zero (mode 0) or its base
 //                     row (mode 1); prev ids are in the target vocabulary
 //   confidence head:  c = proj . [h ; e] + bias on valid slots, 0 on invalid ones
@@ -73,45 +74,30 @@ __global__ void __launch_bounds__(256) heads_prep_kernel(const HeadsArgs a) {
   }
 }
 
-// ---- epilogue of the bias GEMM: corrected row z = base + E.W2^T (compact rows)
+// ---- epilogue of the bias GEMM: the Markov bias rows W2.e (compact by supervised
+// position), 0 on invalid slots; the sweep adds them to the base rows it streams
 // (epilogue functors get a 32 x 32 block of the accumulator, rows m0.., columns n0..,
 // element (r, j) at t[r * tc::kTileLd + j]; lane j handles column n0 + j of every row)
 struct BiasEpi {
   const int32_t* sup_list;
   const WsHeader* hdr;
-  const uint16_t* base;
-  int64_t ld_base;
   const uint8_t* valid;
-  int invalid_row_mode;
-  float* z;
-  int64_t ldz;
+  float* bias;
+  int64_t ldb;
   int V;
-  // lane l: the id of row m0 + l (low 32 bits) and its valid flag (bit 32); bit 33
-  // set past the last supervised row
+  // lane l: bit 0 = row m0 + l is a valid slot, bit 1 = past the last supervised row
   __device__ uint64_t row_state(int m0, int lane) const {
     const int m = m0 + lane;
-    if (m >= hdr->n_sup) return uint64_t(1) << 33;
-    const int32_t row = sup_list[m];
-    return uint64_t(uint32_t(row)) | (uint64_t(valid[row] != 0) << 32);
+    if (m >= hdr->n_sup) return 2;
+    return valid[sup_list[m]] != 0 ? 1 : 0;
   }
   __device__ void operator()(int m0, int n0, int /*split*/, const float* t, int lane, uint64_t rs) const {
     const int c = n0 + lane;
-    const bool col = c < V;
-    // every load of the block before any store (base and z may not alias, but the
-    // compiler cannot know that)
-    float bv[32];
-#pragma unroll
+    const uint32_t st = uint32_t(rs);
+#pragma unroll 8
     for (int r = 0; r < 32; ++r) {
-      const uint64_t q = __shfl_sync(0xffffffffu, rs, r);
-      bv[r] = (col && !(q >> 33)) ? bf(base[size_t(uint32_t(q)) * ld_base + c]) : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const uint64_t q = __shfl_sync(0xffffffffu, rs, r);
-      if (col && !(q >> 33)) {
-        const bool ok = (q >> 32) & 1u;
-        z[size_t(m0 + r) * ldz + c] = ok ? bv[r] + t[r * tc::kTileLd + lane] : (invalid_row_mode == 0 ? 0.f : bv[r]);
-      }
+      const uint32_t q = __shfl_sync(0xffffffffu, st, r);
+      if (c < V && !(q & 2u)) bias[size_t(m0 + r) * ldb + c] = (q & 1u) ? t[r * tc::kTileLd + lane] : 0.f;
     }
   }
 };
@@ -283,7 +269,7 @@ cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   if (!tc::make_map(&ma, a.ws.esup, a.R, a.rank, a.rank, 64, 128)) return cudaErrorInvalidValue;
   if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 256)) return cudaErrorInvalidValue;
-  BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.base, a.ld_base, a.valid, a.invalid_row_mode, a.ws.z, a.V, int(a.V)};
+  BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.valid, a.ws.bias, a.V, int(a.V)};
   return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s,
                                         &a.ws.hdr->n_sup, 0);
 }

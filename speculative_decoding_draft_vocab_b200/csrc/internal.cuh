@@ -50,7 +50,7 @@ struct WsView {
   int32_t* sup_index;  // [R] position of a row in sup_list, -1 if unsupervised
   float* stats;        // [R][kStride]
   // Markov head (present when the problem has it)
-  float* z;            // [R][V] corrected draft rows, compact by supervised position
+  float* bias;         // [R][V] Markov bias rows W2.e (0 on invalid slots), compact by supervised position
   uint16_t* esup;      // [R][rank] bf16 Markov embeddings, compact (0 on invalid slots)
   uint16_t* eall;      // [R][rank] bf16 Markov embeddings by row (0 unless supervised+valid)
   float* dep;          // [splits][R][rank] split-K partials of dE
@@ -142,7 +142,7 @@ inline WsView ws_layout(void* base, const WsDims& d) {
   v.zero_list = reinterpret_cast<int32_t*>(b + o.zero);
   v.sup_index = reinterpret_cast<int32_t*>(b + o.sidx);
   v.stats = reinterpret_cast<float*>(b + o.stats);
-  v.z = d.markov ? reinterpret_cast<float*>(b + o.z) : nullptr;
+  v.bias = d.markov ? reinterpret_cast<float*>(b + o.z) : nullptr;
   v.esup = d.markov ? reinterpret_cast<uint16_t*>(b + o.esup) : nullptr;
   v.eall = d.markov ? reinterpret_cast<uint16_t*>(b + o.eall) : nullptr;
   v.dep = d.markov ? reinterpret_cast<float*>(b + o.dep) : nullptr;
@@ -206,7 +206,8 @@ struct SweepArgs {
   int32_t vvec;              // V / elements per 16-byte vector
   int32_t seg_vec;           // vectors per CTA segment
   int32_t nbuf;              // prefetch depth (1 or 2)
-  int32_t draft_compact;     // draft row of the i-th supervised row is i (corrected rows)
+  const float* bias;         // Markov bias rows (compact by supervised position), or null
+  int64_t ld_b;
   const uint8_t* valid;      // Markov valid-slot mask (with invalid_zero)
   int32_t invalid_zero;      // invalid slots get zero dlogits (all-zero corrected row)
   int32_t target_compact;    // teacher row of list position i is i - row0 (teacher chunk)
@@ -222,8 +223,6 @@ struct SweepArgs {
 // Markov head and confidence head (inputs, weight gradients and workspace).
 struct HeadsArgs {
   int64_t R, V, Vt, rank, H;
-  const uint16_t* base;      // bf16 [R][ld_base] base draft logits
-  int64_t ld_base;
   const int64_t* prev_ids;
   const uint8_t* valid;
   const uint16_t* w1;        // bf16 [Vt][rank], null without the Markov head
@@ -259,9 +258,9 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s);
 enum : int {
   kSweepBf16 = 0,  // bf16 / bf16 / bf16
   kSweepF32 = 1,   // f32 / f32 / f32
-  kSweepZ32 = 2,   // f32 corrected rows (Markov head) / bf16 / bf16
+  kSweepZ32 = 2,   // bf16 + FP32 Markov bias rows / bf16 / bf16
   kSweepT32 = 3,   // bf16 / f32 teacher chunk (teacher from hidden states) / bf16
-  kSweepZT32 = 4,  // f32 corrected rows / f32 teacher chunk / bf16
+  kSweepZT32 = 4,  // bf16 + FP32 Markov bias rows / f32 teacher chunk / bf16
 };
 // False if V exceeds every build of that kind.
 bool sweep_supported(int kind, int64_t V, bool has_target);
@@ -277,7 +276,7 @@ cudaError_t launch_conf_grad(int64_t R, const float* confidence_logits, float co
 cudaError_t launch_bwd_stream(int kind, bool has_target, const SweepArgs& a, int64_t R, cudaStream_t s);
 // Markov embeddings (both copies) and confidence logits
 cudaError_t launch_heads_prep(const HeadsArgs& a, cudaStream_t s);
-// corrected rows ws.z = base + E.W2^T (compact, FP32) on the tensor cores
+// Markov bias rows ws.bias = E.W2^T (compact, FP32; 0 on invalid slots) on the tensor cores
 cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s);
 // dE, dW1, dW2, dconf_w, dconf_b, dhidden from dlogits and the saved dL/dc
 cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s);

@@ -142,21 +142,24 @@ __device__ __forceinline__ void lse_pair_merge(float& m1, float& s1, float& m2, 
 // on chip and a row fits in 4 SMs of a 148-SM part.  Shared memory holds one draft
 // landing buffer and two teacher buffers: the next row's copy is issued as soon as
 // the current draft segment is in registers, one full row ahead of its use.
-// TZ is the draft rows' type (the logits type, or FP32 corrected rows of the Markov
-// head); TT the teacher rows' type (the logits type, or FP32 rows of the teacher
-// computed from hidden states); TO the type of the dlogits.  A launch covers the
-// supervised rows of positions [row0, row1) in the supervised list.
-// The row scalars come from a shared ring filled 64 rows ahead; the partials of the
+// TZ is the draft logits' type; TT the teacher rows' type (the logits type, or FP32
+// rows of the teacher computed from hidden states); TO the type of the dlogits.  With
+// HAS_B (the Markov head) the corrected row z = keep * base + bias is formed on chip
+// from the base row and the FP32 bias row of the head (compact by supervised
+// position; keep = 0 only on an invalid slot whose corrected row is all zero, where
+// the bias is 0 as well).  A launch covers the supervised rows of positions
+// [row0, row1) in the supervised list.
+// The row scalars come from a shared ring filled 32 rows ahead; the partials of the
 // row logsumexps go from every warp straight to every CTA of the cluster.
-template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T>
+template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T, bool HAS_B>
 __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   constexpr int EPV = VecTraits<TO>::EPV;
   constexpr int ZB = EPV * int(sizeof(TZ));  // bytes of one draft group
+  constexpr int BB = HAS_B ? EPV * 4 : 0;    // bytes of one bias group
   constexpr int TB = EPV * int(sizeof(TT));  // bytes of one teacher group
-  // FP32 rows under 16-bit outputs only come from the heads (compact corrected rows
-  // with their valid-slot mask; compact teacher chunks); the other builds carry none
-  // of that code
-  constexpr bool kMarkov = sizeof(TZ) == 4 && sizeof(TO) == 2;
+  constexpr bool kMarkov = HAS_B;
+  // FP32 teacher rows under 16-bit outputs only come from the teacher chunks (compact);
+  // the other builds carry none of that code
   constexpr bool kTChunk = sizeof(TT) == 4 && sizeof(TO) == 2;
   constexpr int NE = NV * EPV;
   constexpr int NW = NT / 32;
@@ -172,13 +175,17 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t G = nclusters_x();
   const uint32_t seg_bytes = uint32_t(a.seg_vec) * uint32_t(TB);   // teacher segment
   const uint32_t zseg_bytes = uint32_t(a.seg_vec) * uint32_t(ZB);  // draft segment
-  // buffers: HAS_T: [draft][teacher 0][teacher 1]; else [draft 0][draft 1]
-  CtrlT* ctrl = reinterpret_cast<CtrlT*>(smem + (HAS_T ? size_t(zseg_bytes) + 2 * size_t(seg_bytes)
-                                                        : 2 * size_t(zseg_bytes)));
+  const uint32_t bseg_bytes = uint32_t(a.seg_vec) * uint32_t(BB);  // bias segment
+  // buffers: HAS_T: [draft][bias][teacher 0][teacher 1]; else [draft 0][draft 1][bias 0][bias 1]
+  CtrlT* ctrl = reinterpret_cast<CtrlT*>(smem + (HAS_T ? size_t(zseg_bytes) + bseg_bytes + 2 * size_t(seg_bytes)
+                                                        : 2 * (size_t(zseg_bytes) + bseg_bytes)));
   auto zbuf = [&](int j) -> uint8_t* { return HAS_T ? smem : smem + size_t(j & 1) * zseg_bytes; };
+  auto bbuf = [&](int j) -> uint8_t* {
+    return HAS_T ? smem + zseg_bytes : smem + 2 * size_t(zseg_bytes) + size_t(j & 1) * bseg_bytes;
+  };
   auto tbuf = [&](int j) -> uint8_t* {
-    if constexpr (ZB == TB) return smem + size_t(1 + (j & 1)) * seg_bytes;  // zseg == seg
-    else return smem + zseg_bytes + size_t(j & 1) * seg_bytes;
+    if constexpr (ZB == TB && BB == 0) return smem + size_t(1 + (j & 1)) * seg_bytes;  // zseg == seg
+    else return smem + zseg_bytes + bseg_bytes + size_t(j & 1) * seg_bytes;
   };
   WsHeader* hdr = a.ws.hdr;
 
@@ -186,6 +193,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const int nvec = max(0, min(a.seg_vec, a.vvec - v0));
   const uint32_t bytes = uint32_t(nvec) * uint32_t(TB);
   const uint32_t zbytes = uint32_t(nvec) * uint32_t(ZB);
+  const uint32_t bbytes = uint32_t(nvec) * uint32_t(BB);
   const uint8_t* draft = static_cast<const uint8_t*>(a.draft);
   const uint8_t* target = static_cast<const uint8_t*>(a.target);
   const bool bwd = a.dlogits != nullptr;
@@ -195,16 +203,18 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   const uint32_t bar_ga = smem_u32(&ctrl->mbar_ga);
   const uint32_t bar_gb = smem_u32(&ctrl->mbar_gb);
 
-  // thread 0: stream the segment of the row at list position sidx (draft and teacher)
+  // thread 0: stream the segment of the row at list position sidx (draft, bias, teacher)
   auto issue = [&](int j, int64_t sidx, int64_t row) {
     const uint32_t bar = (j & 1) ? bar_d1 : bar_d0;
-    const int64_t drow = (kMarkov && a.draft_compact) ? sidx : row;  // compact corrected rows
     const int64_t trow = (kTChunk && a.target_compact) ? sidx - a.row0 : row;  // teacher chunk
-    mbar_arrive_expect_tx(bar, zbytes + (HAS_T ? bytes : 0u));
+    mbar_arrive_expect_tx(bar, zbytes + bbytes + (HAS_T ? bytes : 0u));
     const uint64_t policy = l2_policy_evict_first();
     if (zbytes) {
-      bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(drow) * a.ld_d + size_t(v0) * EPV) * sizeof(TZ),
+      bulk_g2s(smem_u32(zbuf(j)), draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * sizeof(TZ),
                zbytes, bar, policy);
+      if constexpr (HAS_B)  // the bias rows are compact by supervised position
+        bulk_g2s(smem_u32(bbuf(j)), a.bias + (size_t(sidx) * a.ld_b + size_t(v0) * EPV),
+                 bbytes, bar, policy);
       if constexpr (HAS_T)
         bulk_g2s(smem_u32(tbuf(j)), target + (size_t(trow) * a.ld_t + size_t(v0) * EPV) * sizeof(TT),
                  bytes, bar, policy);
@@ -257,11 +267,14 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
   // per-row scalars (row and target id fit 32 bits: R < 2^31, V <= 2^30) of the rows
   // j .. j + kRingFill - 1 in a shared ring, refilled kRingFill rows ahead
+  // (with the Markov head bit 31 of the target id marks an all-zero corrected row)
   auto fill_ring = [&](int j0, int cnt) {
     if (tid < cnt && j0 + tid < my_n) {
       const int32_t r = a.ws.sup_list[sidx_of(j0 + tid)];
+      int32_t t = int32_t(a.tids[r]);
+      if (kMarkov && a.invalid_zero && a.valid[r] == 0) t |= int32_t(0x80000000u);
       ctrl->rrow[(j0 + tid) % kRing] = r;
-      ctrl->rtok[(j0 + tid) % kRing] = int32_t(a.tids[r]);
+      ctrl->rtok[(j0 + tid) % kRing] = t;
       ctrl->rw[(j0 + tid) % kRing] = a.ws.w[r];
     }
   };
@@ -276,10 +289,13 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     const uint32_t phase = uint32_t(j >> 1) & 1u;
     const uint32_t gphase = uint32_t(j) & 1u;
     const int32_t row = ctrl->rrow[j % kRing];
-    const int32_t tok = ctrl->rtok[j % kRing];
+    const int32_t tokf = ctrl->rtok[j % kRing];
+    const int32_t tok = tokf & 0x7fffffff;
+    const bool zero_row = kMarkov && tokf < 0;  // corrected row all zero
     const int tv = tok / EPV - v0;  // target id's vector inside this segment
     const int te = tok % EPV;
     const uint8_t* zb = zbuf(j);
+    const uint8_t* bb = bbuf(j);
     const uint8_t* tb = tbuf(j);
     // rows j + kRingFill .. j + kRing - 1 into the half of the ring that row j is not in
     // (read from row j + kRingFill - 1 on, many barriers later)
@@ -289,18 +305,28 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
     // ---- draft segment -> registers
     float xz[NE];
+    const float keep = zero_row ? 0.f : 1.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int v = tid + i * NT;
       if (v < nvec) {
         load_group<TZ, EPV>(zb + size_t(v) * ZB, &xz[i * EPV]);
+        if constexpr (HAS_B) {  // z = keep * base + bias
+          float b8[EPV];
+          load_group<float, EPV>(bb + size_t(v) * BB, b8);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) xz[i * EPV + e] = fmaf(xz[i * EPV + e], keep, b8[e]);
+        }
       } else {
 #pragma unroll
         for (int e = 0; e < EPV; ++e) xz[i * EPV + e] = -INFINITY;
       }
     }
-    if (tid == 0 && tv >= 0 && tv < nvec)
-      ctrl->ztid = load_elem<TZ>(zb + size_t(tv) * ZB + size_t(te) * sizeof(TZ));
+    if (tid == 0 && tv >= 0 && tv < nvec) {
+      float zt = load_elem<TZ>(zb + size_t(tv) * ZB + size_t(te) * sizeof(TZ));
+      if constexpr (HAS_B) zt = fmaf(zt, keep, load_elem<float>(bb + size_t(tv) * BB + size_t(te) * 4));
+      ctrl->ztid = zt;
+    }
     __syncthreads();  // the draft buffer is free again
     if (tid == 0) {
       // HAS_T: draft buffer + the teacher buffer of row j-1 (its pass 2 is done).
@@ -456,7 +482,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     // ---- pass 3: dlogits = p*(cce - cl1*S) + cl1*u, minus cce at the target id
     if (bwd) {
       // an invalid Markov slot's corrected row is a constant: nothing flows to base
-      const bool zero_out = kMarkov && a.invalid_zero && a.valid[row] == 0;
+      const bool zero_out = zero_row;
       const float g = a.grad_scale ? *a.grad_scale : 1.f;
       const float gw = zero_out ? 0.f : g * ctrl->rw[j % kRing];
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
@@ -517,15 +543,16 @@ struct LaunchCache {
 };
 
 template <typename TZ, typename TT, typename TO, int CL>
-size_t smem_bytes(int64_t V, bool has_t) {
+size_t smem_bytes(int64_t V, bool has_t, bool has_b) {
   constexpr int EPV = VecTraits<TO>::EPV;
   const int64_t vvec = V / EPV;
   const int64_t seg_vec = (vvec + CL - 1) / CL;
   const size_t zseg = size_t(seg_vec) * EPV * sizeof(TZ), tseg = size_t(seg_vec) * EPV * sizeof(TT);
-  return (has_t ? zseg + 2 * tseg : 2 * zseg) + sizeof(Ctrl<CL * 16>);
+  const size_t bseg = has_b ? size_t(seg_vec) * EPV * 4 : 0;
+  return (has_t ? zseg + bseg + 2 * tseg : 2 * (zseg + bseg)) + sizeof(Ctrl<CL * 16>);
 }
 
-template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T>
+template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T, bool HAS_B>
 cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   constexpr int EPV = VecTraits<TO>::EPV;
   SweepArgs a = a0;
@@ -533,10 +560,11 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   a.seg_vec = (a.vvec + CL - 1) / CL;
   a.nbuf = 2;
   // at least the report's reduction scratch (reused at the end)
-  const size_t smem = std::max<size_t>(smem_bytes<TZ, TT, TO, CL>(a.V, HAS_T), size_t(NT / 32) * kNAcc * sizeof(double));
+  const size_t smem = std::max<size_t>(smem_bytes<TZ, TT, TO, CL>(a.V, HAS_T, HAS_B),
+                                       size_t(NT / 32) * kNAcc * sizeof(double));
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
-  auto kern = sweep_kernel<TZ, TT, TO, CL, NT, NV, HAS_T>;
+  auto kern = sweep_kernel<TZ, TT, TO, CL, NT, NV, HAS_T, HAS_B>;
   static LaunchCache cache;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -600,29 +628,29 @@ struct Build {
 constexpr int kNumBuilds = 5;
 constexpr Build kBf16Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {4, 512, 10}, {8, 512, 5}};
 constexpr Build kF32Builds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 8}, {8, 512, 10}, {16, 512, 5}};
-// FP32 draft or teacher rows of the heads with bf16 dlogits
-constexpr Build kHeadBuilds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}, {8, 512, 5}};
+// the heads' kinds (Markov bias rows, FP32 teacher chunks) with bf16 logits
+constexpr Build kHeadBuilds[kNumBuilds] = {{1, 256, 1}, {2, 512, 2}, {4, 512, 4}, {8, 512, 5}, {16, 512, 3}};
 
 using bf16 = __nv_bfloat16;
 
 template <typename TZ, typename TT, typename TO>
-size_t smem_for(int cl, int64_t V, bool has_t) {
+size_t smem_for(int cl, int64_t V, bool has_t, bool has_b) {
   switch (cl) {
-    case 1: return smem_bytes<TZ, TT, TO, 1>(V, has_t);
-    case 2: return smem_bytes<TZ, TT, TO, 2>(V, has_t);
-    case 4: return smem_bytes<TZ, TT, TO, 4>(V, has_t);
-    case 8: return smem_bytes<TZ, TT, TO, 8>(V, has_t);
-    default: return smem_bytes<TZ, TT, TO, 16>(V, has_t);
+    case 1: return smem_bytes<TZ, TT, TO, 1>(V, has_t, has_b);
+    case 2: return smem_bytes<TZ, TT, TO, 2>(V, has_t, has_b);
+    case 4: return smem_bytes<TZ, TT, TO, 4>(V, has_t, has_b);
+    case 8: return smem_bytes<TZ, TT, TO, 8>(V, has_t, has_b);
+    default: return smem_bytes<TZ, TT, TO, 16>(V, has_t, has_b);
   }
 }
 
 size_t kind_smem(int kind, int cl, int64_t V, bool has_t) {
   switch (kind) {
-    case kSweepBf16: return smem_for<bf16, bf16, bf16>(cl, V, has_t);
-    case kSweepF32: return smem_for<float, float, float>(cl, V, has_t);
-    case kSweepZ32: return smem_for<float, bf16, bf16>(cl, V, has_t);
-    case kSweepT32: return smem_for<bf16, float, bf16>(cl, V, has_t);
-    default: return smem_for<float, float, bf16>(cl, V, has_t);
+    case kSweepBf16: return smem_for<bf16, bf16, bf16>(cl, V, has_t, false);
+    case kSweepF32: return smem_for<float, float, float>(cl, V, has_t, false);
+    case kSweepZ32: return smem_for<bf16, bf16, bf16>(cl, V, has_t, true);
+    case kSweepT32: return smem_for<bf16, float, bf16>(cl, V, has_t, false);
+    default: return smem_for<bf16, float, bf16>(cl, V, has_t, true);
   }
 }
 
@@ -636,30 +664,31 @@ int pick_build(int kind, int64_t V, bool has_t) {
   return -1;
 }
 
-template <typename TZ, typename TT, typename TO, bool HT>
+template <typename TZ, typename TT, typename TO, bool HT, bool HB>
 cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
-  if constexpr (sizeof(TZ) == 4 && sizeof(TO) == 4) {
+  if constexpr (sizeof(TZ) == 4) {
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 8, HT>(a, s);
-      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 10, HT>(a, s);
-      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 8, HT, HB>(a, s);
+      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 10, HT, HB>(a, s);
+      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 5, HT, HB>(a, s);
     }
-  } else if constexpr (sizeof(TZ) == 2 && sizeof(TT) == 2) {
+  } else if constexpr (sizeof(TT) == 2 && !HB) {
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT>(a, s);
-      case 3: return launch_cfg<TZ, TT, TO, 4, 512, 10, HT>(a, s);
-      case 4: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s);
+      case 3: return launch_cfg<TZ, TT, TO, 4, 512, 10, HT, HB>(a, s);
+      case 4: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT, HB>(a, s);
     }
   } else {
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT>(a, s);
-      default: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s);
+      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT, HB>(a, s);
+      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 3, HT, HB>(a, s);
     }
   }
   return cudaErrorInvalidValue;
@@ -674,15 +703,18 @@ cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStre
   if (i < 0) return cudaErrorInvalidValue;
   switch (kind) {
     case kSweepBf16:
-      return has_target ? dispatch<bf16, bf16, bf16, true>(i, a, s) : dispatch<bf16, bf16, bf16, false>(i, a, s);
+      return has_target ? dispatch<bf16, bf16, bf16, true, false>(i, a, s)
+                        : dispatch<bf16, bf16, bf16, false, false>(i, a, s);
     case kSweepF32:
-      return has_target ? dispatch<float, float, float, true>(i, a, s) : dispatch<float, float, float, false>(i, a, s);
+      return has_target ? dispatch<float, float, float, true, false>(i, a, s)
+                        : dispatch<float, float, float, false, false>(i, a, s);
     case kSweepZ32:
-      return has_target ? dispatch<float, bf16, bf16, true>(i, a, s) : dispatch<float, bf16, bf16, false>(i, a, s);
+      return has_target ? dispatch<bf16, bf16, bf16, true, true>(i, a, s)
+                        : dispatch<bf16, bf16, bf16, false, true>(i, a, s);
     case kSweepT32:
-      return dispatch<bf16, float, bf16, true>(i, a, s);
+      return dispatch<bf16, float, bf16, true, false>(i, a, s);
     case kSweepZT32:
-      return dispatch<float, float, bf16, true>(i, a, s);
+      return dispatch<bf16, float, bf16, true, true>(i, a, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -691,12 +723,12 @@ cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStre
 // dlogits from saved row statistics: one more read of the logits, no reductions.
 // Covers the supervised rows of list positions [row0, row1) and, with do_zero, the
 // unsupervised rows.
-template <typename TZ, typename TT, typename TO, bool HAS_T>
+template <typename TZ, typename TT, typename TO, bool HAS_T, bool HAS_B>
 __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a) {
   constexpr int EPV = VecTraits<TO>::EPV;
   constexpr int ZB = EPV * int(sizeof(TZ));
   constexpr int TB = EPV * int(sizeof(TT));
-  constexpr bool kMarkov = sizeof(TZ) == 4 && sizeof(TO) == 2;
+  constexpr bool kMarkov = HAS_B;
   constexpr bool kTChunk = sizeof(TT) == 4 && sizeof(TO) == 2;
   const int vvec = int(a.V / EPV);
   const int n_sup = max(0, min(a.ws.hdr->n_sup, a.row1) - a.row0);
@@ -720,13 +752,19 @@ __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a) {
     const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S), kzero = cce - cl1 * S;
     const float lz2 = st[kStLseD] * kLog2e, lt2 = st[kStLseT] * kLog2e;
     const int64_t tok = a.tids[row];
-    const int64_t drow = (kMarkov && a.draft_compact) ? sidx : row;
     const int64_t trow = (kTChunk && a.target_compact) ? int64_t(idx) : row;
-    const uint8_t* zr = static_cast<const uint8_t*>(a.draft) + size_t(drow) * a.ld_d * sizeof(TZ);
+    const uint8_t* zr = static_cast<const uint8_t*>(a.draft) + size_t(row) * a.ld_d * sizeof(TZ);
+    const float* br = HAS_B ? a.bias + size_t(sidx) * a.ld_b : nullptr;
     const uint8_t* tr = static_cast<const uint8_t*>(a.target) + size_t(trow) * a.ld_t * sizeof(TT);
     for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < vvec; v += gridDim.x * blockDim.x) {
       float z[EPV], t[EPV], o[EPV];
       load_group<TZ, EPV>(zr + size_t(v) * ZB, z);
+      if constexpr (HAS_B) {  // a valid slot (the zero rows were handled above): z = base + bias
+        float b8[EPV];
+        load_group<float, EPV>(reinterpret_cast<const uint8_t*>(br + size_t(v) * EPV), b8);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) z[e] += b8[e];
+      }
       if constexpr (HAS_T) load_group<TT, EPV>(tr + size_t(v) * TB, t);
 #pragma unroll
       for (int e = 0; e < EPV; ++e) {
@@ -751,22 +789,22 @@ cudaError_t launch_bwd_stream(int kind, bool has_target, const SweepArgs& a, int
   dim3 grid(gx > 0 ? gx : 1, unsigned(std::max<int64_t>(1, std::min<int64_t>(R, 65535))), 1);
   switch (kind) {
     case kSweepBf16:
-      if (has_target) bwd_stream_kernel<bf16, bf16, bf16, true><<<grid, 256, 0, s>>>(a);
-      else bwd_stream_kernel<bf16, bf16, bf16, false><<<grid, 256, 0, s>>>(a);
+      if (has_target) bwd_stream_kernel<bf16, bf16, bf16, true, false><<<grid, 256, 0, s>>>(a);
+      else bwd_stream_kernel<bf16, bf16, bf16, false, false><<<grid, 256, 0, s>>>(a);
       break;
     case kSweepF32:
-      if (has_target) bwd_stream_kernel<float, float, float, true><<<grid, 256, 0, s>>>(a);
-      else bwd_stream_kernel<float, float, float, false><<<grid, 256, 0, s>>>(a);
+      if (has_target) bwd_stream_kernel<float, float, float, true, false><<<grid, 256, 0, s>>>(a);
+      else bwd_stream_kernel<float, float, float, false, false><<<grid, 256, 0, s>>>(a);
       break;
     case kSweepZ32:
-      if (has_target) bwd_stream_kernel<float, bf16, bf16, true><<<grid, 256, 0, s>>>(a);
-      else bwd_stream_kernel<float, bf16, bf16, false><<<grid, 256, 0, s>>>(a);
+      if (has_target) bwd_stream_kernel<bf16, bf16, bf16, true, true><<<grid, 256, 0, s>>>(a);
+      else bwd_stream_kernel<bf16, bf16, bf16, false, true><<<grid, 256, 0, s>>>(a);
       break;
     case kSweepT32:
-      bwd_stream_kernel<bf16, float, bf16, true><<<grid, 256, 0, s>>>(a);
+      bwd_stream_kernel<bf16, float, bf16, true, false><<<grid, 256, 0, s>>>(a);
       break;
     case kSweepZT32:
-      bwd_stream_kernel<float, float, bf16, true><<<grid, 256, 0, s>>>(a);
+      bwd_stream_kernel<bf16, float, bf16, true, true><<<grid, 256, 0, s>>>(a);
       break;
     default:
       return cudaErrorInvalidValue;
