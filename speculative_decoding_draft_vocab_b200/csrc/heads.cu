@@ -74,65 +74,37 @@ __global__ void __launch_bounds__(256) heads_prep_kernel(const HeadsArgs a) {
   }
 }
 
-// ---- epilogue of the bias GEMM: the Markov bias rows W2.e (compact by supervised
-// position), 0 on invalid slots; the sweep adds them to the base rows it streams
-// (epilogue functors get a 32 x 32 block of the accumulator, rows m0.., columns n0..,
-// element (r, j) at t[r * tc::kTileLd + j]; lane j handles column n0 + j of every row)
+// ---- epilogues (tensor stores of 32 x 32 blocks through the GEMM's TMA epilogue)
+// bias GEMM: the Markov bias rows W2.e, compact by supervised position, 0 on invalid
+// slots and past the last supervised row; the sweep adds them to the base rows.
 struct BiasEpi {
+  static constexpr bool kTma = true;
   const int32_t* sup_list;
   const WsHeader* hdr;
   const uint8_t* valid;
-  float* bias;
-  int64_t ldb;
-  int V;
-  // lane l: bit 0 = row m0 + l is a valid slot, bit 1 = past the last supervised row
-  __device__ uint64_t row_state(int m0, int lane) const {
-    const int m = m0 + lane;
-    if (m >= hdr->n_sup) return 2;
-    return valid[sup_list[m]] != 0 ? 1 : 0;
+  __device__ float row_scale(int m) const {
+    if (m >= hdr->n_sup) return 0.f;
+    return valid[sup_list[m]] != 0 ? 1.f : 0.f;
   }
-  __device__ void operator()(int m0, int n0, int /*split*/, const float* t, int lane, uint64_t rs) const {
-    const int c = n0 + lane;
-    const uint32_t st = uint32_t(rs);
-#pragma unroll 8
-    for (int r = 0; r < 32; ++r) {
-      const uint32_t q = __shfl_sync(0xffffffffu, st, r);
-      if (c < V && !(q & 2u)) bias[size_t(m0 + r) * ldb + c] = (q & 1u) ? t[r * tc::kTileLd + lane] : 0.f;
-    }
-  }
+  __device__ int tma_mode() const { return 1; }
+  __device__ void coords(int m0, int n0, int, int& x, int& y, int& z) const { x = n0, y = m0, z = -1; }
 };
 
-// ---- epilogue of the dE GEMM: one partial per K split
+// dE GEMM: one partial per K split, [split][R][rank] (a 3-D output map)
 struct PartialEpi {
-  float* dep;
-  int R, rank;
-  __device__ uint64_t row_state(int, int) const { return 0; }
-  __device__ void operator()(int m0, int n0, int split, const float* t, int lane, uint64_t) const {
-    const int c = n0 + lane;
-    const int rows = min(32, R - m0);
-    if (c >= rank) return;
-    for (int r = 0; r < rows; ++r) dep[(size_t(split) * R + m0 + r) * rank + c] = t[r * tc::kTileLd + lane];
-  }
+  static constexpr bool kTma = true;
+  __device__ float row_scale(int) const { return 1.f; }
+  __device__ int tma_mode() const { return 1; }
+  __device__ void coords(int m0, int n0, int split, int& x, int& y, int& z) const { x = n0, y = m0, z = split; }
 };
 
-// ---- epilogue of the dW2 GEMM
+// dW2 GEMM: [V][rank], stored, or added to what is there (tensor reduce-add)
 struct WeightEpi {
-  float* dw2;
-  int V, rank, accumulate;
-  __device__ uint64_t row_state(int, int) const { return 0; }
-  __device__ void operator()(int m0, int n0, int /*split*/, const float* t, int lane, uint64_t) const {
-    const int c = n0 + lane;
-    const int rows = min(32, V - m0);
-    if (c >= rank) return;
-    float prev[32];
-    if (accumulate) {  // every load before any store
-#pragma unroll
-      for (int r = 0; r < 32; ++r) prev[r] = r < rows ? dw2[size_t(m0 + r) * rank + c] : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 32; ++r)
-      if (r < rows) dw2[size_t(m0 + r) * rank + c] = (accumulate ? prev[r] : 0.f) + t[r * tc::kTileLd + lane];
-  }
+  static constexpr bool kTma = true;
+  int accumulate;
+  __device__ float row_scale(int) const { return 1.f; }
+  __device__ int tma_mode() const { return accumulate ? 2 : 1; }
+  __device__ void coords(int m0, int n0, int, int& x, int& y, int& z) const { x = n0, y = m0, z = -1; }
 };
 
 // ---- dE = sum of the split partials (+ dc proj_e), then dW1[prev] += dE
@@ -220,20 +192,13 @@ __global__ void __launch_bounds__(256) gather_hidden_kernel(const TeacherArgs a)
   }
 }
 
-// epilogue of the teacher GEMM: FP32 teacher rows of the chunk, row i of the chunk
-// being supervised-list position row0 + i
+// teacher GEMM: FP32 teacher rows of the chunk, row i of the chunk being supervised-
+// list position row0 + i (rows past the last supervised row are never read)
 struct TeacherEpi {
-  const WsHeader* hdr;
-  float* t;
-  int64_t V;
-  int row0, rows;
-  __device__ uint64_t row_state(int, int) const { return 0; }
-  __device__ void operator()(int m0, int n0, int /*split*/, const float* tile, int lane, uint64_t) const {
-    const int64_t c = n0 + lane;
-    const int nr = min(min(32, rows - m0), hdr->n_sup - row0 - m0);
-    if (c >= V) return;
-    for (int r = 0; r < nr; ++r) t[size_t(m0 + r) * V + c] = tile[r * tc::kTileLd + lane];
-  }
+  static constexpr bool kTma = true;
+  __device__ float row_scale(int) const { return 1.f; }
+  __device__ int tma_mode() const { return 1; }
+  __device__ void coords(int m0, int n0, int, int& x, int& y, int& z) const { x = n0, y = m0, z = -1; }
 };
 
 inline int grid_for(int64_t n, int per_block) {
@@ -260,18 +225,21 @@ cudaError_t launch_teacher_chunk(const TeacherArgs& a, int64_t row0, cudaStream_
   CUtensorMap ma, mb;
   if (!tc::make_map(&ma, a.ws.hsup + size_t(row0) * a.Ht, rows, a.Ht, a.Ht, 64, 128)) return cudaErrorInvalidValue;
   if (!tc::make_map(&mb, a.lm_head, a.V, a.Ht, a.Ht, 64, 256)) return cudaErrorInvalidValue;
-  TeacherEpi epi{a.ws.hdr, a.ws.tchunk, a.V, int(row0), int(rows)};
-  return tc::gemm<256, false, false, 4>(ma, mb, int(rows), int(a.V), int(a.Ht), 1, epi, &a.ws.hdr->status, s,
-                                        &a.ws.hdr->n_sup, int(row0));
+  CUtensorMap mo;
+  if (!tc::make_out_map(&mo, a.ws.tchunk, rows, a.V, a.V)) return cudaErrorInvalidValue;
+  return tc::gemm<256, false, false, 4>(ma, mb, int(rows), int(a.V), int(a.Ht), 1, TeacherEpi{}, &a.ws.hdr->status,
+                                        s, &a.ws.hdr->n_sup, int(row0), &mo);
 }
 
 cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   if (!tc::make_map(&ma, a.ws.esup, a.R, a.rank, a.rank, 64, 128)) return cudaErrorInvalidValue;
   if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 256)) return cudaErrorInvalidValue;
-  BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.valid, a.ws.bias, a.V, int(a.V)};
+  CUtensorMap mo;
+  if (!tc::make_out_map(&mo, a.ws.bias, a.R, a.V, a.V)) return cudaErrorInvalidValue;
+  BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.valid};
   return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s,
-                                        &a.ws.hdr->n_sup, 0);
+                                        &a.ws.hdr->n_sup, 0, &mo);
 }
 
 cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
@@ -282,8 +250,10 @@ cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
     CUtensorMap ma, mb;
     if (!tc::make_map(&ma, a.dlogits, a.R, a.V, a.ld_g, 64, 128)) return cudaErrorInvalidValue;
     if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
-    PartialEpi pe{a.ws.dep, int(a.R), int(a.rank)};
-    e = tc::gemm<256, false, true, 4>(ma, mb, int(a.R), int(a.rank), int(a.V), splits, pe, &a.ws.hdr->status, s);
+    CUtensorMap mo;
+    if (!tc::make_out_map(&mo, a.ws.dep, a.R, a.rank, a.rank, splits, a.R * a.rank)) return cudaErrorInvalidValue;
+    e = tc::gemm<256, false, true, 4>(ma, mb, int(a.R), int(a.rank), int(a.V), splits, PartialEpi{},
+                                      &a.ws.hdr->status, s, nullptr, 0, &mo);
     if (e != cudaSuccess) return e;
     // dW2 = dlogits^T . E: A = dlogits as [R][V] (MN-major, M = vocabulary),
     // B = E by row [R][rank] (MN-major)
@@ -291,8 +261,10 @@ cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
       CUtensorMap ma2, mb2;
       if (!tc::make_map(&ma2, a.dlogits, a.R, a.V, a.ld_g, 64, 64)) return cudaErrorInvalidValue;
       if (!tc::make_map(&mb2, a.ws.eall, a.R, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
-      WeightEpi we{a.dw2, int(a.V), int(a.rank), a.accumulate};
-      e = tc::gemm<256, true, true, 4>(ma2, mb2, int(a.V), int(a.rank), int(a.R), 1, we, &a.ws.hdr->status, s);
+      CUtensorMap mo2;
+      if (!tc::make_out_map(&mo2, a.dw2, a.V, a.rank, a.rank)) return cudaErrorInvalidValue;
+      e = tc::gemm<256, true, true, 4>(ma2, mb2, int(a.V), int(a.rank), int(a.R), 1, WeightEpi{a.accumulate},
+                                       &a.ws.hdr->status, s, nullptr, 0, &mo2);
       if (e != cudaSuccess) return e;
     }
     de_reduce_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, splits);

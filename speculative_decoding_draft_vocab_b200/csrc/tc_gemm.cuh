@@ -6,11 +6,15 @@
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16
 //               per instruction, 4 per 64-wide stage) and tcgen05.commit
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator, one TMEM lane (= one tile
-//               row) per thread, 32 columns at a time, transposed through a padded
-//               32 x 33 shared tile so the epilogue functor can have the warp's lanes
-//               walk the columns of one row at a time (coalesced global accesses);
-//               the functor's row_state(m0, lane) is taken once per tile and handed
-//               to every 32-column block
+//               row) per thread, 32 columns at a time.  Two kinds of epilogue:
+//               - tensor store (Epi::kTma): the 32 x 32 block goes into a 128-byte-
+//                 swizzled shared tile (double-buffered per warp), each row scaled by
+//                 the functor's row_scale (0 drops a row), and one lane hands it to the
+//                 TMA engine as a tensor store or a tensor reduce-add into the output
+//                 tensor map;
+//               - functor: the block is transposed through a padded 32 x 33 shared
+//                 tile and the functor's lanes walk the columns of one row at a time;
+//                 its row_state(m0, lane) is taken once per tile.
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue of one
 // tile overlaps the MMAs of the next.  Operands are 128-byte-swizzled tiles, either
 // K-major (rows of 64 K values) or MN-major (rows of 64 M/N values per K index).
@@ -102,14 +106,42 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Epilogue staging: one 32 x 33 fp32 tile per epilogue warp.
+// Epilogue staging, 1024-byte aligned: per epilogue warp either one padded 32 x 33 fp32
+// tile (functor epilogue) or two 4 KB swizzled 32 x 32 fp32 tiles (tensor store).
 constexpr int kTileLd = 33;
-constexpr size_t kStageBytes = 4 * 32 * kTileLd * sizeof(float);
+constexpr size_t kStageBytes = 4 * 2 * 4096;
 
-// Shared memory a configuration needs (dynamic; the base is aligned to 1024 inside).
+// Shared memory a configuration needs (dynamic; the base is aligned to 1024 inside):
+// the operand ring, 1 KB of barriers, the epilogue staging.
 template <int BN, int STAGES>
 constexpr size_t gemm_smem_bytes() {
-  return size_t(STAGES) * (BM * BK * 2 + BN * BK * 2) + 1024 + 256 + kStageBytes;
+  return size_t(STAGES) * (BM * BK * 2 + BN * BK * 2) + 1024 + kStageBytes + 1024;
+}
+
+// Tensor store / reduce-add of a shared tile into the output tensor map (bulk group of
+// the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+               ::"l"(map), "r"(x), "r"(y), "r"(src) : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
+               ::"l"(map), "r"(x), "r"(y), "r"(z), "r"(src) : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];"
+               ::"l"(map), "r"(x), "r"(y), "r"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 // Work item w -> (m-tile, n-tile, k-split) and its range of 64-wide K chunks.  The
@@ -143,7 +175,7 @@ struct WorkMap {
 template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const WorkMap wm, const Epi epi, uint32_t* status) {
+            const __grid_constant__ CUtensorMap tmO, const WorkMap wm, const Epi epi, uint32_t* status) {
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
   constexpr uint32_t SA = BM * BK * 2, SB = BN * BK * 2, SS = SA + SB;
   constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
@@ -155,7 +187,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t accf0 = empty0 + 8 * STAGES;
   const uint32_t acce0 = accf0 + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
-  float* stage = reinterpret_cast<float*>(smem + size_t(STAGES) * SS + 256);
+  uint8_t* stage = smem + size_t(STAGES) * SS + 1024;  // 1024-byte aligned
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ME = wm.m_eff();  // the same in every role
@@ -239,7 +271,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else if (warp >= 2) {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
     const int q = warp & 3;
-    float* tile = stage + q * 32 * kTileLd;
+    float* tile = reinterpret_cast<float*>(stage + q * 8192);  // functor epilogue
+    const uint32_t tbuf0 = smem_u32(stage + q * 8192);         // tensor-store epilogue
+    int blk = 0;
     int tl = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x, ++tl) {
       int mt, nt, s, kc0, kc1;
@@ -249,22 +283,54 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       if (!mbar_wait_bounded(accf0 + 8 * b, use & 1u)) timed_out = true;
       fence_after_sync();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(b * BN);
-      // per-row state of the functor (e.g. gathered row ids), fetched once per tile
-      const uint64_t rs = epi.row_state(mt * BM + q * 32, lane);
+      const int m0 = mt * BM + q * 32;
+      if constexpr (Epi::kTma) {
+        const float scale = epi.row_scale(m0 + lane);  // this thread's row, once per tile
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(taddr + uint32_t(c * 32), v);
+        for (int c = 0; c < BN / 32; ++c, ++blk) {
+          float v[32];
+          tmem_ld32(taddr + uint32_t(c * 32), v);
+          const uint32_t buf = tbuf0 + uint32_t(blk & 1) * 4096u;
+          if (lane == 0) bulk_wait_read<1>();  // the store that last used this buffer has read it
+          __syncwarp();
+          // row `lane`: 128 bytes, 16-byte chunk k at chunk k ^ (lane % 8) (128-byte swizzle)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) tile[lane * kTileLd + i] = v[i];  // row lane, column i
-        __syncwarp();
-        // rows m0 .. m0 + 31, columns n0 .. n0 + 31: element (r, j) at tile[r * kTileLd + j]
-        epi(mt * BM + q * 32, nt * BN + c * 32, s, static_cast<const float*>(tile), lane, rs);
-        __syncwarp();
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(buf + uint32_t(lane) * 128u + uint32_t((k ^ (lane & 7)) * 16), v[4 * k] * scale,
+                         v[4 * k + 1] * scale, v[4 * k + 2] * scale, v[4 * k + 3] * scale);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            int x, y, z;
+            epi.coords(m0, nt * BN + c * 32, s, x, y, z);
+            if (epi.tma_mode() == 2) tma_reduce_add_2d(&tmO, buf, x, y);
+            else if (z >= 0) tma_store_3d(&tmO, buf, x, y, z);
+            else tma_store_2d(&tmO, buf, x, y);
+            bulk_commit();
+          }
+        }
+      } else {
+        // per-row state of the functor (e.g. gathered row ids), fetched once per tile
+        const uint64_t rs = epi.row_state(m0, lane);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(taddr + uint32_t(c * 32), v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) tile[lane * kTileLd + i] = v[i];  // row lane, column i
+          __syncwarp();
+          // rows m0 .. m0 + 31, columns n0 .. n0 + 31: element (r, j) at tile[r * kTileLd + j]
+          epi(m0, nt * BN + c * 32, s, static_cast<const float*>(tile), lane, rs);
+          __syncwarp();
+        }
       }
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * b);
+    }
+    // the staging tiles stay until the TMA engine has read them
+    if constexpr (Epi::kTma) {
+      if (lane == 0) bulk_wait_read<0>();
     }
   }
   if (timed_out) atomicOr(status, kTimeoutFlag);

@@ -46,6 +46,22 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An FP32 output seen by tensor stores of 32 x 32 blocks (128-byte swizzle): a matrix
+// of `rows` x `cols` (row stride `ld` elements), or `planes` such matrices `plane`
+// elements apart (3-D).  Blocks reaching past the matrix are clipped.
+inline bool make_out_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                         uint64_t planes = 0, uint64_t plane = 0) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {cols, rows, planes};
+  const cuuint64_t strides[2] = {ld * 4, plane * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, planes ? 3 : 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -59,7 +75,9 @@ inline int sm_count() {
 // launch error.
 template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi>
 cudaError_t gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int ksplit, const Epi& epi,
-                 uint32_t* status, cudaStream_t s, const int32_t* m_bound = nullptr, int m_base = 0) {
+                 uint32_t* status, cudaStream_t s, const int32_t* m_bound = nullptr, int m_base = 0,
+                 const CUtensorMap* out = nullptr) {
+  if (Epi::kTma && out == nullptr) return cudaErrorInvalidValue;
   WorkMap wm;
   wm.m_bound = m_bound;
   wm.m_base = m_base;
@@ -76,7 +94,7 @@ cudaError_t gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K
   if (attr_err != cudaSuccess) return attr_err;
   const int grid = std::min(W, sm_count());
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kThreads, smem, s>>>(a, b, wm, epi, status);
+  kern<<<grid, kThreads, smem, s>>>(a, b, out ? *out : a, wm, epi, status);
   return cudaGetLastError();
 }
 

@@ -7,6 +7,7 @@
 using namespace dspark;
 
 struct SplitStoreEpi {  // partial of K split s at d[s][m][n]; the block is rows m0.., columns n0..
+  static constexpr bool kTma = false;
   float* d;
   int M, N;
   __device__ uint64_t row_state(int, int) const { return 0; }
