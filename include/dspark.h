@@ -208,7 +208,7 @@ DSPARK_API dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, co
  * a service of this library).  For callers that cannot allocate device memory or pass
  * a workspace, e.g. an operator plugin whose host framework owns all device memory, or
  * a runtime that forbids cudaMalloc/cudaFree while serving because they synchronise the
- * device: the workspace is a fixed __device__ array inside this library, 401,664 bytes,
+ * device: the workspace is a fixed __device__ array inside this library, 467,200 bytes,
  * held on every GPU that loads the library until the process exits.  Same problem,
  * params, outputs and gradients as dspark_loss_fwd; nothing is allocated.
  *  - Serves micro-batches of at most 8192 rows (B*N*K) without the Markov head (whose

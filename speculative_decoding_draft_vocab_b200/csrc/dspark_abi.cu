@@ -251,6 +251,7 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   pa.target_ids = prob->target_ids;
   pa.prev_ids = sh.has_markov ? prob->prev_ids : nullptr;
   pa.valid = prob->valid;
+  pa.invalid_zero = sh.has_markov && params->invalid_row_mode == 0;
   pa.gamma = params->gamma;
   pa.gamma_enabled = params->gamma_enabled;
   pa.ws = v;

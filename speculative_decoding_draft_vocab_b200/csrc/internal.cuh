@@ -48,6 +48,8 @@ struct WsView {
   int32_t* sup_list;   // [R] supervised rows in row order
   int32_t* zero_list;  // [R] unsupervised rows in row order
   int32_t* sup_index;  // [R] position of a row in sup_list, -1 if unsupervised
+  int32_t* sup_tok;    // [R] target id of the i-th supervised row (bit 31: all-zero corrected row)
+  float* sup_w;        // [R] loss weight of the i-th supervised row
   float* stats;        // [R][kStride]
   // Markov head (present when the problem has it)
   float* bias;         // [R][V] Markov bias rows W2.e (0 on invalid slots), compact by supervised position
@@ -83,7 +85,7 @@ constexpr int64_t kTeacherChunk = 512;
 constexpr int64_t teacher_chunk_rows(int64_t R) { return R < kTeacherChunk ? R : kTeacherChunk; }
 
 struct WsOffsets {
-  size_t hdr, m, w, sup, zero, sidx, stats, z, esup, eall, dep, de, hsup, tchunk, dpp, bytes;
+  size_t hdr, m, w, sup, zero, sidx, stok, sw, stats, z, esup, eall, dep, de, hsup, tchunk, dpp, bytes;
 };
 
 constexpr WsOffsets ws_offsets(const WsDims& d) {
@@ -102,6 +104,10 @@ constexpr WsOffsets ws_offsets(const WsDims& d) {
   off = align256(off + sizeof(int32_t) * R);
   o.sidx = off;
   off = align256(off + sizeof(int32_t) * R);
+  o.stok = off;
+  off = align256(off + sizeof(int32_t) * R);
+  o.sw = off;
+  off = align256(off + sizeof(float) * R);
   o.stats = off;
   off = align256(off + sizeof(float) * kStride * R);
   const size_t zr = d.markov ? R : 0, er = d.markov ? R * size_t(d.rank) : 0;
@@ -141,6 +147,8 @@ inline WsView ws_layout(void* base, const WsDims& d) {
   v.sup_list = reinterpret_cast<int32_t*>(b + o.sup);
   v.zero_list = reinterpret_cast<int32_t*>(b + o.zero);
   v.sup_index = reinterpret_cast<int32_t*>(b + o.sidx);
+  v.sup_tok = reinterpret_cast<int32_t*>(b + o.stok);
+  v.sup_w = reinterpret_cast<float*>(b + o.sw);
   v.stats = reinterpret_cast<float*>(b + o.stats);
   v.bias = d.markov ? reinterpret_cast<float*>(b + o.z) : nullptr;
   v.esup = d.markov ? reinterpret_cast<uint16_t*>(b + o.esup) : nullptr;
@@ -168,6 +176,7 @@ struct PrologueArgs {
   const int64_t* target_ids;
   const int64_t* prev_ids;   // checked on valid rows when non-null
   const uint8_t* valid;
+  int32_t invalid_zero;      // Markov head: an invalid slot's corrected row is all zero
   float gamma;
   int32_t gamma_enabled;
   WsView ws;

@@ -267,15 +267,14 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
   // per-row scalars (row and target id fit 32 bits: R < 2^31, V <= 2^30) of the rows
   // j .. j + kRingFill - 1 in a shared ring, refilled kRingFill rows ahead
-  // (with the Markov head bit 31 of the target id marks an all-zero corrected row)
+  // (the prologue wrote them compact by supervised position; with the Markov head bit 31
+  // of the target id marks an all-zero corrected row)
   auto fill_ring = [&](int j0, int cnt) {
     if (tid < cnt && j0 + tid < my_n) {
-      const int32_t r = a.ws.sup_list[sidx_of(j0 + tid)];
-      int32_t t = int32_t(a.tids[r]);
-      if (kMarkov && a.invalid_zero && a.valid[r] == 0) t |= int32_t(0x80000000u);
-      ctrl->rrow[(j0 + tid) % kRing] = r;
-      ctrl->rtok[(j0 + tid) % kRing] = t;
-      ctrl->rw[(j0 + tid) % kRing] = a.ws.w[r];
+      const int64_t si = sidx_of(j0 + tid);
+      ctrl->rrow[(j0 + tid) % kRing] = a.ws.sup_list[si];
+      ctrl->rtok[(j0 + tid) % kRing] = a.ws.sup_tok[si];
+      ctrl->rw[(j0 + tid) % kRing] = a.ws.sup_w[si];
     }
   };
   fill_ring(0, kRing);
