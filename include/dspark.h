@@ -148,7 +148,8 @@ typedef struct {
   float* conf_rows;            /* [R] confidence logit used per row, or NULL            */
 } dspark_fwd_out_t;
 
-/* Backward outputs.  dlogits is written for EVERY row (zeros where unsupervised). */
+/* Backward outputs.  dlogits is written for EVERY row (zeros where unsupervised).  The
+ * head gradients (dW1, dW2, dconf_w, dhidden) must be 16-byte aligned. */
 typedef struct {
   const float* grad_scale;     /* device scalar g = d(objective)/d(loss_num); NULL = 1  */
   void* dlogits;               /* [R, V] dL/d(base draft logits), logits dtype          */

@@ -129,6 +129,10 @@ dspark_status_t check_grads(const dspark_problem_t* p, const dspark_grads_t* g) 
   const size_t es = elem_size(p->logits_dtype);
   if (g->dlogits_ld < p->V) return DSPARK_ERR_INVALID_ARG;
   if (!aligned16(g->dlogits) || (g->dlogits_ld * es) % 16) return DSPARK_ERR_ALIGNMENT;
+  // head gradients are written in 16-byte vectors or by tensor stores
+  if ((g->dW1 && !aligned16(g->dW1)) || (g->dW2 && !aligned16(g->dW2)) || (g->dhidden && !aligned16(g->dhidden)) ||
+      (g->dconf_w && !aligned16(g->dconf_w)))
+    return DSPARK_ERR_ALIGNMENT;
   return DSPARK_OK;
 }
 

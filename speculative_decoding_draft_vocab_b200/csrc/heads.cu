@@ -115,7 +115,18 @@ __global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const
     const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
     float acc = 0.f;
     if (live) {
-      for (int s = 0; s < splits; ++s) acc += a.ws.dep[(size_t(s) * a.R + r) * a.rank + j];
+      const float* dp = a.ws.dep + size_t(r) * a.rank + j;
+      const size_t stride = size_t(a.R) * a.rank;
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;  // loads in flight together; fixed order
+      int s = 0;
+      for (; s + 4 <= splits; s += 4) {
+        p0 += dp[s * stride];
+        p1 += dp[(s + 1) * stride];
+        p2 += dp[(s + 2) * stride];
+        p3 += dp[(s + 3) * stride];
+      }
+      for (; s < splits; ++s) p0 += dp[s * stride];
+      acc = (p0 + p1) + (p2 + p3);
       if (a.conf_w != nullptr && a.conf_with_markov)
         acc += a.ws.stats[r * kStride + kStDC] * bf(a.conf_w[a.H + j]);
       const int64_t pv = a.prev_ids[r];
@@ -126,56 +137,82 @@ __global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const
 }
 
 // ---- dproj = sum_r dc_r [h_r ; e_r] and dbias = sum_r dc_r: partial sums over blocks
-// of kDprojRows rows, then the partials in order (a fixed summation order)
+// of kDprojRows rows (eight columns per thread, every row's loads in flight together),
+// then the partials summed in a fixed order
 __global__ void __launch_bounds__(256) dproj_part_kernel(const HeadsArgs a) {
   const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
-  const int64_t j = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-  const int64_t r0 = int64_t(blockIdx.y) * kDprojRows, r1 = min(a.R, r0 + kDprojRows);
-  if (j >= cols) return;
-  float acc = 0.f;
-  for (int64_t r = r0; r < r1; ++r) {
-    if (a.ws.m[r] == 0 || a.valid[r] == 0) continue;  // the same r in every thread
-    const float dc = a.ws.stats[r * kStride + kStDC];
-    const float x = j < a.H ? bf(a.hidden[size_t(r) * a.H + j]) : bf(a.ws.eall[size_t(r) * a.rank + (j - a.H)]);
-    acc = fmaf(dc, x, acc);
+  const int64_t c8 = 8 * (blockIdx.x * int64_t(blockDim.x) + threadIdx.x);  // first of 8 columns
+  const int64_t r0 = int64_t(blockIdx.y) * kDprojRows;
+  if (c8 >= cols) return;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int rr = 0; rr < kDprojRows; ++rr) {
+    const int64_t r = r0 + rr;
+    if (r >= a.R) break;  // the same r in every thread
+    const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
+    const float dc = live ? a.ws.stats[r * kStride + kStDC] : 0.f;
+    const uint16_t* src = c8 < a.H ? a.hidden + size_t(r) * a.H + c8 : a.ws.eall + size_t(r) * a.rank + (c8 - a.H);
+    const uint4 q = *reinterpret_cast<const uint4*>(src);
+    const uint16_t* x = reinterpret_cast<const uint16_t*>(&q);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(dc, bf(x[k]), acc[k]);
   }
-  a.ws.dpp[size_t(blockIdx.y) * cols + j] = acc;
+  float4* out = reinterpret_cast<float4*>(a.ws.dpp + size_t(blockIdx.y) * cols + c8);
+  out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
+// 32 columns per block; 8 threads per column sum interleaved partials, combined in a
+// fixed order in shared memory
 __global__ void __launch_bounds__(256) dproj_final_kernel(const HeadsArgs a) {
   const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
   const int64_t nchunks = (a.R + kDprojRows - 1) / kDprojRows;
-  const int64_t j = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-  if (j < cols) {
-    float acc = 0.f;
-    for (int64_t c = 0; c < nchunks; ++c) acc += a.ws.dpp[size_t(c) * cols + j];
-    a.dconf_w[j] = a.accumulate ? a.dconf_w[j] + acc : acc;
+  const int cl = threadIdx.x & 31, part = threadIdx.x >> 5;
+  const int64_t j = blockIdx.x * 32 + cl;
+  __shared__ float sp[8][32];
+  float acc = 0.f;
+  if (j < cols)
+    for (int64_t c = part; c < nchunks; c += 8) acc += a.ws.dpp[size_t(c) * cols + j];
+  sp[part][cl] = acc;
+  __syncthreads();
+  if (part == 0 && j < cols) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += sp[k][cl];
+    a.dconf_w[j] = a.accumulate ? a.dconf_w[j] + t : t;
   }
   if (blockIdx.x == 0) {
-    __shared__ float part[8];
-    float acc = 0.f;
+    __shared__ float pb[8];
+    float b = 0.f;
     for (int64_t r = threadIdx.x; r < a.R; r += blockDim.x)
-      if (a.ws.m[r] != 0 && a.valid[r] != 0) acc += a.ws.stats[r * kStride + kStDC];
+      if (a.ws.m[r] != 0 && a.valid[r] != 0) b += a.ws.stats[r * kStride + kStDC];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
+    for (int off = 16; off > 0; off >>= 1) b += __shfl_xor_sync(0xffffffffu, b, off);
+    if ((threadIdx.x & 31) == 0) pb[threadIdx.x / 32] = b;
     __syncthreads();
     if (threadIdx.x == 0) {
       float t = 0.f;
-      for (int i = 0; i < int(blockDim.x / 32); ++i) t += part[i];
+      for (int i = 0; i < int(blockDim.x / 32); ++i) t += pb[i];
       if (a.dconf_b) *a.dconf_b = a.accumulate ? *a.dconf_b + t : t;
     }
   }
 }
 
-// ---- dh_r = dc_r proj_h on supervised valid rows, 0 elsewhere (bf16)
+// ---- dh_r = dc_r proj_h on supervised valid rows, 0 elsewhere (bf16, eight per thread)
 __global__ void __launch_bounds__(256) dhidden_kernel(const HeadsArgs a) {
-  const int64_t n = a.R * a.H;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = i / a.H, j = i - r * a.H;
+  const int64_t n8 = a.R * a.H / 8;
+  const int64_t h8 = a.H / 8;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / h8, j8 = (i - r * h8) * 8;
     const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
-    const float v = live ? a.ws.stats[r * kStride + kStDC] * bf(a.conf_w[j]) : 0.f;
-    a.dhidden[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    const float dc = live ? a.ws.stats[r * kStride + kStDC] : 0.f;
+    const uint4 w = *reinterpret_cast<const uint4*>(a.conf_w + j8);
+    const uint16_t* wv = reinterpret_cast<const uint16_t*>(&w);
+    uint4 o;
+    uint16_t* ov = reinterpret_cast<uint16_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ov[k] = __bfloat16_as_ushort(__float2bfloat16_rn(dc * bf(wv[k])));
+    *reinterpret_cast<uint4*>(a.dhidden + size_t(r) * a.H + j8) = o;
   }
 }
 
@@ -273,13 +310,13 @@ cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
   if (a.conf_w != nullptr) {
     const int64_t cols = a.H + (a.conf_with_markov ? a.rank : 0);
     if (a.dconf_w != nullptr) {
-      const dim3 grid(unsigned((cols + 255) / 256), unsigned((a.R + kDprojRows - 1) / kDprojRows));
+      const dim3 grid(unsigned((cols / 8 + 255) / 256), unsigned((a.R + kDprojRows - 1) / kDprojRows));
       dproj_part_kernel<<<grid, 256, 0, s>>>(a);
-      dproj_final_kernel<<<unsigned((cols + 255) / 256), 256, 0, s>>>(a);
+      dproj_final_kernel<<<unsigned((cols + 31) / 32), 256, 0, s>>>(a);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.dhidden != nullptr) {
-      dhidden_kernel<<<grid_for(a.R * a.H, 256), 256, 0, s>>>(a);
+      dhidden_kernel<<<grid_for(a.R * a.H / 8, 256), 256, 0, s>>>(a);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }

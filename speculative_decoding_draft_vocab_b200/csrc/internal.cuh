@@ -77,7 +77,7 @@ struct WsDims {
 };
 
 // Rows per partial sum of the confidence head's weight gradient.
-constexpr int64_t kDprojRows = 64;
+constexpr int64_t kDprojRows = 16;
 
 // Supervised rows per teacher chunk (the FP32 teacher rows of a chunk are the only
 // vocabulary-wide teacher buffer; a multiple of the GEMM's 128-row tile).

@@ -237,3 +237,14 @@ def test_teacher_from_hidden_validation_and_workspace(abi):
         R = B * N * K
         assert n >= base + R * 256 * 2 + min(R, 512) * 4096 * 4
         assert n < base + R * 256 * 2 + min(R, 512) * 4096 * 4 + 4096
+
+
+def test_head_gradient_alignment(abi):
+    p = _with_conf_head(abi, _with_markov(abi, _problem(abi)), with_markov=1)
+    g = abi.dspark_grads_t()
+    g.dlogits, g.dlogits_ld = ctypes.c_void_p(0x70000), p.V
+    g.dhidden = ctypes.c_void_p(0x80008)  # not 16-byte aligned
+    assert _fwd(abi, p, _params(abi), grads=g) == abi.DSPARK_ERR_ALIGNMENT
+    g.dhidden = None
+    g.dW2 = ctypes.c_void_p(0x90004)
+    assert _fwd(abi, p, _params(abi), grads=g) == abi.DSPARK_ERR_ALIGNMENT
