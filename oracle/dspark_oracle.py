@@ -35,6 +35,9 @@ the design notes of the repository):
   * report pairs: loss/ce/l1/conf = [sum w*term, num_tokens];
     accept = [sum m*a, num_tokens]; tau = [sum keep*tau_blk, sum keep].
   * without target logits: L1 = 0 (so accept = 1), CE only.
+  * pre-norm target hidden states (the vLLM case of the [TS-PR] review) get the
+    target's final RMS norm, y = w * x / sqrt(mean(x^2) + eps), before lm_head; the
+    normed state is rounded to bf16 once, as the norm's output in the model's dtype.
 
 Every function below is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, invariants, brute force and finite differences.
@@ -173,6 +176,19 @@ def markov_corrected_rows(base_rows, e_rows, valid_rows, w2, invalid_row_mode=0)
     return z
 
 
+def target_final_norm(hidden_rows, weight, eps) -> np.ndarray:
+    """The target's final RMS norm on pre-norm hidden states ([TS-PR] review of the
+    vLLM path: its stored last hidden states precede the final norm, which must be
+    applied before lm_head): y = w * x / sqrt(mean_h(x^2) + eps), each row on its own,
+    computed in FP64 and rounded once to bf16 (the dtype in which the norm hands its
+    output to the lm_head product)."""
+    import torch
+    x = np.asarray(hidden_rows, dtype=np.float64)
+    w = np.asarray(weight, dtype=np.float64).reshape(-1)
+    y = w * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + float(eps))
+    return torch.from_numpy(y).to(torch.bfloat16).double().numpy()
+
+
 def teacher_rows_from_hidden(hidden_rows, lm_head) -> np.ndarray:
     """t = lm_head @ h per row: [TS-PR] scope list, the teacher distribution comes
     from the target model's output projection applied to its last hidden state
@@ -243,6 +259,7 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
                 confidence_logits=None, prev_ids=None, valid=None, markov_w1=None,
                 markov_w2=None, draft_hidden=None, conf_w=None, conf_b=None,
                 conf_with_markov=False, target_hidden=None, lm_head=None,
+                target_norm_weight=None, target_norm_eps=1e-6,
                 ce_alpha=0.1, l1_alpha=0.9, conf_alpha=1.0, gamma: Optional[float] = 4.0,
                 grad_scale=1.0, invalid_row_mode=0, want_grads=True,
                 rows: Optional[np.ndarray] = None, keep_rows: Optional[np.ndarray] = None,
@@ -315,7 +332,10 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
         else:
             z_rows = base
         if lm_head is not None:
-            t_rows = _matmul_rows_by_table(_as_rows(target_hidden, R)[rr], lm_head)
+            h_rows = _as_rows(target_hidden, R)[rr]
+            if target_norm_weight is not None:
+                h_rows = target_final_norm(h_rows, target_norm_weight, target_norm_eps)
+            t_rows = _matmul_rows_by_table(h_rows, lm_head)
         elif target_r is not None:
             t_rows = target_r[rr].astype(np.float64)
         else:

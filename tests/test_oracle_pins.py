@@ -387,6 +387,50 @@ def test_reference_scale_tensor_size_from_pages():
     gib = g["num_blocks"] * g["block_size"] * g["vocab"] * 4 / 2 ** 30
     assert round(gib, 2) == g["value"]
 
+def _bf16(x):
+    import torch
+    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def test_target_final_norm_closed_forms():
+    """RMS norm: a constant row c*1 normalises to sign(c) * w (eps = 0); with w = 1 and
+    eps = 0 every row has unit mean square (to bf16 rounding); scaling a row by a power
+    of two changes nothing; an all-zero row stays zero with eps > 0."""
+    rng = np.random.default_rng(31)
+    Ht = 64
+    w = _bf16(rng.normal(1.0, 0.2, Ht))
+    for c in (3.0, -0.25, 17.5):
+        y = O.target_final_norm(np.full((1, Ht), c), w, 0.0)
+        np.testing.assert_array_equal(y[0], np.sign(c) * w)
+    x = rng.normal(0, 2.0, (5, Ht))
+    y = O.target_final_norm(x, np.ones(Ht), 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=1), 1.0, rtol=2 * 2.0 ** -8)
+    np.testing.assert_array_equal(O.target_final_norm(4.0 * x, w, 0.0), O.target_final_norm(x, w, 0.0))
+    np.testing.assert_array_equal(O.target_final_norm(np.zeros((2, Ht)), w, 1e-6), 0.0)
+    # by hand for one row: w * x / sqrt(mean(x^2) + eps), rounded to bf16
+    xr = np.array([[1.0, -2.0, 3.0, 0.5]])
+    wr = np.array([1.0, 0.5, 2.0, -1.0])
+    ms = (1.0 + 4.0 + 9.0 + 0.25) / 4.0
+    want = _bf16(wr * xr[0] / math.sqrt(ms + 0.1))
+    np.testing.assert_array_equal(O.target_final_norm(xr, wr, 0.1)[0], want)
+
+
+def test_teacher_from_prenorm_hidden_equals_normed_teacher():
+    """The loss on pre-norm hidden states with the norm weight equals the loss on the
+    normed states given directly."""
+    rng = np.random.default_rng(32)
+    B, N, K, V, Ht = 1, 2, 3, 12, 16
+    h = rng.normal(0, 3.0, (B, N, K, Ht))
+    w = _bf16(rng.normal(1.0, 0.3, Ht))
+    lm = rng.normal(0, 0.3, (V, Ht))
+    d, _, ids, ev = _rand_problem(rng, B, N, K, V)
+    a = O.dspark_loss(d, ids, ev, target_hidden=h, lm_head=lm, target_norm_weight=w, target_norm_eps=1e-5)
+    hn = O.target_final_norm(h.reshape(-1, Ht), w, 1e-5).reshape(h.shape)
+    b = O.dspark_loss(d, ids, ev, target_hidden=hn, lm_head=lm)
+    assert a["loss_num"] == b["loss_num"]
+    for r in a["dlogits"]:
+        np.testing.assert_array_equal(a["dlogits"][r], b["dlogits"][r])
+
 
 # --------------------------------------------------------------- planted mistakes
 def _mutant_half_l1(z, t, tid, _orig=O.row_terms):
@@ -424,11 +468,17 @@ def _mutant_w2_transposed(base_rows, e_rows, valid_rows, w2, invalid_row_mode=0,
     return _orig(base_rows, e_rows, valid_rows, w2[:, ::-1], invalid_row_mode)
 
 
+def _mutant_norm_no_square(hidden_rows, weight, eps, _orig=O.target_final_norm):
+    x = np.asarray(hidden_rows, dtype=np.float64)
+    return _orig(np.abs(x) ** 0.5 * np.sign(x), weight, eps)
+
+
 @pytest.mark.parametrize("target,mutant,pins", [
     ("row_terms", _mutant_half_l1, [test_disjoint_saturated_rows_match_the_pages_values]),
     ("row_terms", _mutant_no_S, [lambda: test_finite_differences_all_gradients(False, "given")]),
     ("row_terms", _mutant_sign_flip, [lambda: test_finite_differences_all_gradients(False, "given")]),
     ("loss_weights", _mutant_decay_index, [test_weights_slot0_is_one_and_decay_ratio_constant]),
+    ("target_final_norm", _mutant_norm_no_square, [test_target_final_norm_closed_forms]),
     ("markov_corrected_rows", _mutant_w2_transposed,
      [test_markov_bias_matches_explicit_loops_and_zero_w2_reduces]),
 ])
