@@ -60,7 +60,7 @@ def workload_desc(name: str, inp) -> str:
     return ", ".join(parts)
 
 
-WEIGHTS = ("markov_w1", "markov_w2", "conf_w", "conf_b", "lm_head")  # resident across steps
+WEIGHTS = ("markov_w1", "markov_w2", "conf_w", "conf_b", "lm_head", "target_norm_weight")  # resident
 
 
 def algorithmic_bytes(inp, n_sup: int) -> int:
@@ -120,7 +120,9 @@ def oracle_kwargs(inp):
                 confidence_logits=a(inp.confidence_logits), prev_ids=a(inp.prev_ids), valid=a(inp.valid),
                 markov_w1=a(inp.markov_w1), markov_w2=a(inp.markov_w2), draft_hidden=a(inp.draft_hidden),
                 conf_w=a(inp.conf_w), conf_b=a(inp.conf_b), conf_with_markov=inp.conf_with_markov,
-                target_hidden=a(inp.target_hidden), lm_head=a(inp.lm_head), gamma=inp.gamma)
+                target_hidden=a(inp.target_hidden), lm_head=a(inp.lm_head),
+                target_norm_weight=a(inp.target_norm_weight), target_norm_eps=inp.target_norm_eps,
+                gamma=inp.gamma)
 
 
 def sources_sha() -> str:

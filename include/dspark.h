@@ -125,6 +125,12 @@ typedef struct {
   const void* conf_w;          /* bf16 [hidden_size (+ markov_rank)]: proj.weight       */
   const float* conf_b;         /* [1] proj.bias                                         */
   int64_t conf_with_markov;    /* 1: proj input is [hidden ; markov embedding]          */
+  /* pre-norm teacher hidden states (NULL when target_hidden is already normed): the
+   * target's final RMS norm, y = w * x / sqrt(mean(x^2) + eps) per row, rounded to bf16,
+   * is applied to target_hidden before lm_head (TorchSpec pull request #132, review of
+   * the vLLM path, whose stored last hidden states precede the final norm) */
+  const void* target_norm_weight; /* bf16 [target_hidden_size], 16-byte aligned        */
+  float target_norm_eps;       /* e.g. 1e-6                                             */
 } dspark_problem_t;
 
 typedef struct {

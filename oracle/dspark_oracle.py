@@ -180,8 +180,8 @@ def target_final_norm(hidden_rows, weight, eps) -> np.ndarray:
     """The target's final RMS norm on pre-norm hidden states ([TS-PR] review of the
     vLLM path: its stored last hidden states precede the final norm, which must be
     applied before lm_head): y = w * x / sqrt(mean_h(x^2) + eps), each row on its own,
-    computed in FP64 and rounded once to bf16 (the dtype in which the norm hands its
-    output to the lm_head product)."""
+    computed in FP64 and converted to bf16 through FP32 by torch's cast (the dtype in
+    which the norm hands its output to the lm_head product)."""
     import torch
     x = np.asarray(hidden_rows, dtype=np.float64)
     w = np.asarray(weight, dtype=np.float64).reshape(-1)

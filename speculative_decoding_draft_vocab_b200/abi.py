@@ -55,6 +55,7 @@ class dspark_problem_t(ctypes.Structure):
         ("markov_w1", c_vp), ("markov_w2", c_vp), ("markov_rank", c_i64),
         ("draft_hidden", c_vp), ("hidden_size", c_i64),
         ("conf_w", c_vp), ("conf_b", c_vp), ("conf_with_markov", c_i64),
+        ("target_norm_weight", c_vp), ("target_norm_eps", ctypes.c_float),
     ]
 
 

@@ -89,13 +89,16 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
     if (prm->gamma_enabled && !(prm->gamma > 0.f)) return DSPARK_ERR_INVALID_ARG;
     if (prm->invalid_row_mode != 0 && prm->invalid_row_mode != 1) return DSPARK_ERR_INVALID_ARG;
   }
+  if (p->target_norm_weight && !s.has_lm_head) return DSPARK_ERR_INVALID_ARG;
   if (s.has_lm_head) {
     if (!p->lm_head || !p->target_hidden || p->target_hidden_size <= 0) return DSPARK_ERR_INVALID_ARG;
     // the teacher rows come from the tensor cores in FP32; the sweep pairs them with
     // bf16 logits
     if (p->logits_dtype != DSPARK_BF16) return DSPARK_ERR_UNSUPPORTED;
-    if (p->target_hidden_size % 8 || !aligned16(p->lm_head) || !aligned16(p->target_hidden))
+    if (p->target_hidden_size % 8 || !aligned16(p->lm_head) || !aligned16(p->target_hidden) ||
+        (p->target_norm_weight && !aligned16(p->target_norm_weight)))
       return DSPARK_ERR_ALIGNMENT;
+    if (p->target_norm_weight && !(p->target_norm_eps >= 0.f)) return DSPARK_ERR_INVALID_ARG;
   }
   if (s.has_markov) {
     if (!p->markov_w1 || !p->markov_w2 || !p->prev_ids || !p->valid) return DSPARK_ERR_INVALID_ARG;
@@ -176,6 +179,8 @@ TeacherArgs teacher_args(const dspark_problem_t* p, const WsView& ws) {
   t.Ht = p->target_hidden_size;
   t.hidden = static_cast<const uint16_t*>(p->target_hidden);
   t.lm_head = static_cast<const uint16_t*>(p->lm_head);
+  t.norm_w = static_cast<const uint16_t*>(p->target_norm_weight);
+  t.norm_eps = p->target_norm_eps;
   t.ws = ws;
   return t;
 }

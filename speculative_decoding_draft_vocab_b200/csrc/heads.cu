@@ -216,7 +216,10 @@ __global__ void __launch_bounds__(256) dhidden_kernel(const HeadsArgs a) {
   }
 }
 
-// ---- teacher from hidden states: gather, then t = lm_head . h per supervised row
+// ---- teacher from hidden states: gather (with the target's final RMS norm when the
+// states are pre-norm: y = w * x / sqrt(mean(x^2) + eps)), then t = lm_head . y per
+// supervised row.  The norm runs in FP64 and its result goes to bf16 through FP32 (one
+// rounding each), so the bf16 values do not depend on the order of the sum of squares.
 __global__ void __launch_bounds__(256) gather_hidden_kernel(const TeacherArgs a) {
   const int warps = blockDim.x / 32;
   const int lane = threadIdx.x & 31;
@@ -225,7 +228,37 @@ __global__ void __launch_bounds__(256) gather_hidden_kernel(const TeacherArgs a)
     const int64_t row = a.ws.sup_list[si];
     const uint4* src = reinterpret_cast<const uint4*>(a.hidden + size_t(row) * a.Ht);
     uint4* dst = reinterpret_cast<uint4*>(a.ws.hsup + size_t(si) * a.Ht);
-    for (int64_t j = lane; j < a.Ht / 8; j += 32) dst[j] = src[j];
+    if (a.norm_w == nullptr) {
+      for (int64_t j = lane; j < a.Ht / 8; j += 32) dst[j] = src[j];
+      continue;
+    }
+    double ss = 0.0;
+    for (int64_t j = lane; j < a.Ht / 8; j += 32) {
+      const uint4 q = src[j];
+      const uint16_t* x = reinterpret_cast<const uint16_t*>(&q);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const double v = double(bf(x[k]));
+        ss = fma(v, v, ss);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const double rs = 1.0 / sqrt(ss / double(a.Ht) + double(a.norm_eps));
+    const uint4* wv = reinterpret_cast<const uint4*>(a.norm_w);
+    for (int64_t j = lane; j < a.Ht / 8; j += 32) {
+      const uint4 q = src[j], wq = wv[j];
+      const uint16_t* x = reinterpret_cast<const uint16_t*>(&q);
+      const uint16_t* w = reinterpret_cast<const uint16_t*>(&wq);
+      uint4 o;
+      uint16_t* ov = reinterpret_cast<uint16_t*>(&o);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float y = __double2float_rn(double(bf(w[k])) * double(bf(x[k])) * rs);
+        ov[k] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+      }
+      dst[j] = o;
+    }
   }
 }
 

@@ -295,6 +295,8 @@ struct TeacherArgs {
   int64_t R, V, Ht;
   const uint16_t* hidden;    // bf16 [R][Ht]
   const uint16_t* lm_head;   // bf16 [V][Ht]
+  const uint16_t* norm_w;    // bf16 [Ht] final RMS-norm weight, or null (already normed)
+  float norm_eps;
   WsView ws;
 };
 cudaError_t launch_gather_hidden(const TeacherArgs& a, cudaStream_t s);

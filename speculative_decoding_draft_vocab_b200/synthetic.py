@@ -79,6 +79,8 @@ class DSparkInputs:
     conf_with_markov: bool = False
     target_hidden: Optional[torch.Tensor] = None  # bf16 [B,N,K,Ht]
     lm_head: Optional[torch.Tensor] = None      # bf16 [V, Ht]
+    target_norm_weight: Optional[torch.Tensor] = None  # bf16 [Ht]: target_hidden is pre-norm
+    target_norm_eps: float = 1e-6
     gamma: Optional[float] = 4.0
     ce_alpha: float = 0.1
     l1_alpha: float = 0.9
@@ -128,14 +130,17 @@ def make_inputs(name: str = "recipe", device="cpu", seed: Optional[int] = None,
     ones after each prefix so the cumprod inside the loss has work to do),
     ``no_target`` (CE-only), ``gamma``, ``grad_scale``, ``conf_with_markov``,
     ``markov_std`` (std of both Markov tables; 0.02 is the initialisation scale, a
-    larger one makes the correction visible in tests), ``conf_bias``.
+    larger one makes the correction visible in tests), ``conf_bias``,
+    ``target_prenorm`` (teacher hidden states drawn before the target's final RMS norm:
+    N(0, 4) with a norm weight N(1, 0.1) and eps 1e-6; the labels are drawn from the
+    normed teacher).
     The default seed is 1234 + the configuration's index.
     """
     base = dict(CONFIGS[name])
     base.update(dict(hidden=HIDDEN, target_hidden_size=HIDDEN, rank=MARKOV_RANK,
                      target_vocab=None, valid_p=0.9, mask_holes=False, no_target=False,
                      gamma=4.0, grad_scale=1.0, conf_with_markov=None, markov_std=0.02,
-                     conf_bias=0.0))
+                     conf_bias=0.0, target_prenorm=False))
     unknown = set(overrides) - set(base)
     if unknown:
         raise TypeError(f"unknown overrides {sorted(unknown)}")
@@ -170,13 +175,17 @@ def make_inputs(name: str = "recipe", device="cpu", seed: Optional[int] = None,
     else:
         draft = _normal(gen, (B, N, K, V), 3.0, device, torch.bfloat16)
         target = (0.8 * draft.float() + _normal(gen, (B, N, K, V), 1.5, device)).to(torch.bfloat16)
+    norm_w = None
     if c["lm_head"]:
         Ht = c["target_hidden_size"]
-        target_hidden = _normal(gen, (B, N, K, Ht), 1.0, device, torch.bfloat16)
+        target_hidden = _normal(gen, (B, N, K, Ht), 4.0 if c["target_prenorm"] else 1.0, device, torch.bfloat16)
         lm_head = _normal(gen, (V, Ht), 0.02, device, torch.bfloat16)
         # the teacher rows only serve to draw labels here; the loss recomputes them
         teacher = torch.empty((R, V), dtype=torch.float32, device=device)
         h2 = target_hidden.reshape(R, Ht).float()
+        if c["target_prenorm"]:
+            norm_w = (1.0 + _normal(gen, (Ht,), 0.1, device)).to(torch.bfloat16)
+            h2 = h2 * torch.rsqrt(h2.pow(2).mean(-1, keepdim=True) + 1e-6) * norm_w.float()
         w = lm_head.float()
         for r0 in range(0, R, 64):
             teacher[r0:r0 + 64] = h2[r0:r0 + 64] @ w.t()
@@ -193,7 +202,8 @@ def make_inputs(name: str = "recipe", device="cpu", seed: Optional[int] = None,
     inp = DSparkInputs(B=B, N=N, K=K, V=V, dtype=c["dtype"], draft_logits=draft,
                        target_logits=target, target_ids=target_ids, eval_mask=eval_mask,
                        block_keep=block_keep, gamma=c["gamma"], grad_scale=c["grad_scale"],
-                       name=name, target_hidden=target_hidden, lm_head=lm_head)
+                       name=name, target_hidden=target_hidden, lm_head=lm_head,
+                       target_norm_weight=norm_w)
 
     # ---- Markov head ---------------------------------------------------------
     r = c["rank"]

@@ -50,6 +50,9 @@ def problem_struct(inp: DSparkInputs) -> abi.dspark_problem_t:
         p.target_hidden = _ptr(_need(inp.target_hidden, torch.bfloat16, "target_hidden"))
         p.lm_head = _ptr(_need(inp.lm_head, torch.bfloat16, "lm_head"))
         p.target_hidden_size = inp.lm_head.shape[1]
+        if inp.target_norm_weight is not None:
+            p.target_norm_weight = _ptr(_need(inp.target_norm_weight, torch.bfloat16, "target_norm_weight"))
+            p.target_norm_eps = float(inp.target_norm_eps)
     if inp.markov_w2 is not None:
         p.prev_ids = _ptr(_need(inp.prev_ids, torch.int64, "prev_ids"))
         p.markov_w1 = _ptr(_need(inp.markov_w1, torch.bfloat16, "markov_w1"))

@@ -59,7 +59,8 @@ def oracle_run(inp, rows=None, keep_rows=None, invalid_row_mode=0, want_grads=Tr
         valid=np32(inp.valid), markov_w1=np32(inp.markov_w1), markov_w2=np32(inp.markov_w2),
         draft_hidden=np32(inp.draft_hidden), conf_w=np32(inp.conf_w), conf_b=np64(inp.conf_b),
         conf_with_markov=inp.conf_with_markov, target_hidden=np32(inp.target_hidden),
-        lm_head=np32(inp.lm_head), ce_alpha=inp.ce_alpha, l1_alpha=inp.l1_alpha if (
+        lm_head=np32(inp.lm_head), target_norm_weight=np32(inp.target_norm_weight),
+        target_norm_eps=inp.target_norm_eps, ce_alpha=inp.ce_alpha, l1_alpha=inp.l1_alpha if (
             inp.target_logits is not None or inp.lm_head is not None) else 0.0,
         conf_alpha=inp.conf_alpha, gamma=inp.gamma, grad_scale=inp.grad_scale,
         invalid_row_mode=invalid_row_mode, want_grads=want_grads, rows=rows, keep_rows=keep_rows)

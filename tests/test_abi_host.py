@@ -248,3 +248,16 @@ def test_head_gradient_alignment(abi):
     g.dhidden = None
     g.dW2 = ctypes.c_void_p(0x90004)
     assert _fwd(abi, p, _params(abi), grads=g) == abi.DSPARK_ERR_ALIGNMENT
+
+
+def test_target_norm_validation(abi):
+    prm = _params(abi)
+    p = _problem(abi)
+    p.target_norm_weight = ctypes.c_void_p(0x110000)  # a norm weight without hidden states
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+    p = _with_lm_head(abi, _problem(abi))
+    p.target_norm_weight = ctypes.c_void_p(0x110008)
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_ALIGNMENT
+    p.target_norm_weight = ctypes.c_void_p(0x110000)
+    p.target_norm_eps = -1.0
+    assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG

@@ -94,3 +94,20 @@ def test_lm_head_teacher_config_every_row():
     inp = make_inputs("lm_head_teacher", device="cuda")
     call, ref = _run(inp)
     assert np.all(ref["l1"][ref["rows"]] > 0)
+
+
+@pytest.mark.parametrize("heads", [False, True])
+def test_teacher_from_prenorm_hidden(heads):
+    """Pre-norm teacher hidden states: the target's final RMS norm is applied in the
+    gather before the teacher GEMM."""
+    kw = dict(markov=False, conf=None) if not heads else dict(rank=64, target_vocab=900, markov_std=0.3, hidden=128)
+    inp = make_inputs("lm_head_teacher", device="cuda", seed=51 + heads, B=2, N=4, K=7, V=8192,
+                      target_hidden_size=256, target_prenorm=True, **kw)
+    assert inp.target_norm_weight is not None
+    _run(inp)
+
+
+def test_prenorm_teacher_config_every_row():
+    """The C4 shape with pre-norm 4096-wide hidden states."""
+    inp = make_inputs("lm_head_teacher", device="cuda", seed=53, target_prenorm=True)
+    _run(inp)
