@@ -35,6 +35,9 @@ the design notes of the repository):
   * report pairs: loss/ce/l1/conf = [sum w*term, num_tokens];
     accept = [sum m*a, num_tokens]; tau = [sum keep*tau_blk, sum keep].
   * without target logits: L1 = 0 (so accept = 1), CE only.
+  * vocabulary-parallel ranks ([RL-HEADS] Tensor Parallelism) combine per-shard
+    partials: logsumexp partials (m, s) merged in rank order, then (L1, S) partials
+    summed in rank order.
   * pre-norm target hidden states (the vLLM case of the [TS-PR] review) get the
     target's final RMS norm, y = w * x / sqrt(mean(x^2) + eps), before lm_head; the
     normed state is rounded to bf16 once, as the norm's output in the model's dtype.
@@ -114,6 +117,56 @@ def row_terms(z: np.ndarray, t: Optional[np.ndarray], tid: int) -> dict:
     q = np.exp(t - lse_t)
     s = np.sign(p - q)
     out.update(lse_t=lse_t, q=q, s=s, l1=float(np.sum(np.abs(p - q))), S=float(np.sum(p * s)))
+    return out
+
+
+# ---------------------------------------------------- vocabulary-parallel form
+# [RL-HEADS] Tensor Parallelism: each tensor-parallel rank holds the base logits of
+# its own contiguous shard of the draft vocabulary.  A full-vocabulary row term then
+# needs the shards' partial sums.  The reading taken here: a rank reduces its
+# columns to a logsumexp partial (m, s); the ranks' partials are merged in rank
+# order; then each rank reduces its columns to an (L1, S) partial against the merged
+# normalisers, and those are summed in rank order.
+def lse_partial(x_shard: np.ndarray) -> tuple:
+    """(m, s) of one shard: m = max_j x_j, s = sum_j exp(x_j - m); (-inf, 0) if empty."""
+    x = np.asarray(x_shard, dtype=np.float64)
+    if x.size == 0:
+        return (-math.inf, 0.0)
+    m = float(np.max(x))
+    return (m, float(np.sum(np.exp(x - m))))
+
+
+def merge_lse_partials(parts) -> float:
+    """log sum_j exp(x_j) of the whole row from its shards' (m, s) partials:
+    M = max_k m_k, lse = M + log sum_k s_k exp(m_k - M) (empty shards add nothing)."""
+    M = max(m for m, _ in parts)
+    total = sum(s * math.exp(m - M) for m, s in parts if m != -math.inf)
+    return M + math.log(total)
+
+
+def l1_partial(z_shard: np.ndarray, t_shard: np.ndarray, lse_d: float, lse_t: float) -> tuple:
+    """(sum_j |p_j - q_j|, sum_j p_j sign(p_j - q_j)) over one shard's columns, with
+    p = exp(z - lse_d) and q = exp(t - lse_t) normalised over the whole row."""
+    p = np.exp(np.asarray(z_shard, dtype=np.float64) - lse_d)
+    q = np.exp(np.asarray(t_shard, dtype=np.float64) - lse_t)
+    return (float(np.sum(np.abs(p - q))), float(np.sum(p * np.sign(p - q))))
+
+
+def tp_row_terms(z: np.ndarray, t: Optional[np.ndarray], tid: int, bounds) -> dict:
+    """CE, L1 and S of one row computed shard by shard: ``bounds`` = [v_0 = 0, v_1, ...,
+    v_T = V] splits the columns into T contiguous shards (empty ones allowed).  Same
+    quantities as ``row_terms``, reached through the partials above."""
+    z = np.asarray(z, dtype=np.float64)
+    shards = [(bounds[k], bounds[k + 1]) for k in range(len(bounds) - 1)]
+    lse_d = merge_lse_partials([lse_partial(z[a:b]) for a, b in shards])
+    out = dict(lse_d=lse_d, ce=lse_d - float(z[tid]))
+    if t is None:
+        out.update(lse_t=0.0, l1=0.0, S=0.0)
+        return out
+    t = np.asarray(t, dtype=np.float64)
+    lse_t = merge_lse_partials([lse_partial(t[a:b]) for a, b in shards])
+    parts = [l1_partial(z[a:b], t[a:b], lse_d, lse_t) for a, b in shards]
+    out.update(lse_t=lse_t, l1=float(sum(l for l, _ in parts)), S=float(sum(s for _, s in parts)))
     return out
 
 

@@ -432,6 +432,69 @@ def test_teacher_from_prenorm_hidden_equals_normed_teacher():
         np.testing.assert_array_equal(a["dlogits"][r], b["dlogits"][r])
 
 
+# ------------------------------------------------------ vocabulary-parallel form
+def _random_bounds(rng, V, T):
+    """T contiguous shards of [0, V), some of them empty."""
+    cuts = np.sort(rng.integers(0, V + 1, size=T - 1))
+    return [0, *cuts.tolist(), V]
+
+
+def test_lse_partials_merge_to_library_logsumexp():
+    """Shard partials merged in order give scipy's logsumexp of the whole row, for
+    rows far from 0, with large spreads, and with empty shards (the merge's identity)."""
+    rng = np.random.default_rng(41)
+    for V, T, loc, scale in [(1, 1, 0.0, 1.0), (17, 3, -1e4, 3.0), (1000, 8, 80.0, 10.0),
+                             (4096, 5, 0.0, 40.0), (333, 16, -50.0, 0.5)]:
+        x = loc + scale * rng.standard_normal(V)
+        bounds = _random_bounds(rng, V, T)
+        parts = [O.lse_partial(x[a:b]) for a, b in zip(bounds[:-1], bounds[1:])]
+        want = float(scipy.special.logsumexp(x))
+        assert abs(O.merge_lse_partials(parts) - want) <= 1e-12 * max(1.0, abs(want))
+        assert O.merge_lse_partials(parts + [(-math.inf, 0.0)]) == O.merge_lse_partials(parts)
+    assert O.lse_partial(np.zeros(0)) == (-math.inf, 0.0)
+    # two equal halves: log(2) above each half's logsumexp
+    h = rng.standard_normal(64)
+    one = O.lse_partial(h)
+    assert abs(O.merge_lse_partials([one, one]) - (scipy.special.logsumexp(h) + math.log(2.0))) <= 1e-12
+
+
+def test_tp_row_terms_closed_forms():
+    """Disjoint saturated rows in different shards: L1 = 2, S = 1.  Identical rows:
+    L1 = 0, S = 0.  A flat draft row against a saturated teacher: L1 = 2 (1 - 1/V)."""
+    V = 96
+    z = np.full(V, -60.0); z[5] = 60.0
+    t = np.full(V, -60.0); t[70] = 60.0
+    for bounds in ([0, 32, 64, 96], [0, 6, 6, 96], [0, 96]):
+        r = O.tp_row_terms(z, t, 5, bounds)
+        assert abs(r["l1"] - 2.0) <= 1e-12 and abs(r["S"] - 1.0) <= 1e-12
+        assert abs(r["ce"]) <= 1e-12
+        r = O.tp_row_terms(z, z.copy(), 70, bounds)
+        assert r["l1"] == 0.0 and r["S"] == 0.0 and abs(r["ce"] - 120.0) <= 1e-9
+        r = O.tp_row_terms(np.zeros(V), t, 0, bounds)
+        assert abs(r["l1"] - 2.0 * (1.0 - 1.0 / V)) <= 1e-12
+        assert abs(r["ce"] - math.log(V)) <= 1e-12
+
+
+def test_tp_row_terms_match_brute_force_for_any_split():
+    """Every split of a row (1 to 9 shards, empty ones included) gives the brute-force
+    softmax sums of the whole row, written out here without any shift."""
+    rng = np.random.default_rng(43)
+    for trial in range(20):
+        V = int(rng.integers(1, 300))
+        z = 2.0 * rng.standard_normal(V)
+        t = 0.8 * z + 1.5 * rng.standard_normal(V)
+        tid = int(rng.integers(0, V))
+        ez, et = np.exp(z), np.exp(t)
+        p, q = ez / ez.sum(), et / et.sum()
+        l1 = sum(abs(p[j] - q[j]) for j in range(V))
+        S = sum(p[j] * np.sign(p[j] - q[j]) for j in range(V))
+        ce = -math.log(p[tid])
+        for T in (1, 2, 3, 9):
+            r = O.tp_row_terms(z, t, tid, _random_bounds(rng, V, T))
+            assert abs(r["l1"] - l1) <= 1e-12 and abs(r["S"] - S) <= 1e-12
+            assert abs(r["ce"] - ce) <= 1e-11
+
+
 # --------------------------------------------------------------- planted mistakes
 def _mutant_half_l1(z, t, tid, _orig=O.row_terms):
     out = _orig(z, t, tid)
@@ -473,6 +536,19 @@ def _mutant_norm_no_square(hidden_rows, weight, eps, _orig=O.target_final_norm):
     return _orig(np.abs(x) ** 0.5 * np.sign(x), weight, eps)
 
 
+def _mutant_merge_no_rescale(parts, _orig=O.merge_lse_partials):
+    M = max(m for m, _ in parts)
+    return M + math.log(sum(s for m, s in parts if m != -math.inf))
+
+
+def _mutant_l1_shard_normalised(z_shard, t_shard, lse_d, lse_t, _orig=O.l1_partial):
+    z = np.asarray(z_shard, dtype=np.float64)
+    t = np.asarray(t_shard, dtype=np.float64)
+    if z.size == 0:
+        return (0.0, 0.0)
+    return _orig(z, t, float(scipy.special.logsumexp(z)), float(scipy.special.logsumexp(t)))
+
+
 @pytest.mark.parametrize("target,mutant,pins", [
     ("row_terms", _mutant_half_l1, [test_disjoint_saturated_rows_match_the_pages_values]),
     ("row_terms", _mutant_no_S, [lambda: test_finite_differences_all_gradients(False, "given")]),
@@ -481,6 +557,8 @@ def _mutant_norm_no_square(hidden_rows, weight, eps, _orig=O.target_final_norm):
     ("target_final_norm", _mutant_norm_no_square, [test_target_final_norm_closed_forms]),
     ("markov_corrected_rows", _mutant_w2_transposed,
      [test_markov_bias_matches_explicit_loops_and_zero_w2_reduces]),
+    ("merge_lse_partials", _mutant_merge_no_rescale, [test_lse_partials_merge_to_library_logsumexp]),
+    ("l1_partial", _mutant_l1_shard_normalised, [test_tp_row_terms_match_brute_force_for_any_split]),
 ])
 def test_planted_mistakes(monkeypatch, target, mutant, pins):
     """Each planted slip in the oracle makes at least one pin fail."""
