@@ -13,6 +13,10 @@ write) before every timed call and the flush is not timed.  `e2e` is the same me
 through the same call with the inputs in pinned host memory: every step copies the
 micro-batch to the device, runs the call and reads the loss and report back.
 `--impl reference` times the FP64 CPU oracle instead, on a bounded sample of rows.
+`--tp T` (one GPU) times instead one rank of a T-way vocabulary-parallel group: the three
+calls dspark_tp_partials, dspark_tp_l1 and dspark_tp_finish on that rank's 1/T shard of
+the micro-batch, the other ranks' records computed beforehand (the two all-gathers
+between the calls are not timed).
 """
 
 from __future__ import annotations
@@ -263,6 +267,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--tp", type=int, default=1, help="time one rank of a vocabulary-parallel group of this size")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
@@ -286,6 +291,10 @@ def main():
 
     seed = 1234 + ["tiny", "recipe", "recipe_heads", "lm_head_teacher", "large"].index(args.workload) + 1000 * rank
     inp = make_inputs(args.workload, device="cuda", seed=seed)
+    if args.tp > 1:
+        if world > 1:
+            raise SystemExit("--tp times one rank on one GPU")
+        return run_tp(args, inp, torch_api)
     call = torch_api.Call(inp, grads=True, rows=False)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     for _ in range(args.warmup):
@@ -381,6 +390,70 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_tp(args, inp, torch_api):
+    """One rank (rank 0) of a vocabulary-parallel group of args.tp ranks: its three calls
+    per step on its shard, L2 flushed before each step, CUDA events around the three."""
+    ranks = torch_api.tp_group_emulated(inp, args.tp, rows=False)
+    torch.cuda.synchronize()
+    for r in ranks:
+        if r.check_status() != 0:
+            raise SystemExit("device status after the emulated group")
+    rec1_all = torch.stack([r.rec1 for r in ranks])
+    rec2_all = torch.stack([r.rec2 for r in ranks])
+    r0 = ranks[0]
+    del ranks[1:]
+    n_sup = int(r0.num_tokens.item())
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def step():
+        r0.partials()
+        r0.l1(rec1_all)
+        r0.finish(rec2_all)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    if r0.check_status() != 0:
+        raise SystemExit("device status after the timed steps")
+    per_step = [s_.elapsed_time(e) for s_, e in zip(starts, ends)]
+    mean_ms = statistics.mean(per_step)
+    es = 2 if inp.dtype == "bf16" else 4
+    width = r0.width
+    # this rank's share of the single-pass bytes: its columns of the supervised rows'
+    # draft and teacher read once, its columns of every row's dlogits written once
+    alg = n_sup * width * es * 2 + inp.R * width * es
+    peak, peak_kind = hbm_peak()
+    achieved = alg / (mean_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(n_sup / (mean_ms / 1e3), 1), "unit": "rows/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_ms, 5),
+        "higher_is_better": True, "scaling": None, "vs_baseline": None,
+        "dtype": "bf16" if inp.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, inp), "parallelism": f"tp{args.tp} (one rank timed)",
+                   "shard_columns": width, "supervised_rows": n_sup,
+                   "l2": "flushed before every timed step (512 MiB write, untimed)",
+                   "not_timed": "the two all-gathers of per-row records between the calls"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                     "algorithmic_bytes": alg,
+                     "timed": "dspark_tp_partials + dspark_tp_l1 + dspark_tp_finish of one rank "
+                              "(mask prologue, three passes over the shard, report), mean CUDA-event time"},
+        "cpu_baseline": None, "e2e": None,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_e2e(inp, steps: int, torch_api):

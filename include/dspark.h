@@ -236,6 +236,71 @@ DSPARK_API dspark_status_t dspark_loss_fwd_noalloc(const dspark_problem_t* prob,
                                                    const dspark_grads_t* grads,
                                                    dspark_stream_t stream);
 
+/*
+ * Vocabulary-parallel (tensor-parallel) loss.  NeMo RL design doc "DSpark Auxiliary
+ * Heads", Tensor Parallelism: each tensor-parallel rank receives the base logits of
+ * its own shard of the draft vocabulary.  The row terms are full-vocabulary sums, so
+ * each rank reduces its columns to per-row partials, the ranks exchange them, and
+ * every rank merges all ranks' partials in rank order: every rank then holds bitwise
+ * the same row statistics and writes the same forward outputs.  One micro-batch is
+ * three calls per rank, with an all-gather over the tensor-parallel group (done by
+ * the caller, e.g. NCCL all_gather) after each of the first two:
+ *
+ *   dspark_tp_partials(prob, params, tp, rec1, ws, ...)        rec1:     [R][8] floats
+ *   all-gather rec1 in rank order                               rec1_all: [tp_size][R][8]
+ *   dspark_tp_l1(prob, params, tp, rec1_all, rec2, ws, ...)     rec2:     [R][4] floats
+ *   all-gather rec2 in rank order                               rec2_all: [tp_size][R][4]
+ *   dspark_tp_finish(prob, params, tp, rec2_all, out, grads, ws, ...)
+ *
+ * `prob` describes this rank's shard: V is the shard's width; draft_logits,
+ * target_logits and dlogits point at the shard's first column, with the full rows'
+ * strides as their leading dimensions; target_ids are GLOBAL ids in [0, vocab_size).
+ * The ranks' shards must tile [0, vocab_size) without overlap.  Shard widths obey the
+ * 16-byte rule above (multiples of 8 bf16 or 4 fp32 columns).  The Markov head, the
+ * confidence head and the teacher from hidden states are not taken on this path
+ * (DSPARK_ERR_UNSUPPORTED); given confidence logits are.  Sum the forward outputs over
+ * data-parallel ranks only: every tensor-parallel rank holds the same values.  The
+ * three calls of a micro-batch take the same problem, params, tp and workspace
+ * (dspark_workspace_size(prob) bytes), in stream order.
+ *
+ * Record 1 of row r (rec1 + 8r): [m_d, s_d, m_t, s_t, zt, 0, 0, 0] where, over this
+ * shard's columns, m = max_j x_j*log2(e) (-inf for no column) and s = sum_j
+ * 2^(x_j*log2(e) - m) for the draft (d) and the teacher (t; -inf, 0 without one), and
+ * zt is the draft logit at the target id if this shard holds that id, else 0.
+ * Record 2 of row r (rec2 + 4r): [L1 part, S part, 0, 0], this shard's sums of
+ * |p_j - q_j| and p_j*sign(p_j - q_j) (an exact tie counts as +p_j).  Only supervised
+ * rows' records are written; the others are left as they were.  Records are
+ * 16-byte aligned device buffers owned by the caller.
+ */
+typedef struct {
+  int64_t tp_size;      /* ranks sharing the vocabulary, in [1, 1024]                  */
+  int64_t vocab_begin;  /* global id of this shard's first column                      */
+  int64_t vocab_size;   /* the whole vocabulary: vocab_begin + V <= vocab_size <= 2^30 */
+} dspark_tp_t;
+
+enum { DSPARK_TP_REC1_FLOATS = 8, DSPARK_TP_REC2_FLOATS = 4 };
+
+/* Step 1: the mask prologue (ids checked against vocab_size) and this shard's
+ * logsumexp partials and target logit -> rec1. */
+DSPARK_API dspark_status_t dspark_tp_partials(const dspark_problem_t* prob, const dspark_params_t* params,
+                                              const dspark_tp_t* tp, float* rec1, void* ws,
+                                              size_t ws_bytes, dspark_stream_t stream);
+
+/* Step 2: merges rec1_all (every rank's rec1, rank order) into the row logsumexps and
+ * the target logit, saved in `ws`, then this shard's (L1, S) partials -> rec2. */
+DSPARK_API dspark_status_t dspark_tp_l1(const dspark_problem_t* prob, const dspark_params_t* params,
+                                        const dspark_tp_t* tp, const float* rec1_all, float* rec2,
+                                        void* ws, size_t ws_bytes, dspark_stream_t stream);
+
+/* Step 3: sums rec2_all (rank order) into L1 and S, writes the forward outputs (as
+ * dspark_loss_fwd) and, with `grads`, dlogits of this shard's columns for every row
+ * (zeros where unsupervised) and dconf.  The head-gradient fields of `grads` must be
+ * NULL. */
+DSPARK_API dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_params_t* params,
+                                            const dspark_tp_t* tp, const float* rec2_all,
+                                            const dspark_fwd_out_t* out, const dspark_grads_t* grads,
+                                            void* ws, size_t ws_bytes, dspark_stream_t stream);
+
 /* Synchronises `stream` and returns the first device-side error recorded in `ws`
  * by the last call that used it (DSPARK_OK if none). */
 DSPARK_API dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream);

@@ -85,6 +85,14 @@ class dspark_grads_t(ctypes.Structure):
     ]
 
 
+class dspark_tp_t(ctypes.Structure):
+    _fields_ = [("tp_size", c_i64), ("vocab_begin", c_i64), ("vocab_size", c_i64)]
+
+
+# floats per row of the two exchange records of the vocabulary-parallel path
+DSPARK_TP_REC1_FLOATS = 8
+DSPARK_TP_REC2_FLOATS = 4
+
 P = ctypes.POINTER
 lib.dspark_workspace_size.argtypes = [P(dspark_problem_t)]
 lib.dspark_workspace_size.restype = ctypes.c_size_t
@@ -99,6 +107,15 @@ lib.dspark_loss_fwd_noalloc.argtypes = [P(dspark_problem_t), P(dspark_params_t),
 lib.dspark_loss_fwd_noalloc.restype = ctypes.c_int
 lib.dspark_acceptance.argtypes = [c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]
 lib.dspark_acceptance.restype = ctypes.c_int
+lib.dspark_tp_partials.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_tp_t), c_vp, c_vp,
+                                   ctypes.c_size_t, c_vp]
+lib.dspark_tp_partials.restype = ctypes.c_int
+lib.dspark_tp_l1.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_tp_t), c_vp, c_vp, c_vp,
+                             ctypes.c_size_t, c_vp]
+lib.dspark_tp_l1.restype = ctypes.c_int
+lib.dspark_tp_finish.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_tp_t), c_vp,
+                                 P(dspark_fwd_out_t), P(dspark_grads_t), c_vp, ctypes.c_size_t, c_vp]
+lib.dspark_tp_finish.restype = ctypes.c_int
 lib.dspark_check_status.argtypes = [c_vp, c_vp]
 lib.dspark_check_status.restype = ctypes.c_int
 lib.dspark_status_string.argtypes = [ctypes.c_int]
@@ -112,6 +129,9 @@ dspark_loss_fwd_noalloc = lib.dspark_loss_fwd_noalloc
 # Rows (B*N*K) the fixed scratch of dspark_loss_fwd_noalloc serves.
 NOALLOC_MAX_ROWS = 8192
 dspark_acceptance = lib.dspark_acceptance
+dspark_tp_partials = lib.dspark_tp_partials
+dspark_tp_l1 = lib.dspark_tp_l1
+dspark_tp_finish = lib.dspark_tp_finish
 dspark_check_status = lib.dspark_check_status
 dspark_status_string = lib.dspark_status_string
 

@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "internal.cuh"
+#include "tp.cuh"
 
 using namespace dspark;
 
@@ -58,7 +59,9 @@ inline int sweep_kind(const dspark_problem_t* p) {
   return z32 ? (t32 ? kSweepZT32 : kSweepZ32) : (t32 ? kSweepT32 : kSweepBf16);
 }
 
-dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* prm, Shape* sh) {
+// `sweep`: the fused row sweep will run this problem (its builds bound V).
+dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* prm, Shape* sh,
+                              bool sweep = true) {
   if (p == nullptr) return DSPARK_ERR_INVALID_ARG;
   if (p->B <= 0 || p->N <= 0 || p->K <= 0 || p->V <= 0) return DSPARK_ERR_INVALID_ARG;
   if (p->logits_dtype != DSPARK_F32 && p->logits_dtype != DSPARK_BF16) return DSPARK_ERR_INVALID_ARG;
@@ -113,7 +116,7 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
     if (p->conf_with_markov && !s.has_markov) return DSPARK_ERR_INVALID_ARG;
     if (p->hidden_size % 8 || !aligned16(p->conf_w) || !aligned16(p->draft_hidden)) return DSPARK_ERR_ALIGNMENT;
   }
-  if (!sweep_supported(sweep_kind(p), p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
+  if (sweep && !sweep_supported(sweep_kind(p), p->V, s.has_teacher)) return DSPARK_ERR_UNSUPPORTED;
   *sh = s;
   return DSPARK_OK;
 }
@@ -214,6 +217,44 @@ HeadsArgs heads_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
   }
   h.ws = ws;
   return h;
+}
+
+// A vocabulary-parallel shard: the plain problem's rules, no heads, and a shard that
+// lies inside the vocabulary.
+dspark_status_t check_tp(const dspark_problem_t* p, const dspark_params_t* prm, const dspark_tp_t* tp,
+                         Shape* sh) {
+  if (prm == nullptr || tp == nullptr) return DSPARK_ERR_INVALID_ARG;
+  dspark_status_t st = check_problem(p, prm, sh, false);
+  if (st != DSPARK_OK) return st;
+  if (sh->has_markov || sh->has_conf_head || sh->has_lm_head) return DSPARK_ERR_UNSUPPORTED;
+  if (tp->tp_size < 1 || tp->tp_size > 1024) return DSPARK_ERR_INVALID_ARG;
+  if (tp->vocab_size <= 0 || tp->vocab_size > (int64_t(1) << 30) || tp->vocab_begin < 0 ||
+      tp->vocab_begin > tp->vocab_size - p->V)
+    return DSPARK_ERR_INVALID_ARG;
+  return DSPARK_OK;
+}
+
+dspark_status_t check_rec(const float* r) {
+  if (r == nullptr) return DSPARK_ERR_INVALID_ARG;
+  return aligned16(r) ? DSPARK_OK : DSPARK_ERR_ALIGNMENT;
+}
+
+TpArgs tp_args(const dspark_problem_t* p, const dspark_params_t* prm, const dspark_tp_t* tp,
+               const WsView& ws) {
+  TpArgs a{};
+  a.draft = p->draft_logits;
+  a.ld_d = p->draft_ld;
+  a.target = p->target_logits;
+  a.ld_t = p->target_ld;
+  a.tids = p->target_ids;
+  a.R = p->B * p->N * p->K;
+  a.V = p->V;
+  a.vocab_begin = tp->vocab_begin;
+  a.tp_size = int32_t(tp->tp_size);
+  a.ce_alpha = prm->ce_alpha;
+  a.l1_alpha = p->target_logits ? prm->l1_alpha : 0.f;
+  a.ws = ws;
+  return a;
 }
 
 }  // namespace
@@ -365,6 +406,91 @@ dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, const float* 
   if (!l1_rows || !eval_mask || !accept_pair || !tau_pair) return DSPARK_ERR_INVALID_ARG;
   return cuda_status(launch_acceptance(B, N, K, l1_rows, eval_mask, block_keep, accept_pair,
                                        tau_pair, accept_rows, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status_t dspark_tp_partials(const dspark_problem_t* prob, const dspark_params_t* params,
+                                   const dspark_tp_t* tp, float* rec1, void* ws, size_t ws_bytes,
+                                   dspark_stream_t stream) {
+  Shape sh{};
+  dspark_status_t st = check_tp(prob, params, tp, &sh);
+  if (st != DSPARK_OK) return st;
+  if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
+  if ((st = check_rec(rec1)) != DSPARK_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsView v = ws_layout(ws, ws_dims(prob));
+  PrologueArgs pa{};
+  pa.B = prob->B; pa.N = prob->N; pa.K = prob->K;
+  pa.V = tp->vocab_size;  // target ids are global
+  pa.eval_mask = prob->eval_mask;
+  pa.block_keep = prob->block_keep;
+  pa.target_ids = prob->target_ids;
+  pa.gamma = params->gamma;
+  pa.gamma_enabled = params->gamma_enabled;
+  pa.ws = v;
+  cudaError_t e = launch_prologue(pa, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  TpArgs a = tp_args(prob, params, tp, v);
+  a.rec1 = rec1;
+  return cuda_status(launch_tp_partials(prob->logits_dtype == DSPARK_F32, a, s));
+}
+
+dspark_status_t dspark_tp_l1(const dspark_problem_t* prob, const dspark_params_t* params,
+                             const dspark_tp_t* tp, const float* rec1_all, float* rec2, void* ws,
+                             size_t ws_bytes, dspark_stream_t stream) {
+  Shape sh{};
+  dspark_status_t st = check_tp(prob, params, tp, &sh);
+  if (st != DSPARK_OK) return st;
+  if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
+  if ((st = check_rec(rec1_all)) != DSPARK_OK || (st = check_rec(rec2)) != DSPARK_OK) return st;
+  const WsView v = ws_layout(ws, ws_dims(prob));
+  TpArgs a = tp_args(prob, params, tp, v);
+  a.rec1_all = rec1_all;
+  a.rec2 = rec2;
+  return cuda_status(launch_tp_l1(prob->logits_dtype == DSPARK_F32, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_params_t* params,
+                                 const dspark_tp_t* tp, const float* rec2_all,
+                                 const dspark_fwd_out_t* out, const dspark_grads_t* grads, void* ws,
+                                 size_t ws_bytes, dspark_stream_t stream) {
+  if (out == nullptr) return DSPARK_ERR_INVALID_ARG;
+  Shape sh{};
+  dspark_status_t st = check_tp(prob, params, tp, &sh);
+  if (st != DSPARK_OK) return st;
+  if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
+  if ((st = check_rec(rec2_all)) != DSPARK_OK) return st;
+  if (grads) {
+    if ((st = check_grads(prob, grads)) != DSPARK_OK) return st;
+    if (grads->dW1 || grads->dW2 || grads->dconf_w || grads->dconf_b || grads->dhidden)
+      return DSPARK_ERR_INVALID_ARG;
+  }
+  const WsView v = ws_layout(ws, ws_dims(prob));
+  TpArgs a = tp_args(prob, params, tp, v);
+  a.rec2_all = rec2_all;
+  if (grads) {
+    a.dlogits = grads->dlogits;
+    a.ld_g = grads->dlogits_ld;
+    a.grad_scale = grads->grad_scale;
+  }
+  FinalizeArgs f{};
+  f.B = prob->B; f.N = prob->N; f.K = prob->K;
+  f.block_keep = prob->block_keep;
+  f.confidence_logits = prob->confidence_logits;
+  f.has_conf = sh.has_conf_given;
+  f.ce_alpha = params->ce_alpha;
+  f.l1_alpha = params->l1_alpha;
+  f.conf_alpha = params->conf_alpha;
+  f.grad_scale = grads ? grads->grad_scale : nullptr;
+  f.ws = v;
+  f.loss_num = out->loss_num;
+  f.num_tokens = out->num_tokens;
+  f.report = out->report;
+  f.ce_rows = out->ce_rows;
+  f.l1_rows = out->l1_rows;
+  f.accept_rows = out->accept_rows;
+  f.conf_rows = out->conf_rows;
+  f.dconf = grads ? grads->dconf : nullptr;
+  return cuda_status(launch_tp_finish(prob->logits_dtype == DSPARK_F32, a, f, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream) {

@@ -743,7 +743,8 @@ cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStre
 }
 
 // ------------------------------------------------------- backward-only stream
-// dlogits from saved row statistics: one more read of the logits, no reductions.
+// dlogits from saved row statistics: one more read of the logits, no reductions.  An
+// exact tie p_j == q_j takes sign +1, the sub-gradient the forward's S counted.
 // Covers the supervised rows of list positions [row0, row1) and, with do_zero, the
 // unsupervised rows.
 template <typename TZ, typename TT, typename TO, bool HAS_T, bool HAS_B>
@@ -772,7 +773,7 @@ __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a) {
     const float gw = g * a.ws.w[row];
     const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
     const float S = st[kStS];
-    const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S), kzero = cce - cl1 * S;
+    const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S);
     const float lz2 = st[kStLseD] * kLog2e, lt2 = st[kStLseT] * kLog2e;
     const int64_t tok = a.tids[row];
     const int64_t trow = (kTChunk && a.target_compact) ? int64_t(idx) : row;
@@ -794,7 +795,7 @@ __global__ void __launch_bounds__(256) bwd_stream_kernel(const SweepArgs a) {
         const float p = ex2(fmaf(z[e], kLog2e, -lz2));
         if constexpr (HAS_T) {
           const float d = p - ex2(fmaf(t[e], kLog2e, -lt2));
-          o[e] = p * (d > 0.f ? kpos : (d < 0.f ? kneg : kzero));
+          o[e] = p * (d >= 0.f ? kpos : kneg);
         } else {
           o[e] = p * cce;
         }

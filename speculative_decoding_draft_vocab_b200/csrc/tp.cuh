@@ -1,0 +1,37 @@
+// Vocabulary-parallel steps: kernel arguments and launchers (csrc/tp.cu).
+#pragma once
+#include "internal.cuh"
+
+namespace dspark {
+
+// One rank's shard of a micro-batch and the exchange records of the three steps.
+struct TpArgs {
+  const void* draft;         // shard columns of the base draft rows
+  int64_t ld_d;
+  const void* target;        // shard columns of the teacher rows, or null (CE only)
+  int64_t ld_t;
+  void* dlogits;             // shard columns of dL/dz, or null (forward only)
+  int64_t ld_g;
+  const int64_t* tids;       // global target ids
+  const float* grad_scale;   // null: 1
+  int64_t R;
+  int64_t V;                 // shard width
+  int64_t vocab_begin;       // global id of the shard's first column
+  int32_t tp_size;
+  float* rec1;               // [R][8] this shard's logsumexp partials
+  const float* rec1_all;     // [tp_size][R][8] every rank's, rank order
+  float* rec2;               // [R][4] this shard's (L1, S) partials
+  const float* rec2_all;     // [tp_size][R][4]
+  float ce_alpha, l1_alpha;
+  WsView ws;
+};
+
+constexpr int kTpRec1 = 8;
+constexpr int kTpRec2 = 4;
+
+cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s);
+cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s);
+// the rows' L1 and S, dlogits of the shard, then the per-row epilogue and the report
+cudaError_t launch_tp_finish(bool f32, const TpArgs& a, const FinalizeArgs& f, cudaStream_t s);
+
+}  // namespace dspark

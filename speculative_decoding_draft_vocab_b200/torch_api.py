@@ -194,3 +194,136 @@ def acceptance(l1_rows: torch.Tensor, eval_mask: torch.Tensor, block_keep: Optio
                                _ptr(tp), _ptr(ar), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     abi.check(st, "dspark_acceptance")
     return ap, tp, ar
+
+
+# ------------------------------------------------------- vocabulary-parallel path
+def even_shards(V: int, tp_size: int, align: int) -> list:
+    """Bounds [0, v_1, ..., V] of tp_size contiguous vocabulary shards whose widths are
+    multiples of ``align`` columns (8 bf16 / 4 fp32: the 16-byte rule), as even as
+    that allows (the first shards take the remainder)."""
+    if V % align or tp_size < 1:
+        raise ValueError("V must be a multiple of align and tp_size >= 1")
+    base, extra = divmod(V // align, tp_size)
+    bounds = [0]
+    for k in range(tp_size):
+        bounds.append(bounds[-1] + (base + (1 if k < extra else 0)) * align)
+    return bounds
+
+
+class TPRank:
+    """One tensor-parallel rank's three calls (dspark_tp_partials, dspark_tp_l1,
+    dspark_tp_finish) on its vocabulary shard of a micro-batch.
+
+    ``inp`` holds rows that contain this rank's shard at columns [col0, col0 + width):
+    the full rows (single-device emulation of a group) or just the shard (one rank per
+    GPU, col0 = 0).  The shard is addressed in place, with the rows' stride.  dlogits of
+    the shard go to the same columns of ``dlogits`` (rows shaped like ``inp``'s), or of
+    a buffer this rank allocates.  Every rank writes its own copy of the forward outputs.
+    """
+
+    def __init__(self, inp: DSparkInputs, tp_size: int, vocab_begin: int, vocab_size: int,
+                 col0: int = 0, width: Optional[int] = None, dlogits: Optional[torch.Tensor] = None,
+                 grads: bool = True, rows: bool = True):
+        dev = inp.draft_logits.device
+        R = inp.R
+        es = 4 if inp.dtype == "f32" else 2
+        width = inp.V - col0 if width is None else width
+        self.inp, self.col0, self.width = inp, col0, width
+        p = problem_struct(inp)
+        p.V = width
+        p.draft_logits = ctypes.c_void_p(inp.draft_logits.data_ptr() + col0 * es)
+        if inp.target_logits is not None:
+            p.target_logits = ctypes.c_void_p(inp.target_logits.data_ptr() + col0 * es)
+        self.prob = p
+        self.prm = params_struct(inp)
+        self.tp = abi.dspark_tp_t(tp_size, vocab_begin, vocab_size)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.rec1 = torch.empty(R, abi.DSPARK_TP_REC1_FLOATS, **f32)
+        self.rec2 = torch.empty(R, abi.DSPARK_TP_REC2_FLOATS, **f32)
+        self.loss_num = torch.zeros(1, **f32)
+        self.num_tokens = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.report = torch.zeros(abi.DSPARK_REP_COUNT, 2, **f32)
+        self.ce_rows = torch.zeros(R, **f32) if rows else None
+        self.l1_rows = torch.zeros(R, **f32) if rows else None
+        self.accept_rows = torch.zeros(R, **f32) if rows else None
+        self.conf_rows = torch.zeros(R, **f32) if rows else None
+        self.grad_scale = torch.full((1,), float(inp.grad_scale), **f32)
+        self.dconf = torch.zeros(R, **f32) if grads else None
+        if grads and dlogits is None:
+            dlogits = torch.zeros_like(inp.draft_logits)
+        self.dlogits = dlogits if grads else None
+        o = abi.dspark_fwd_out_t()
+        o.loss_num, o.num_tokens, o.report = _ptr(self.loss_num), _ptr(self.num_tokens), _ptr(self.report)
+        o.ce_rows, o.l1_rows = _ptr(self.ce_rows), _ptr(self.l1_rows)
+        o.accept_rows, o.conf_rows = _ptr(self.accept_rows), _ptr(self.conf_rows)
+        self.fwd = o
+        self.grads = None
+        if grads:
+            g = abi.dspark_grads_t()
+            g.grad_scale = _ptr(self.grad_scale)
+            g.dlogits = ctypes.c_void_p(self.dlogits.data_ptr() + col0 * es)
+            g.dlogits_ld = inp.V
+            g.dconf = _ptr(self.dconf)
+            self.grads = g
+        self.ws = new_workspace(inp)
+        self.ws_ptr, self.ws_len = _aligned_ws(self.ws)
+
+    @staticmethod
+    def _stream(stream):
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream if stream is None else stream)
+
+    def partials(self, stream=None) -> torch.Tensor:
+        st = abi.dspark_tp_partials(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.tp),
+                                    _ptr(self.rec1), self.ws_ptr, self.ws_len, self._stream(stream))
+        abi.check(st, "dspark_tp_partials")
+        return self.rec1
+
+    def l1(self, rec1_all: torch.Tensor, stream=None) -> torch.Tensor:
+        _need(rec1_all, torch.float32, "rec1_all")
+        st = abi.dspark_tp_l1(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.tp),
+                              _ptr(rec1_all), _ptr(self.rec2), self.ws_ptr, self.ws_len, self._stream(stream))
+        abi.check(st, "dspark_tp_l1")
+        return self.rec2
+
+    def finish(self, rec2_all: torch.Tensor, stream=None) -> None:
+        _need(rec2_all, torch.float32, "rec2_all")
+        st = abi.dspark_tp_finish(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.tp),
+                                  _ptr(rec2_all), ctypes.byref(self.fwd),
+                                  ctypes.byref(self.grads) if self.grads is not None else None,
+                                  self.ws_ptr, self.ws_len, self._stream(stream))
+        abi.check(st, "dspark_tp_finish")
+
+    def run(self, exchange) -> None:
+        """The three calls, with ``exchange`` (this rank's records -> every rank's records
+        stacked in rank order, e.g. ``tp_exchange``) after each of the first two."""
+        rec1_all = exchange(self.partials())
+        self.finish(exchange(self.l1(rec1_all)))
+
+    def check_status(self, stream=None) -> int:
+        return int(abi.dspark_check_status(self.ws_ptr, self._stream(stream)))
+
+
+def tp_exchange(local: torch.Tensor, group=None) -> torch.Tensor:
+    """Every rank's records in rank order, [world, *local.shape]: an all-gather over the
+    tensor-parallel process group (NCCL for CUDA tensors)."""
+    import torch.distributed as dist
+    parts = [torch.empty_like(local) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, local.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def tp_group_emulated(inp: DSparkInputs, tp_size: int, grads: bool = True, rows: bool = True) -> list:
+    """A whole tensor-parallel group on this device: tp_size ranks over even shards of
+    ``inp``'s full rows, stepped together, the exchange being a stack of the ranks'
+    records (what the all-gather delivers).  The ranks share one dlogits buffer, each
+    writing its own columns.  Returns the ranks (launched, not synchronised)."""
+    align = 4 if inp.dtype == "f32" else 8
+    bounds = even_shards(inp.V, tp_size, align)
+    dl = torch.zeros_like(inp.draft_logits) if grads else None
+    ranks = [TPRank(inp, tp_size, bounds[k], inp.V, col0=bounds[k], width=bounds[k + 1] - bounds[k],
+                    dlogits=dl, grads=grads, rows=rows) for k in range(tp_size)]
+    rec1_all = torch.stack([r.partials() for r in ranks])
+    rec2_all = torch.stack([r.l1(rec1_all) for r in ranks])
+    for r in ranks:
+        r.finish(rec2_all)
+    return ranks

@@ -50,7 +50,8 @@ BODY
 
 def test_struct_layout_matches_ctypes(abi):
     lines = []
-    for cls in (abi.dspark_problem_t, abi.dspark_params_t, abi.dspark_fwd_out_t, abi.dspark_grads_t):
+    for cls in (abi.dspark_problem_t, abi.dspark_params_t, abi.dspark_fwd_out_t, abi.dspark_grads_t,
+                abi.dspark_tp_t):
         t = cls.__name__
         lines.append(f"  S({t})")
         for f, _ in cls._fields_:
@@ -66,7 +67,8 @@ def test_struct_layout_matches_ctypes(abi):
     for line in out.splitlines():
         t, f, v = line.split()
         got[(t, f)] = int(v)
-    for cls in (abi.dspark_problem_t, abi.dspark_params_t, abi.dspark_fwd_out_t, abi.dspark_grads_t):
+    for cls in (abi.dspark_problem_t, abi.dspark_params_t, abi.dspark_fwd_out_t, abi.dspark_grads_t,
+                abi.dspark_tp_t):
         t = cls.__name__
         assert got[(t, "sizeof")] == ctypes.sizeof(cls), t
         for f, _ in cls._fields_:
@@ -261,3 +263,70 @@ def test_target_norm_validation(abi):
     p.target_norm_weight = ctypes.c_void_p(0x110000)
     p.target_norm_eps = -1.0
     assert _fwd(abi, p, prm) == abi.DSPARK_ERR_INVALID_ARG
+
+
+def _tp_calls(abi, p, prm, tp, rec=0x200000, ws=0x100000, ws_bytes=1 << 30, grads=None):
+    """Status of each of the three vocabulary-parallel calls on the same arguments."""
+    r = ctypes.c_void_p(rec)
+    out = abi.dspark_fwd_out_t()
+    return (abi.dspark_tp_partials(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r,
+                                   ctypes.c_void_p(ws), ws_bytes, None),
+            abi.dspark_tp_l1(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r, r,
+                             ctypes.c_void_p(ws), ws_bytes, None),
+            abi.dspark_tp_finish(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r, ctypes.byref(out),
+                                 ctypes.byref(grads) if grads is not None else None,
+                                 ctypes.c_void_p(ws), ws_bytes, None))
+
+
+def test_vocab_parallel_validation(abi):
+    """Shard bounds, record buffers, the heads (not taken on this path) and head
+    gradients are checked on the host, by all three calls alike."""
+    prm = _params(abi)
+    p = _problem(abi, V=1024)
+    every = lambda st: (st,) * 3
+    # the shard must lie inside the vocabulary
+    assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2, 1024, 1024 + 1000)) == every(abi.DSPARK_ERR_INVALID_ARG)
+    assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2, -8, 4096)) == every(abi.DSPARK_ERR_INVALID_ARG)
+    assert _tp_calls(abi, p, prm, abi.dspark_tp_t(0, 0, 4096)) == every(abi.DSPARK_ERR_INVALID_ARG)
+    assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2000, 0, 4096)) == every(abi.DSPARK_ERR_INVALID_ARG)
+    assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2, 0, (1 << 30) + 8)) == every(abi.DSPARK_ERR_INVALID_ARG)
+    # records: present and 16-byte aligned
+    tp = abi.dspark_tp_t(4, 1024, 4096)
+    assert _tp_calls(abi, p, prm, tp, rec=0) == every(abi.DSPARK_ERR_INVALID_ARG)
+    assert _tp_calls(abi, p, prm, tp, rec=0x200008) == every(abi.DSPARK_ERR_ALIGNMENT)
+    # the plain problem's rules still hold (shard width under the 16-byte rule, workspace)
+    assert _tp_calls(abi, _problem(abi, V=1020), prm, tp) == every(abi.DSPARK_ERR_ALIGNMENT)
+    assert _tp_calls(abi, p, prm, tp, ws_bytes=16) == every(abi.DSPARK_ERR_WORKSPACE)
+    assert _tp_calls(abi, _problem(abi, target=False), prm, tp) == every(abi.DSPARK_ERR_MISSING_TARGET)
+    # heads are not taken on the vocabulary-parallel path
+    assert _tp_calls(abi, _with_markov(abi, _problem(abi)), prm, tp) == every(abi.DSPARK_ERR_UNSUPPORTED)
+    assert _tp_calls(abi, _with_conf_head(abi, _problem(abi)), prm, tp) == every(abi.DSPARK_ERR_UNSUPPORTED)
+    assert _tp_calls(abi, _with_lm_head(abi, _problem(abi, target=False)), prm, tp) == \
+        every(abi.DSPARK_ERR_UNSUPPORTED)
+    # head-gradient fields must stay NULL; a misaligned dlogits stride is refused
+    g = abi.dspark_grads_t()
+    g.dlogits, g.dlogits_ld = ctypes.c_void_p(0x70000), 4096
+    g.dW2 = ctypes.c_void_p(0x80000)
+    assert _tp_calls(abi, p, prm, tp, grads=g)[2] == abi.DSPARK_ERR_INVALID_ARG
+    g.dW2, g.dlogits_ld = None, 1028
+    assert _tp_calls(abi, p, prm, tp, grads=g)[2] == abi.DSPARK_ERR_ALIGNMENT
+    # NULL params / tp / outputs
+    out = abi.dspark_fwd_out_t()
+    assert abi.dspark_tp_partials(ctypes.byref(p), None, ctypes.byref(tp), ctypes.c_void_p(0x200000),
+                                  ctypes.c_void_p(0x100000), 1 << 30, None) == abi.DSPARK_ERR_INVALID_ARG
+    assert abi.dspark_tp_l1(ctypes.byref(p), ctypes.byref(prm), None, ctypes.c_void_p(0x200000),
+                            ctypes.c_void_p(0x200000), ctypes.c_void_p(0x100000), 1 << 30,
+                            None) == abi.DSPARK_ERR_INVALID_ARG
+    assert abi.dspark_tp_finish(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), ctypes.c_void_p(0x200000),
+                                None, None, ctypes.c_void_p(0x100000), 1 << 30, None) == abi.DSPARK_ERR_INVALID_ARG
+    del out
+
+
+def test_even_shards():
+    from speculative_decoding_draft_vocab_b200.torch_api import even_shards
+    assert even_shards(151936, 8, 8) == [0, 18992, 37984, 56976, 75968, 94960, 113952, 132944, 151936]
+    b = even_shards(50008, 3, 8)
+    assert b[0] == 0 and b[-1] == 50008 and all((y - x) % 8 == 0 and y > x for x, y in zip(b, b[1:]))
+    assert max(y - x for x, y in zip(b, b[1:])) - min(y - x for x, y in zip(b, b[1:])) <= 8
+    with pytest.raises(ValueError):
+        even_shards(1001, 2, 8)

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from speculative_decoding_draft_vocab_b200.synthetic import make_inputs
-from tests.parity_util import compare, oracle_run, run_gpu
+from tests.parity_util import check_dlogit_row, compare, oracle_run, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +72,31 @@ def test_identical_rows_give_zero_l1():
     assert np.allclose(call.out.accept_rows.cpu().numpy(), 1.0, atol=1e-6)
     tau = call.out.report[5].tolist()
     assert tau[1] == 3.0 and abs(tau[0] - 3.0 * 8) <= 1e-4 * 24
+
+
+@pytest.mark.parametrize("separate", [False, True])
+def test_identical_rows_dlogits_every_element(separate):
+    """draft == teacher puts every |p_j - q_j| at its kink.  The forward's S counts each
+    exact tie as +p_j; the fused and the separate backward take that same sign, which
+    makes dL/dz = g w ce_alpha (p - onehot), the oracle's value (its sign(0) = 0 gives
+    S = 0 and the same dz), on every element, none skipped."""
+    from speculative_decoding_draft_vocab_b200 import torch_api
+    inp = make_inputs("recipe", device="cuda", B=1, N=3, K=7, V=16384, prefix=(7, 7), seed=6)
+    inp.target_logits = inp.draft_logits.clone()
+    call = torch_api.Call(inp, grads=True)
+    if separate:
+        call.out.dlogits.fill_(5.0)
+        torch_api.Call(inp, out=call.out, grads=False).launch()
+        call.backward()
+    else:
+        call.launch()
+    torch.cuda.synchronize()
+    assert call.check_status() == 0
+    ref = oracle_run(inp)
+    g = call.out.dlogits.view(inp.R, inp.V)
+    for r in ref["rows"]:
+        check_dlogit_row(g[r].float().cpu().double().numpy(), ref["dlogits"][r],
+                         np.zeros(inp.V, dtype=bool), inp.dtype, tag=f"row {r}")
 
 
 def test_disjoint_rows_l1_two():

@@ -1,0 +1,147 @@
+"""GPU parity of the vocabulary-parallel path (dspark_tp_partials, dspark_tp_l1,
+dspark_tp_finish) against the FP64 oracle of the whole rows.
+
+A tensor-parallel group is emulated on one device: its ranks run one after another over
+even shards of the full rows, and the exchange is a stack of their records (what the
+all-gather would deliver).  No kernel waits on another.  Every rank must report the
+same forward outputs, bit for bit; dlogits are assembled from the ranks' columns.
+NeMo RL design doc "DSpark Auxiliary Heads", Tensor Parallelism.
+"""
+
+import math
+from types import SimpleNamespace
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dspark_oracle as O
+from speculative_decoding_draft_vocab_b200.synthetic import make_inputs
+from tests.parity_util import check_dlogit_row, compare, np32, oracle_run
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from speculative_decoding_draft_vocab_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+
+
+def _group(inp, tp_size, grads=True):
+    from speculative_decoding_draft_vocab_b200 import torch_api
+    ranks = torch_api.tp_group_emulated(inp, tp_size, grads=grads)
+    torch.cuda.synchronize()
+    for r in ranks:
+        assert r.check_status() == 0
+    return ranks
+
+
+def _as_call(rank):
+    """The fields of one rank that the parity helpers read."""
+    return SimpleNamespace(out=SimpleNamespace(
+        num_tokens=rank.num_tokens, report=rank.report, loss_num=rank.loss_num, ce_rows=rank.ce_rows,
+        l1_rows=rank.l1_rows, accept_rows=rank.accept_rows, dconf=rank.dconf, dlogits=rank.dlogits))
+
+
+def _check_group(inp, ranks, ref, **kw):
+    compare(inp, _as_call(ranks[0]), ref, **kw)
+    for r in ranks[1:]:  # every rank holds the same forward outputs
+        for name in ("loss_num", "num_tokens", "report", "ce_rows", "l1_rows", "accept_rows", "dconf"):
+            assert torch.equal(getattr(r, name), getattr(ranks[0], name)), name
+
+
+@pytest.mark.parametrize("dtype,V,T", [("bf16", 4096, 1), ("bf16", 4096, 2), ("bf16", 50008, 3),
+                                       ("bf16", 151936, 8), ("f32", 5000, 3), ("f32", 30000, 4)])
+def test_tp_group_matches_oracle(dtype, V, T):
+    """Even shards (uneven where V does not divide), ragged prefix masks with stray ones."""
+    inp = make_inputs("recipe", device="cuda", B=2, N=5, K=7, V=V, dtype=dtype, mask_holes=True, seed=40 + V + T)
+    ranks = _group(inp, T)
+    _check_group(inp, ranks, oracle_run(inp))
+
+
+def test_tp_given_confidence_gamma_none_grad_scale():
+    inp = make_inputs("recipe", device="cuda", B=2, N=4, K=7, V=8192, conf="given", gamma=None,
+                      grad_scale=0.37, seed=41)
+    _check_group(inp, _group(inp, 4), oracle_run(inp))
+
+
+def test_tp_ce_only_without_teacher():
+    inp = make_inputs("recipe", device="cuda", B=2, N=4, K=7, V=8192, no_target=True, seed=42)
+    _check_group(inp, _group(inp, 2), oracle_run(inp))
+
+
+def test_tp_forward_only_and_all_masked():
+    inp = make_inputs("recipe", device="cuda", B=2, N=3, K=7, V=4096, seed=43)
+    ranks = _group(inp, 2, grads=False)
+    compare(inp, _as_call(ranks[0]), oracle_run(inp, want_grads=False))
+    inp = make_inputs("recipe", device="cuda", B=2, N=3, K=7, V=4096, prefix=(0, 0), seed=44)
+    ranks = _group(inp, 4)
+    assert int(ranks[0].num_tokens.item()) == 0 and float(ranks[0].loss_num.item()) == 0.0
+    assert bool((ranks[0].dlogits == 0).all())
+
+
+def test_tp_records_follow_the_header():
+    """Record 1 holds the shard's base-2 maximum and sum of 2^(x log2 e - m) for draft and
+    teacher, and the target logit only on the shard that holds the id."""
+    from speculative_decoding_draft_vocab_b200 import torch_api
+    inp = make_inputs("recipe", device="cuda", B=1, N=2, K=7, V=8192, prefix=(7, 7), seed=45)
+    ranks = _group(inp, 4)
+    bounds = torch_api.even_shards(inp.V, 4, 8)
+    z = np32(inp.draft_logits).reshape(inp.R, inp.V).astype(np.float64)
+    t = np32(inp.target_logits).reshape(inp.R, inp.V).astype(np.float64)
+    ids = np32(inp.target_ids).reshape(-1)
+    log2e = 1.0 / math.log(2.0)
+    for k, rk in enumerate(ranks):
+        lo, hi = bounds[k], bounds[k + 1]
+        rec = rk.rec1.double().cpu().numpy()
+        for r in range(inp.R):
+            md, sd = O.lse_partial(z[r, lo:hi])
+            mt, st = O.lse_partial(t[r, lo:hi])
+            assert abs(rec[r, 0] - md * log2e) <= 1e-6 * abs(md * log2e) + 1e-6
+            assert abs(rec[r, 1] - sd) <= 1e-5 * sd
+            assert abs(rec[r, 2] - mt * log2e) <= 1e-6 * abs(mt * log2e) + 1e-6
+            assert abs(rec[r, 3] - st) <= 1e-5 * st
+            assert rec[r, 4] == (z[r, ids[r]] if lo <= ids[r] < hi else 0.0)
+
+
+def test_tp_out_of_range_id_is_flagged_and_skipped():
+    inp = make_inputs("recipe", device="cuda", B=1, N=2, K=7, V=4096, prefix=(7, 7), seed=46)
+    inp.target_ids[0, 1, 3] = 4096 + 5
+    from speculative_decoding_draft_vocab_b200 import abi, torch_api
+    ranks = torch_api.tp_group_emulated(inp, 2)
+    assert ranks[0].check_status() == abi.DSPARK_ERR_ID_OUT_OF_RANGE
+    assert int(ranks[1].num_tokens.item()) == 13
+    assert bool((ranks[0].dlogits[0, 1, 3] == 0).all())
+
+
+def test_tp_identical_rows():
+    """draft == teacher: every |p_j - q_j| is at its kink; the ranks' S counts each tie
+    as +p_j and dL/dz takes the same sign, which makes dz = g w ce_alpha (p - onehot),
+    the oracle's value, on every element (none skipped)."""
+    inp = make_inputs("recipe", device="cuda", B=1, N=3, K=7, V=16384, prefix=(7, 7), seed=6)
+    inp.target_logits = inp.draft_logits.clone()
+    ranks = _group(inp, 4)
+    ref = oracle_run(inp)
+    assert np.allclose(ranks[0].l1_rows.cpu().numpy(), 0.0, atol=1e-6)
+    g = ranks[0].dlogits.view(inp.R, inp.V)
+    for r in ref["rows"]:
+        check_dlogit_row(g[r].float().cpu().double().numpy(), ref["dlogits"][r],
+                         np.zeros(inp.V, dtype=bool), inp.dtype, tag=f"row {r}")
+
+
+def test_tp_recipe_workload_every_row():
+    """The bench workload (4 x 16 x 7 rows of 151936 bf16 logits) over 8 ranks, every row
+    checked, and the group agrees with the single-device fused call."""
+    from speculative_decoding_draft_vocab_b200 import torch_api
+    inp = make_inputs("recipe", device="cuda")
+    ranks = _group(inp, 8)
+    ref = oracle_run(inp)
+    _check_group(inp, ranks, ref)
+    fused = torch_api.Call(inp)
+    fused.launch()
+    torch.cuda.synchronize()
+    assert torch.equal(fused.out.num_tokens, ranks[0].num_tokens)
+    rel = (fused.out.report - ranks[0].report).abs() / fused.out.report.abs().clamp_min(1e-6)
+    assert float(rel.max()) <= 2e-5
