@@ -472,7 +472,7 @@ dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_para
     a.ld_g = grads->dlogits_ld;
     a.grad_scale = grads->grad_scale;
   }
-  FinalizeArgs f{};
+  FinalizeArgs& f = a.fin;
   f.B = prob->B; f.N = prob->N; f.K = prob->K;
   f.block_keep = prob->block_keep;
   f.confidence_logits = prob->confidence_logits;
@@ -490,7 +490,7 @@ dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_para
   f.accept_rows = out->accept_rows;
   f.conf_rows = out->conf_rows;
   f.dconf = grads ? grads->dconf : nullptr;
-  return cuda_status(launch_tp_finish(prob->logits_dtype == DSPARK_F32, a, f, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_tp_finish(prob->logits_dtype == DSPARK_F32, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream) {

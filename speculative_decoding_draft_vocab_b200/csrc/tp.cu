@@ -13,7 +13,8 @@
 //   step 3  L1, S = the parts summed in rank order; over the shard
 //           dL/dz_j = g w [ce_alpha (p_j - [j = id]) + l1_alpha p_j (sign(p_j - q_j) - S)]
 // An exact tie p_j == q_j counts as sign +1 in S and in dL/dz alike.  Each step is one
-// pass over the shard's columns with one CTA per supervised row; a rank's shard of a
+// pass over the shard's columns with one CTA per supervised row (the last CTA of step 3
+// also writes the per-row epilogue and the report); a rank's shard of a
 // micro-batch (rows x V / tp_size) is small enough to stay in L2 from one step to the
 // next.  Every rank merges the same records in the same order, so all ranks hold
 // bitwise the same row statistics.
@@ -28,7 +29,6 @@ namespace {
 
 constexpr int kTpThreads = 512;
 constexpr int kTpWarps = kTpThreads / 32;
-constexpr int kTpFinThreads = 1024;
 
 // One 16-byte vector of logits as floats (8 bf16 or 4 fp32).
 template <typename T> struct Vec;
@@ -143,6 +143,8 @@ template <typename T, bool HAS_T>
 __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[2 * kTpWarps];
+  // launched behind the mask prologue: its row lists are complete past this point
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int nvec = int(a.V / VT::N);
   const int n_sup = a.ws.hdr->n_sup;
   for (int idx = blockIdx.x; idx < n_sup; idx += gridDim.x) {
@@ -238,6 +240,8 @@ template <typename T, bool HAS_T>
 __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float rowS;
+  __shared__ int last;
+  __shared__ double scratch[kTpWarps * kNAcc];
   const int nvec = int(a.V / VT::N);
   const int n_sup = a.ws.hdr->n_sup;
   const int total = n_sup + (a.dlogits ? a.ws.hdr->n_zero : 0);
@@ -302,11 +306,17 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
     }
     __syncthreads();  // rowS is rewritten for the next row
   }
-}
-
-__global__ void __launch_bounds__(kTpFinThreads) tp_final_kernel(const FinalizeArgs f) {
-  __shared__ double scratch[(kTpFinThreads / 32) * kNAcc];
-  finalize_rows(f, scratch);
+  // the last CTA to finish writes the per-row epilogue and the report
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(&a.ws.hdr->done, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (last) {
+    __threadfence();
+    finalize_rows(a.fin, scratch);
+    if (threadIdx.x == 0) a.ws.hdr->done = 0;
+  }
 }
 
 unsigned tp_grid(int64_t rows) {
@@ -316,15 +326,23 @@ unsigned tp_grid(int64_t rows) {
 }  // namespace
 
 cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s) {
-  const unsigned g = tp_grid(a.R);
+  // programmatic dependent launch: scheduled while the mask prologue runs, waiting for
+  // it (griddepcontrol.wait) before reading its lists
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tp_grid(a.R), 1, 1);
+  cfg.blockDim = dim3(kTpThreads, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   if (f32) {
-    if (a.target) tp_partials_kernel<float, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_partials_kernel<float, false><<<g, kTpThreads, 0, s>>>(a);
-  } else {
-    if (a.target) tp_partials_kernel<__nv_bfloat16, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_partials_kernel<__nv_bfloat16, false><<<g, kTpThreads, 0, s>>>(a);
+    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, true>, a)
+                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, false>, a);
   }
-  return cudaGetLastError();
+  return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<__nv_bfloat16, true>, a)
+                  : cudaLaunchKernelEx(&cfg, tp_partials_kernel<__nv_bfloat16, false>, a);
 }
 
 cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s) {
@@ -339,7 +357,7 @@ cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_tp_finish(bool f32, const TpArgs& a, const FinalizeArgs& f, cudaStream_t s) {
+cudaError_t launch_tp_finish(bool f32, const TpArgs& a, cudaStream_t s) {
   const unsigned g = tp_grid(a.R);
   if (f32) {
     if (a.target) tp_finish_kernel<float, true><<<g, kTpThreads, 0, s>>>(a);
@@ -348,9 +366,6 @@ cudaError_t launch_tp_finish(bool f32, const TpArgs& a, const FinalizeArgs& f, c
     if (a.target) tp_finish_kernel<__nv_bfloat16, true><<<g, kTpThreads, 0, s>>>(a);
     else tp_finish_kernel<__nv_bfloat16, false><<<g, kTpThreads, 0, s>>>(a);
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  tp_final_kernel<<<1, kTpFinThreads, 0, s>>>(f);
   return cudaGetLastError();
 }
 

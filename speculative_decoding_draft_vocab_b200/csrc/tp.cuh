@@ -24,6 +24,7 @@ struct TpArgs {
   const float* rec2_all;     // [tp_size][R][4]
   float ce_alpha, l1_alpha;
   WsView ws;
+  FinalizeArgs fin;          // the per-row epilogue and report the last CTA of step 3 runs
 };
 
 constexpr int kTpRec1 = 8;
@@ -31,7 +32,7 @@ constexpr int kTpRec2 = 4;
 
 cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s);
 cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s);
-// the rows' L1 and S, dlogits of the shard, then the per-row epilogue and the report
-cudaError_t launch_tp_finish(bool f32, const TpArgs& a, const FinalizeArgs& f, cudaStream_t s);
+// the rows' L1 and S, dlogits of the shard, then (last CTA) the per-row epilogue and the report
+cudaError_t launch_tp_finish(bool f32, const TpArgs& a, cudaStream_t s);
 
 }  // namespace dspark
