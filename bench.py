@@ -450,7 +450,7 @@ def run_tp(args, inp, torch_api):
                      "timed": "dspark_tp_partials + dspark_tp_l1 + dspark_tp_finish of one rank "
                               "(mask prologue, three passes over the shard, report), mean CUDA-event time"},
         "cpu_baseline": None, "e2e": None,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
