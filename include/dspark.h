@@ -250,17 +250,25 @@ DSPARK_API dspark_status_t dspark_loss_fwd_noalloc(const dspark_problem_t* prob,
  *   all-gather rec1 in rank order                               rec1_all: [tp_size][R][8]
  *   dspark_tp_l1(prob, params, tp, rec1_all, rec2, ws, ...)     rec2:     [R][4] floats
  *   all-gather rec2 in rank order                               rec2_all: [tp_size][R][4]
- *   dspark_tp_finish(prob, params, tp, rec2_all, out, grads, ws, ...)
+ *   dspark_tp_finish(prob, params, tp, rec2_all, out, grads, de_part, ws, ...)
+ * and with a head and gradients a fourth call after one more all-gather:
+ *   all-gather de_part in rank order (Markov head only)         de_all: [tp_size][R][rank]
+ *   dspark_tp_heads_bwd(prob, params, tp, de_all, grads, ws, ...)
  *
  * `prob` describes this rank's shard: V is the shard's width; draft_logits,
  * target_logits and dlogits point at the shard's first column, with the full rows'
  * strides as their leading dimensions; target_ids are GLOBAL ids in [0, vocab_size).
  * The ranks' shards must tile [0, vocab_size) without overlap.  Shard widths obey the
- * 16-byte rule above (multiples of 8 bf16 or 4 fp32 columns).  The Markov head, the
- * confidence head and the teacher from hidden states are not taken on this path
- * (DSPARK_ERR_UNSUPPORTED); given confidence logits are.  Sum the forward outputs over
- * data-parallel ranks only: every tensor-parallel rank holds the same values.  The
- * three calls of a micro-batch take the same problem, params, tp and workspace
+ * 16-byte rule above (multiples of 8 bf16 or 4 fp32 columns).  Heads follow the same
+ * design doc section: markov_w2 points at this shard's rows [V, markov_rank] (its rows
+ * split over the ranks) while markov_w1 and the confidence head are replicated; dW2 is
+ * written for this shard's rows, and the embedding gradient dL/de is the sum of the
+ * ranks' parts (the reduce across tensor parallelism) before dW1 is scattered and the
+ * confidence head's own term dc*proj_e is added once.  dW1, dconf_w, dconf_b and dhidden
+ * come out the same on every rank.  The teacher from hidden states is not taken on this
+ * path (DSPARK_ERR_UNSUPPORTED).  Sum the forward outputs and the replicated gradients
+ * over data-parallel ranks only: every tensor-parallel rank holds the same values.  The
+ * calls of a micro-batch take the same problem, params, tp and workspace
  * (dspark_workspace_size(prob) bytes), in stream order.
  *
  * Record 1 of row r (rec1 + 8r): [m_d, s_d, m_t, s_t, zt, 0, 0, 0] where, over this
@@ -294,12 +302,23 @@ DSPARK_API dspark_status_t dspark_tp_l1(const dspark_problem_t* prob, const dspa
 
 /* Step 3: sums rec2_all (rank order) into L1 and S, writes the forward outputs (as
  * dspark_loss_fwd) and, with `grads`, dlogits of this shard's columns for every row
- * (zeros where unsupervised) and dconf.  The head-gradient fields of `grads` must be
- * NULL. */
+ * (zeros where unsupervised) and dconf.  With the Markov head and `grads` it also writes
+ * dW2 for this shard's rows and this shard's part of dL/de, W2_shard^T dz_r for every
+ * row r (0 where no gradient flows), into de_part ([R][markov_rank] floats, 16-byte
+ * aligned, owned by the caller); de_part may be NULL otherwise. */
 DSPARK_API dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_params_t* params,
                                             const dspark_tp_t* tp, const float* rec2_all,
                                             const dspark_fwd_out_t* out, const dspark_grads_t* grads,
-                                            void* ws, size_t ws_bytes, dspark_stream_t stream);
+                                            float* de_part, void* ws, size_t ws_bytes, dspark_stream_t stream);
+
+/* Step 4, with a head and gradients: dL/de_r = the ranks' de_part rows summed (de_all,
+ * [tp_size][R][markov_rank], rank order; NULL without the Markov head) + dc_r*proj_e,
+ * dW1[prev_r] += dL/de_r, and the confidence head's dconf_w, dconf_b and dhidden.  The
+ * same on every rank.  Returns DSPARK_OK without work when the problem has no head. */
+DSPARK_API dspark_status_t dspark_tp_heads_bwd(const dspark_problem_t* prob, const dspark_params_t* params,
+                                               const dspark_tp_t* tp, const float* de_all,
+                                               const dspark_grads_t* grads, void* ws, size_t ws_bytes,
+                                               dspark_stream_t stream);
 
 /* Synchronises `stream` and returns the first device-side error recorded in `ws`
  * by the last call that used it (DSPARK_OK if none). */

@@ -114,8 +114,11 @@ lib.dspark_tp_l1.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_t
                              ctypes.c_size_t, c_vp]
 lib.dspark_tp_l1.restype = ctypes.c_int
 lib.dspark_tp_finish.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_tp_t), c_vp,
-                                 P(dspark_fwd_out_t), P(dspark_grads_t), c_vp, ctypes.c_size_t, c_vp]
+                                 P(dspark_fwd_out_t), P(dspark_grads_t), c_vp, c_vp, ctypes.c_size_t, c_vp]
 lib.dspark_tp_finish.restype = ctypes.c_int
+lib.dspark_tp_heads_bwd.argtypes = [P(dspark_problem_t), P(dspark_params_t), P(dspark_tp_t), c_vp,
+                                    P(dspark_grads_t), c_vp, ctypes.c_size_t, c_vp]
+lib.dspark_tp_heads_bwd.restype = ctypes.c_int
 lib.dspark_check_status.argtypes = [c_vp, c_vp]
 lib.dspark_check_status.restype = ctypes.c_int
 lib.dspark_status_string.argtypes = [ctypes.c_int]
@@ -132,6 +135,7 @@ dspark_acceptance = lib.dspark_acceptance
 dspark_tp_partials = lib.dspark_tp_partials
 dspark_tp_l1 = lib.dspark_tp_l1
 dspark_tp_finish = lib.dspark_tp_finish
+dspark_tp_heads_bwd = lib.dspark_tp_heads_bwd
 dspark_check_status = lib.dspark_check_status
 dspark_status_string = lib.dspark_status_string
 

@@ -219,14 +219,14 @@ HeadsArgs heads_args(const dspark_problem_t* p, const dspark_params_t* prm, cons
   return h;
 }
 
-// A vocabulary-parallel shard: the plain problem's rules, no heads, and a shard that
-// lies inside the vocabulary.
+// A vocabulary-parallel shard: the plain problem's rules, no teacher from hidden states,
+// and a shard that lies inside the vocabulary.
 dspark_status_t check_tp(const dspark_problem_t* p, const dspark_params_t* prm, const dspark_tp_t* tp,
                          Shape* sh) {
   if (prm == nullptr || tp == nullptr) return DSPARK_ERR_INVALID_ARG;
   dspark_status_t st = check_problem(p, prm, sh, false);
   if (st != DSPARK_OK) return st;
-  if (sh->has_markov || sh->has_conf_head || sh->has_lm_head) return DSPARK_ERR_UNSUPPORTED;
+  if (sh->has_lm_head) return DSPARK_ERR_UNSUPPORTED;
   if (tp->tp_size < 1 || tp->tp_size > 1024) return DSPARK_ERR_INVALID_ARG;
   if (tp->vocab_size <= 0 || tp->vocab_size > (int64_t(1) << 30) || tp->vocab_begin < 0 ||
       tp->vocab_begin > tp->vocab_size - p->V)
@@ -253,6 +253,7 @@ TpArgs tp_args(const dspark_problem_t* p, const dspark_params_t* prm, const dspa
   a.tp_size = int32_t(tp->tp_size);
   a.ce_alpha = prm->ce_alpha;
   a.l1_alpha = p->target_logits ? prm->l1_alpha : 0.f;
+  a.bias = markov_present(p) ? ws.bias : nullptr;
   a.ws = ws;
   return a;
 }
@@ -421,14 +422,24 @@ dspark_status_t dspark_tp_partials(const dspark_problem_t* prob, const dspark_pa
   PrologueArgs pa{};
   pa.B = prob->B; pa.N = prob->N; pa.K = prob->K;
   pa.V = tp->vocab_size;  // target ids are global
+  pa.Vt = prob->target_vocab;
   pa.eval_mask = prob->eval_mask;
   pa.block_keep = prob->block_keep;
   pa.target_ids = prob->target_ids;
+  pa.prev_ids = sh.has_markov ? prob->prev_ids : nullptr;
+  pa.valid = prob->valid;
+  pa.invalid_zero = sh.has_markov && params->invalid_row_mode == 0;
   pa.gamma = params->gamma;
   pa.gamma_enabled = params->gamma_enabled;
   pa.ws = v;
   cudaError_t e = launch_prologue(pa, s);
   if (e != cudaSuccess) return cuda_status(e);
+  if (sh.has_markov || sh.has_conf_head) {
+    // embeddings and confidence logits (replicated), the bias rows of this shard
+    const HeadsArgs ha = heads_args(prob, params, v, nullptr);
+    if ((e = launch_heads_prep(ha, s)) != cudaSuccess) return cuda_status(e);
+    if (sh.has_markov && (e = launch_markov_bias(ha, s)) != cudaSuccess) return cuda_status(e);
+  }
   TpArgs a = tp_args(prob, params, tp, v);
   a.rec1 = rec1;
   return cuda_status(launch_tp_partials(prob->logits_dtype == DSPARK_F32, a, s));
@@ -451,8 +462,8 @@ dspark_status_t dspark_tp_l1(const dspark_problem_t* prob, const dspark_params_t
 
 dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_params_t* params,
                                  const dspark_tp_t* tp, const float* rec2_all,
-                                 const dspark_fwd_out_t* out, const dspark_grads_t* grads, void* ws,
-                                 size_t ws_bytes, dspark_stream_t stream) {
+                                 const dspark_fwd_out_t* out, const dspark_grads_t* grads, float* de_part,
+                                 void* ws, size_t ws_bytes, dspark_stream_t stream) {
   if (out == nullptr) return DSPARK_ERR_INVALID_ARG;
   Shape sh{};
   dspark_status_t st = check_tp(prob, params, tp, &sh);
@@ -461,8 +472,8 @@ dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_para
   if ((st = check_rec(rec2_all)) != DSPARK_OK) return st;
   if (grads) {
     if ((st = check_grads(prob, grads)) != DSPARK_OK) return st;
-    if (grads->dW1 || grads->dW2 || grads->dconf_w || grads->dconf_b || grads->dhidden)
-      return DSPARK_ERR_INVALID_ARG;
+    // this shard's part of dL/de goes to de_part
+    if (sh.has_markov && (st = check_rec(de_part)) != DSPARK_OK) return st;
   }
   const WsView v = ws_layout(ws, ws_dims(prob));
   TpArgs a = tp_args(prob, params, tp, v);
@@ -476,7 +487,7 @@ dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_para
   f.B = prob->B; f.N = prob->N; f.K = prob->K;
   f.block_keep = prob->block_keep;
   f.confidence_logits = prob->confidence_logits;
-  f.has_conf = sh.has_conf_given;
+  f.has_conf = sh.has_conf_given || sh.has_conf_head;
   f.ce_alpha = params->ce_alpha;
   f.l1_alpha = params->l1_alpha;
   f.conf_alpha = params->conf_alpha;
@@ -490,7 +501,26 @@ dspark_status_t dspark_tp_finish(const dspark_problem_t* prob, const dspark_para
   f.accept_rows = out->accept_rows;
   f.conf_rows = out->conf_rows;
   f.dconf = grads ? grads->dconf : nullptr;
-  return cuda_status(launch_tp_finish(prob->logits_dtype == DSPARK_F32, a, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_tp_finish(prob->logits_dtype == DSPARK_F32, a, s);
+  if (e == cudaSuccess && grads && sh.has_markov)
+    e = launch_markov_bwd_shard(heads_args(prob, params, v, grads), de_part, s);
+  return cuda_status(e);
+}
+
+dspark_status_t dspark_tp_heads_bwd(const dspark_problem_t* prob, const dspark_params_t* params,
+                                    const dspark_tp_t* tp, const float* de_all, const dspark_grads_t* grads,
+                                    void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  Shape sh{};
+  dspark_status_t st = check_tp(prob, params, tp, &sh);
+  if (st != DSPARK_OK) return st;
+  if ((st = check_ws(prob, ws, ws_bytes)) != DSPARK_OK) return st;
+  if ((st = check_grads(prob, grads)) != DSPARK_OK) return st;
+  if (sh.has_markov && (st = check_rec(de_all)) != DSPARK_OK) return st;
+  if (!sh.has_markov && !sh.has_conf_head) return DSPARK_OK;  // no head: nothing to do
+  const WsView v = ws_layout(ws, ws_dims(prob));
+  return cuda_status(launch_heads_bwd_merge(heads_args(prob, params, v, grads), de_all, int(tp->tp_size),
+                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream) {

@@ -107,15 +107,17 @@ struct WeightEpi {
   __device__ void coords(int m0, int n0, int, int& x, int& y, int& z) const { x = n0, y = m0, z = -1; }
 };
 
-// ---- dE = sum of the split partials (+ dc proj_e), then dW1[prev] += dE
-__global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const int splits) {
+// ---- dE = sum of the partials (+ dc proj_e), then dW1[prev] += dE.  The partials are
+// [splits][R][rank]: the K splits of the dE GEMM, or the vocabulary-parallel ranks' parts
+// in rank order.
+__global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const float* parts, const int splits) {
   const int64_t n = a.R * a.rank;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t r = i / a.rank, j = i - r * a.rank;
     const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
     float acc = 0.f;
     if (live) {
-      const float* dp = a.ws.dep + size_t(r) * a.rank + j;
+      const float* dp = parts + size_t(r) * a.rank + j;
       const size_t stride = size_t(a.R) * a.rank;
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;  // loads in flight together; fixed order
       int s = 0;
@@ -133,6 +135,31 @@ __global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const
       if (a.dw1 != nullptr) atomicAdd(a.dw1 + size_t(pv) * a.rank + j, acc);
     }
     a.ws.de[i] = acc;
+  }
+}
+
+// ---- one vocabulary-parallel rank's part of dE: the K splits of its dE GEMM summed in
+// the order de_reduce_kernel uses (0 on rows without a gradient)
+__global__ void __launch_bounds__(256) de_split_sum_kernel(const HeadsArgs a, const int splits, float* out) {
+  const int64_t n = a.R * a.rank;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / a.rank, j = i - r * a.rank;
+    float acc = 0.f;
+    if (a.ws.m[r] != 0 && a.valid[r] != 0) {
+      const float* dp = a.ws.dep + size_t(r) * a.rank + j;
+      const size_t stride = size_t(a.R) * a.rank;
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+      int s = 0;
+      for (; s + 4 <= splits; s += 4) {
+        p0 += dp[s * stride];
+        p1 += dp[(s + 1) * stride];
+        p2 += dp[(s + 2) * stride];
+        p3 += dp[(s + 3) * stride];
+      }
+      for (; s < splits; ++s) p0 += dp[s * stride];
+      acc = (p0 + p1) + (p2 + p3);
+    }
+    out[i] = acc;
   }
 }
 
@@ -312,32 +339,38 @@ cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
                                         &a.ws.hdr->n_sup, 0, &mo);
 }
 
-cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
+namespace {
+
+// dE split partials into ws.dep and dW2 (its rows of the vocabulary) from the bf16 dlogits
+cudaError_t markov_grad_gemms(const HeadsArgs& a, int splits, cudaStream_t s) {
+  // dE partials: A = dlogits [R][V] (K-major), B = W2 as [V][rank] (MN-major)
+  CUtensorMap ma, mb;
+  if (!tc::make_map(&ma, a.dlogits, a.R, a.V, a.ld_g, 64, 128)) return cudaErrorInvalidValue;
+  if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
+  CUtensorMap mo;
+  if (!tc::make_out_map(&mo, a.ws.dep, a.R, a.rank, a.rank, splits, a.R * a.rank)) return cudaErrorInvalidValue;
+  cudaError_t e = tc::gemm<256, false, true, 4>(ma, mb, int(a.R), int(a.rank), int(a.V), splits, PartialEpi{},
+                                                &a.ws.hdr->status, s, nullptr, 0, &mo);
+  if (e != cudaSuccess) return e;
+  // dW2 = dlogits^T . E: A = dlogits as [R][V] (MN-major, M = vocabulary),
+  // B = E by row [R][rank] (MN-major)
+  if (a.dw2 != nullptr) {
+    CUtensorMap ma2, mb2;
+    if (!tc::make_map(&ma2, a.dlogits, a.R, a.V, a.ld_g, 64, 64)) return cudaErrorInvalidValue;
+    if (!tc::make_map(&mb2, a.ws.eall, a.R, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
+    CUtensorMap mo2;
+    if (!tc::make_out_map(&mo2, a.dw2, a.V, a.rank, a.rank)) return cudaErrorInvalidValue;
+    e = tc::gemm<256, true, true, 4>(ma2, mb2, int(a.V), int(a.rank), int(a.R), 1, WeightEpi{a.accumulate},
+                                     &a.ws.hdr->status, s, nullptr, 0, &mo2);
+  }
+  return e;
+}
+
+// dE from its partials, dW1, then the confidence head's gradients
+cudaError_t merge_and_conf_grads(const HeadsArgs& a, const float* parts, int nparts, cudaStream_t s) {
   cudaError_t e = cudaSuccess;
   if (a.w1 != nullptr) {
-    const int splits = heads_splits(a.R, a.V);
-    // dE partials: A = dlogits [R][V] (K-major), B = W2 as [V][rank] (MN-major)
-    CUtensorMap ma, mb;
-    if (!tc::make_map(&ma, a.dlogits, a.R, a.V, a.ld_g, 64, 128)) return cudaErrorInvalidValue;
-    if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
-    CUtensorMap mo;
-    if (!tc::make_out_map(&mo, a.ws.dep, a.R, a.rank, a.rank, splits, a.R * a.rank)) return cudaErrorInvalidValue;
-    e = tc::gemm<256, false, true, 4>(ma, mb, int(a.R), int(a.rank), int(a.V), splits, PartialEpi{},
-                                      &a.ws.hdr->status, s, nullptr, 0, &mo);
-    if (e != cudaSuccess) return e;
-    // dW2 = dlogits^T . E: A = dlogits as [R][V] (MN-major, M = vocabulary),
-    // B = E by row [R][rank] (MN-major)
-    if (a.dw2 != nullptr) {
-      CUtensorMap ma2, mb2;
-      if (!tc::make_map(&ma2, a.dlogits, a.R, a.V, a.ld_g, 64, 64)) return cudaErrorInvalidValue;
-      if (!tc::make_map(&mb2, a.ws.eall, a.R, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
-      CUtensorMap mo2;
-      if (!tc::make_out_map(&mo2, a.dw2, a.V, a.rank, a.rank)) return cudaErrorInvalidValue;
-      e = tc::gemm<256, true, true, 4>(ma2, mb2, int(a.V), int(a.rank), int(a.R), 1, WeightEpi{a.accumulate},
-                                       &a.ws.hdr->status, s, nullptr, 0, &mo2);
-      if (e != cudaSuccess) return e;
-    }
-    de_reduce_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, splits);
+    de_reduce_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, parts, nparts);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.conf_w != nullptr) {
@@ -354,6 +387,29 @@ cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
     }
   }
   return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
+  const int splits = a.w1 != nullptr ? heads_splits(a.R, a.V) : 0;
+  if (a.w1 != nullptr) {
+    const cudaError_t e = markov_grad_gemms(a, splits, s);
+    if (e != cudaSuccess) return e;
+  }
+  return merge_and_conf_grads(a, a.ws.dep, splits, s);
+}
+
+cudaError_t launch_markov_bwd_shard(const HeadsArgs& a, float* de_part, cudaStream_t s) {
+  const int splits = heads_splits(a.R, a.V);
+  const cudaError_t e = markov_grad_gemms(a, splits, s);
+  if (e != cudaSuccess) return e;
+  de_split_sum_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, splits, de_part);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_heads_bwd_merge(const HeadsArgs& a, const float* de_all, int nranks, cudaStream_t s) {
+  return merge_and_conf_grads(a, de_all, nranks, s);
 }
 
 }  // namespace dspark

@@ -12,6 +12,9 @@
 //           S part = sum_j p_j sign(p_j - q_j), p = 2^(z' - lse'_z), q = 2^(t' - lse'_t)
 //   step 3  L1, S = the parts summed in rank order; over the shard
 //           dL/dz_j = g w [ce_alpha (p_j - [j = id]) + l1_alpha p_j (sign(p_j - q_j) - S)]
+// With the Markov head the shard's corrected logits z = keep * base + bias are formed on
+// chip from the base rows and the head's FP32 bias rows of the shard (keep = 0 only on an
+// invalid slot whose corrected row is all zero; no gradient flows to its base row).
 // An exact tie p_j == q_j counts as sign +1 in S and in dL/dz alike.  Each step is one
 // pass over the shard's columns with one CTA per supervised row (the last CTA of step 3
 // also writes the per-row epilogue and the report); a rank's shard of a
@@ -133,13 +136,27 @@ __device__ __forceinline__ void block_sum2(float& x, float& y, float2* sh) {
   __syncthreads();
 }
 
+// z = keep * base + bias for one vector of the shard (bias rows are FP32, N per vector)
+template <int N>
+__device__ __forceinline__ void add_bias(float* x, const float* brow, int v, float keep) {
+  const float4* b4 = reinterpret_cast<const float4*>(brow + size_t(v) * N);
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    const float4 b = b4[q];
+    x[4 * q + 0] = fmaf(x[4 * q + 0], keep, b.x);
+    x[4 * q + 1] = fmaf(x[4 * q + 1], keep, b.y);
+    x[4 * q + 2] = fmaf(x[4 * q + 2], keep, b.z);
+    x[4 * q + 3] = fmaf(x[4 * q + 3], keep, b.w);
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ const uint8_t* row_ptr(const void* base, int64_t row, int64_t ld) {
   return static_cast<const uint8_t*>(base) + size_t(row) * size_t(ld) * sizeof(T);
 }
 
 // ---------------------------------------------------------------- step 1
-template <typename T, bool HAS_T>
+template <typename T, bool HAS_T, bool HAS_B>
 __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[2 * kTpWarps];
@@ -151,11 +168,14 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
     const int64_t row = a.ws.sup_list[idx];
     const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
     const uint8_t* tr = HAS_T ? row_ptr<T>(a.target, row, a.ld_t) : nullptr;
+    const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
+    const float keep = (HAS_B && a.ws.sup_tok[idx] < 0) ? 0.f : 1.f;
     float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
 #pragma unroll 2
     for (int v = threadIdx.x; v < nvec; v += kTpThreads) {
       float x[VT::N];
       VT::load(zr + size_t(v) * 16, x);
+      if constexpr (HAS_B) add_bias<VT::N>(x, br, v, keep);
       if constexpr (HAS_T) {
         float y[VT::N];
         VT::load(tr + size_t(v) * 16, y);
@@ -166,7 +186,11 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
     block_lse2(mz, sz, mt, st, sh);
     if (threadIdx.x == 0) {
       const int64_t col = a.tids[row] - a.vocab_begin;
-      const float zt = (col >= 0 && col < a.V) ? VT::elem(zr + size_t(col) * sizeof(T)) : 0.f;
+      float zt = 0.f;
+      if (col >= 0 && col < a.V) {
+        zt = VT::elem(zr + size_t(col) * sizeof(T));
+        if constexpr (HAS_B) zt = fmaf(zt, keep, br[col]);
+      }
       float4* rec = reinterpret_cast<float4*>(a.rec1 + size_t(row) * kTpRec1);
       rec[0] = make_float4(mz, sz, HAS_T ? mt : -INFINITY, HAS_T ? st : 0.f);
       rec[1] = make_float4(zt, 0.f, 0.f, 0.f);
@@ -175,7 +199,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
 }
 
 // ---------------------------------------------------------------- step 2
-template <typename T, bool HAS_T>
+template <typename T, bool HAS_T, bool HAS_B>
 __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[kTpWarps];
@@ -214,10 +238,13 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
       const float lz = lse2.x, lt = lse2.y;
       const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
       const uint8_t* tr = row_ptr<T>(a.target, row, a.ld_t);
+      const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
+      const float keep = (HAS_B && a.ws.sup_tok[idx] < 0) ? 0.f : 1.f;
 #pragma unroll 2
       for (int v = threadIdx.x; v < nvec; v += kTpThreads) {
         float x[VT::N], y[VT::N];
         VT::load(zr + size_t(v) * 16, x);
+        if constexpr (HAS_B) add_bias<VT::N>(x, br, v, keep);
         VT::load(tr + size_t(v) * 16, y);
 #pragma unroll
         for (int e = 0; e < VT::N; ++e) {
@@ -236,7 +263,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
 }
 
 // ---------------------------------------------------------------- step 3
-template <typename T, bool HAS_T>
+template <typename T, bool HAS_T, bool HAS_B>
 __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float rowS;
@@ -270,18 +297,23 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
     if (a.dlogits) {
       const float S = rowS;
       const float g = a.grad_scale ? *a.grad_scale : 1.f;
-      const float gw = g * a.ws.w[row];
+      // an all-zero corrected row is a constant: nothing flows to its base row
+      const bool zero_row = HAS_B && a.ws.sup_tok[idx] < 0;
+      const float gw = zero_row ? 0.f : g * a.ws.w[row];
       const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
       const float kpos = cce + cl1 * (1.f - S), kneg = cce + cl1 * (-1.f - S);
       const float lz = st[kStLseD] * kLog2e, lt = st[kStLseT] * kLog2e;
       const int64_t col = a.tids[row] - a.vocab_begin;
       const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
       const uint8_t* tr = HAS_T ? row_ptr<T>(a.target, row, a.ld_t) : nullptr;
+      const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
+      const float keep = zero_row ? 0.f : 1.f;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * size_t(a.ld_g) * sizeof(T);
 #pragma unroll 2
       for (int v = threadIdx.x; v < nvec; v += kTpThreads) {
         float x[VT::N], o[VT::N];
         VT::load(zr + size_t(v) * 16, x);
+        if constexpr (HAS_B) add_bias<VT::N>(x, br, v, keep);
         if constexpr (HAS_T) {
           float y[VT::N];
           VT::load(tr + size_t(v) * 16, y);
@@ -337,34 +369,47 @@ cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at;
   cfg.numAttrs = 1;
+  using bf16 = __nv_bfloat16;
   if (f32) {
-    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, true>, a)
-                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, false>, a);
+    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, true, false>, a)
+                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, false, false>, a);
   }
-  return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<__nv_bfloat16, true>, a)
-                  : cudaLaunchKernelEx(&cfg, tp_partials_kernel<__nv_bfloat16, false>, a);
+  if (a.bias) {  // the Markov head needs bf16 logits
+    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, true>, a)
+                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, true>, a);
+  }
+  return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, false>, a)
+                  : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, false>, a);
 }
 
 cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s) {
   const unsigned g = tp_grid(a.R);
+  using bf16 = __nv_bfloat16;
   if (f32) {
-    if (a.target) tp_l1_kernel<float, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_l1_kernel<float, false><<<g, kTpThreads, 0, s>>>(a);
+    if (a.target) tp_l1_kernel<float, true, false><<<g, kTpThreads, 0, s>>>(a);
+    else tp_l1_kernel<float, false, false><<<g, kTpThreads, 0, s>>>(a);
+  } else if (a.bias) {
+    if (a.target) tp_l1_kernel<bf16, true, true><<<g, kTpThreads, 0, s>>>(a);
+    else tp_l1_kernel<bf16, false, true><<<g, kTpThreads, 0, s>>>(a);
   } else {
-    if (a.target) tp_l1_kernel<__nv_bfloat16, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_l1_kernel<__nv_bfloat16, false><<<g, kTpThreads, 0, s>>>(a);
+    if (a.target) tp_l1_kernel<bf16, true, false><<<g, kTpThreads, 0, s>>>(a);
+    else tp_l1_kernel<bf16, false, false><<<g, kTpThreads, 0, s>>>(a);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_tp_finish(bool f32, const TpArgs& a, cudaStream_t s) {
   const unsigned g = tp_grid(a.R);
+  using bf16 = __nv_bfloat16;
   if (f32) {
-    if (a.target) tp_finish_kernel<float, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_finish_kernel<float, false><<<g, kTpThreads, 0, s>>>(a);
+    if (a.target) tp_finish_kernel<float, true, false><<<g, kTpThreads, 0, s>>>(a);
+    else tp_finish_kernel<float, false, false><<<g, kTpThreads, 0, s>>>(a);
+  } else if (a.bias) {
+    if (a.target) tp_finish_kernel<bf16, true, true><<<g, kTpThreads, 0, s>>>(a);
+    else tp_finish_kernel<bf16, false, true><<<g, kTpThreads, 0, s>>>(a);
   } else {
-    if (a.target) tp_finish_kernel<__nv_bfloat16, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_finish_kernel<__nv_bfloat16, false><<<g, kTpThreads, 0, s>>>(a);
+    if (a.target) tp_finish_kernel<bf16, true, false><<<g, kTpThreads, 0, s>>>(a);
+    else tp_finish_kernel<bf16, false, false><<<g, kTpThreads, 0, s>>>(a);
   }
   return cudaGetLastError();
 }

@@ -22,6 +22,7 @@ struct TpArgs {
   const float* rec1_all;     // [tp_size][R][8] every rank's, rank order
   float* rec2;               // [R][4] this shard's (L1, S) partials
   const float* rec2_all;     // [tp_size][R][4]
+  const float* bias;         // Markov bias rows of the shard (compact by supervised position), or null
   float ce_alpha, l1_alpha;
   WsView ws;
   FinalizeArgs fin;          // the per-row epilogue and report the last CTA of step 3 runs
@@ -34,5 +35,12 @@ cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s);
 cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s);
 // the rows' L1 and S, dlogits of the shard, then (last CTA) the per-row epilogue and the report
 cudaError_t launch_tp_finish(bool f32, const TpArgs& a, cudaStream_t s);
+
+// Markov head on a vocabulary shard (csrc/heads.cu): the dE GEMM against this shard's
+// W2 rows, its K splits summed into de_part [R][rank], and dW2 for this shard's rows
+cudaError_t launch_markov_bwd_shard(const HeadsArgs& a, float* de_part, cudaStream_t s);
+// dE from the ranks' parts de_all [nranks][R][rank] (+ dc proj_e), dW1, and the
+// confidence head's gradients
+cudaError_t launch_heads_bwd_merge(const HeadsArgs& a, const float* de_all, int nranks, cudaStream_t s);
 
 }  // namespace dspark

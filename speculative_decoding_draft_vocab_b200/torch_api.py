@@ -211,19 +211,24 @@ def even_shards(V: int, tp_size: int, align: int) -> list:
 
 
 class TPRank:
-    """One tensor-parallel rank's three calls (dspark_tp_partials, dspark_tp_l1,
-    dspark_tp_finish) on its vocabulary shard of a micro-batch.
+    """One tensor-parallel rank's calls (dspark_tp_partials, dspark_tp_l1,
+    dspark_tp_finish, and with a head dspark_tp_heads_bwd) on its vocabulary shard of a
+    micro-batch.
 
     ``inp`` holds rows that contain this rank's shard at columns [col0, col0 + width):
     the full rows (single-device emulation of a group) or just the shard (one rank per
-    GPU, col0 = 0).  The shard is addressed in place, with the rows' stride.  dlogits of
-    the shard go to the same columns of ``dlogits`` (rows shaped like ``inp``'s), or of
-    a buffer this rank allocates.  Every rank writes its own copy of the forward outputs.
+    GPU, col0 = 0).  The shard is addressed in place, with the rows' stride; so are the
+    shard's rows of ``inp.markov_w2`` (rows col0 .. col0 + width).  dlogits of the shard
+    go to the same columns of ``dlogits`` (rows shaped like ``inp``'s), and dW2 of the
+    shard to the same rows of ``dW2`` (shaped like ``inp.markov_w2``), or to buffers this
+    rank allocates.  Every rank writes its own copy of the forward outputs and of the
+    replicated gradients (dW1, dconf_w, dconf_b, dhidden).
     """
 
     def __init__(self, inp: DSparkInputs, tp_size: int, vocab_begin: int, vocab_size: int,
                  col0: int = 0, width: Optional[int] = None, dlogits: Optional[torch.Tensor] = None,
-                 grads: bool = True, rows: bool = True):
+                 dW2: Optional[torch.Tensor] = None, grads: bool = True, rows: bool = True,
+                 invalid_row_mode: int = 0):
         dev = inp.draft_logits.device
         R = inp.R
         es = 4 if inp.dtype == "f32" else 2
@@ -234,8 +239,12 @@ class TPRank:
         p.draft_logits = ctypes.c_void_p(inp.draft_logits.data_ptr() + col0 * es)
         if inp.target_logits is not None:
             p.target_logits = ctypes.c_void_p(inp.target_logits.data_ptr() + col0 * es)
+        markov = inp.markov_w2 is not None
+        rank_ = inp.markov_w2.shape[1] if markov else 0
+        if markov:
+            p.markov_w2 = ctypes.c_void_p(inp.markov_w2.data_ptr() + col0 * rank_ * 2)
         self.prob = p
-        self.prm = params_struct(inp)
+        self.prm = params_struct(inp, invalid_row_mode)
         self.tp = abi.dspark_tp_t(tp_size, vocab_begin, vocab_size)
         f32 = dict(dtype=torch.float32, device=dev)
         self.rec1 = torch.empty(R, abi.DSPARK_TP_REC1_FLOATS, **f32)
@@ -252,6 +261,15 @@ class TPRank:
         if grads and dlogits is None:
             dlogits = torch.zeros_like(inp.draft_logits)
         self.dlogits = dlogits if grads else None
+        self.dW1 = self.dW2 = self.dconf_w = self.dconf_b = self.dhidden = self.de_part = None
+        if grads and markov:
+            self.dW1 = torch.zeros(inp.markov_w1.shape, **f32)
+            self.dW2 = torch.zeros(inp.markov_w2.shape, **f32) if dW2 is None else dW2
+            self.de_part = torch.zeros(R, rank_, **f32)
+        if grads and inp.conf_w is not None:
+            self.dconf_w = torch.zeros(inp.conf_w.numel(), **f32)
+            self.dconf_b = torch.zeros(1, **f32)
+            self.dhidden = torch.zeros(inp.draft_hidden.shape, dtype=torch.bfloat16, device=dev)
         o = abi.dspark_fwd_out_t()
         o.loss_num, o.num_tokens, o.report = _ptr(self.loss_num), _ptr(self.num_tokens), _ptr(self.report)
         o.ce_rows, o.l1_rows = _ptr(self.ce_rows), _ptr(self.l1_rows)
@@ -264,7 +282,12 @@ class TPRank:
             g.dlogits = ctypes.c_void_p(self.dlogits.data_ptr() + col0 * es)
             g.dlogits_ld = inp.V
             g.dconf = _ptr(self.dconf)
+            g.dW1 = _ptr(self.dW1)
+            if self.dW2 is not None:
+                g.dW2 = ctypes.c_void_p(self.dW2.data_ptr() + col0 * rank_ * 4)
+            g.dconf_w, g.dconf_b, g.dhidden = _ptr(self.dconf_w), _ptr(self.dconf_b), _ptr(self.dhidden)
             self.grads = g
+        self.has_heads = markov or inp.conf_w is not None
         self.ws = new_workspace(inp)
         self.ws_ptr, self.ws_len = _aligned_ws(self.ws)
 
@@ -290,14 +313,25 @@ class TPRank:
         st = abi.dspark_tp_finish(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.tp),
                                   _ptr(rec2_all), ctypes.byref(self.fwd),
                                   ctypes.byref(self.grads) if self.grads is not None else None,
-                                  self.ws_ptr, self.ws_len, self._stream(stream))
+                                  _ptr(self.de_part), self.ws_ptr, self.ws_len, self._stream(stream))
         abi.check(st, "dspark_tp_finish")
+        return self.de_part
+
+    def heads_bwd(self, de_all: Optional[torch.Tensor], stream=None) -> None:
+        _need(de_all, torch.float32, "de_all")
+        st = abi.dspark_tp_heads_bwd(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.tp),
+                                     _ptr(de_all), ctypes.byref(self.grads), self.ws_ptr, self.ws_len,
+                                     self._stream(stream))
+        abi.check(st, "dspark_tp_heads_bwd")
 
     def run(self, exchange) -> None:
-        """The three calls, with ``exchange`` (this rank's records -> every rank's records
-        stacked in rank order, e.g. ``tp_exchange``) after each of the first two."""
+        """The calls, with ``exchange`` (this rank's records -> every rank's records
+        stacked in rank order, e.g. ``tp_exchange``) after each of the first two and, with
+        the Markov head, after the third."""
         rec1_all = exchange(self.partials())
-        self.finish(exchange(self.l1(rec1_all)))
+        de_part = self.finish(exchange(self.l1(rec1_all)))
+        if self.grads is not None and self.has_heads:
+            self.heads_bwd(exchange(de_part) if de_part is not None else None)
 
     def check_status(self, stream=None) -> int:
         return int(abi.dspark_check_status(self.ws_ptr, self._stream(stream)))
@@ -312,7 +346,8 @@ def tp_exchange(local: torch.Tensor, group=None) -> torch.Tensor:
     return torch.stack(parts)
 
 
-def tp_group_emulated(inp: DSparkInputs, tp_size: int, grads: bool = True, rows: bool = True) -> list:
+def tp_group_emulated(inp: DSparkInputs, tp_size: int, grads: bool = True, rows: bool = True,
+                      invalid_row_mode: int = 0) -> list:
     """A whole tensor-parallel group on this device: tp_size ranks over even shards of
     ``inp``'s full rows, stepped together, the exchange being a stack of the ranks'
     records (what the all-gather delivers).  The ranks share one dlogits buffer, each
@@ -320,10 +355,16 @@ def tp_group_emulated(inp: DSparkInputs, tp_size: int, grads: bool = True, rows:
     align = 4 if inp.dtype == "f32" else 8
     bounds = even_shards(inp.V, tp_size, align)
     dl = torch.zeros_like(inp.draft_logits) if grads else None
+    dw2 = torch.zeros(inp.markov_w2.shape, dtype=torch.float32, device=inp.draft_logits.device) \
+        if (grads and inp.markov_w2 is not None) else None
     ranks = [TPRank(inp, tp_size, bounds[k], inp.V, col0=bounds[k], width=bounds[k + 1] - bounds[k],
-                    dlogits=dl, grads=grads, rows=rows) for k in range(tp_size)]
+                    dlogits=dl, dW2=dw2, grads=grads, rows=rows, invalid_row_mode=invalid_row_mode)
+             for k in range(tp_size)]
     rec1_all = torch.stack([r.partials() for r in ranks])
     rec2_all = torch.stack([r.l1(rec1_all) for r in ranks])
-    for r in ranks:
-        r.finish(rec2_all)
+    parts = [r.finish(rec2_all) for r in ranks]
+    if grads and ranks[0].has_heads:
+        de_all = torch.stack(parts) if parts[0] is not None else None
+        for r in ranks:
+            r.heads_bwd(de_all)
     return ranks

@@ -266,24 +266,31 @@ def test_target_norm_validation(abi):
 
 
 def _tp_calls(abi, p, prm, tp, rec=0x200000, ws=0x100000, ws_bytes=1 << 30, grads=None):
-    """Status of each of the three vocabulary-parallel calls on the same arguments."""
+    """Status of each of the four vocabulary-parallel calls on the same arguments (the
+    head call gets a gradient struct of its own when none is given)."""
     r = ctypes.c_void_p(rec)
     out = abi.dspark_fwd_out_t()
+    g4 = grads
+    if g4 is None:
+        g4 = abi.dspark_grads_t()
+        g4.dlogits, g4.dlogits_ld = ctypes.c_void_p(0x70000), p.V
     return (abi.dspark_tp_partials(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r,
                                    ctypes.c_void_p(ws), ws_bytes, None),
             abi.dspark_tp_l1(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r, r,
                              ctypes.c_void_p(ws), ws_bytes, None),
             abi.dspark_tp_finish(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r, ctypes.byref(out),
-                                 ctypes.byref(grads) if grads is not None else None,
-                                 ctypes.c_void_p(ws), ws_bytes, None))
+                                 ctypes.byref(grads) if grads is not None else None, r,
+                                 ctypes.c_void_p(ws), ws_bytes, None),
+            abi.dspark_tp_heads_bwd(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), r, ctypes.byref(g4),
+                                    ctypes.c_void_p(ws), ws_bytes, None))
 
 
 def test_vocab_parallel_validation(abi):
-    """Shard bounds, record buffers, the heads (not taken on this path) and head
-    gradients are checked on the host, by all three calls alike."""
+    """Shard bounds, record buffers, the teacher from hidden states (not taken on this
+    path) and the gradient buffers are checked on the host, by every call alike."""
     prm = _params(abi)
     p = _problem(abi, V=1024)
-    every = lambda st: (st,) * 3
+    every = lambda st: (st,) * 4
     # the shard must lie inside the vocabulary
     assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2, 1024, 1024 + 1000)) == every(abi.DSPARK_ERR_INVALID_ARG)
     assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2, -8, 4096)) == every(abi.DSPARK_ERR_INVALID_ARG)
@@ -292,24 +299,27 @@ def test_vocab_parallel_validation(abi):
     assert _tp_calls(abi, p, prm, abi.dspark_tp_t(2, 0, (1 << 30) + 8)) == every(abi.DSPARK_ERR_INVALID_ARG)
     # records: present and 16-byte aligned
     tp = abi.dspark_tp_t(4, 1024, 4096)
-    assert _tp_calls(abi, p, prm, tp, rec=0) == every(abi.DSPARK_ERR_INVALID_ARG)
-    assert _tp_calls(abi, p, prm, tp, rec=0x200008) == every(abi.DSPARK_ERR_ALIGNMENT)
+    # (without the Markov head the fourth call reads no record and has no work)
+    assert _tp_calls(abi, p, prm, tp, rec=0) == (abi.DSPARK_ERR_INVALID_ARG,) * 3 + (abi.DSPARK_OK,)
+    assert _tp_calls(abi, p, prm, tp, rec=0x200008) == (abi.DSPARK_ERR_ALIGNMENT,) * 3 + (abi.DSPARK_OK,)
     # the plain problem's rules still hold (shard width under the 16-byte rule, workspace)
     assert _tp_calls(abi, _problem(abi, V=1020), prm, tp) == every(abi.DSPARK_ERR_ALIGNMENT)
     assert _tp_calls(abi, p, prm, tp, ws_bytes=16) == every(abi.DSPARK_ERR_WORKSPACE)
     assert _tp_calls(abi, _problem(abi, target=False), prm, tp) == every(abi.DSPARK_ERR_MISSING_TARGET)
-    # heads are not taken on the vocabulary-parallel path
-    assert _tp_calls(abi, _with_markov(abi, _problem(abi)), prm, tp) == every(abi.DSPARK_ERR_UNSUPPORTED)
-    assert _tp_calls(abi, _with_conf_head(abi, _problem(abi)), prm, tp) == every(abi.DSPARK_ERR_UNSUPPORTED)
+    # the teacher from hidden states is not taken on the vocabulary-parallel path
     assert _tp_calls(abi, _with_lm_head(abi, _problem(abi, target=False)), prm, tp) == \
         every(abi.DSPARK_ERR_UNSUPPORTED)
-    # head-gradient fields must stay NULL; a misaligned dlogits stride is refused
+    # with the Markov head the shard's dE part and the ranks' parts are records too
+    pm = _with_markov(abi, _problem(abi))
     g = abi.dspark_grads_t()
     g.dlogits, g.dlogits_ld = ctypes.c_void_p(0x70000), 4096
-    g.dW2 = ctypes.c_void_p(0x80000)
-    assert _tp_calls(abi, p, prm, tp, grads=g)[2] == abi.DSPARK_ERR_INVALID_ARG
-    g.dW2, g.dlogits_ld = None, 1028
-    assert _tp_calls(abi, p, prm, tp, grads=g)[2] == abi.DSPARK_ERR_ALIGNMENT
+    assert _tp_calls(abi, pm, prm, tp, rec=0x200008, grads=g) == every(abi.DSPARK_ERR_ALIGNMENT)
+    assert _tp_calls(abi, pm, prm, tp, rec=0, grads=g) == every(abi.DSPARK_ERR_INVALID_ARG)
+    # a misaligned dlogits stride or head gradient is refused
+    g.dlogits_ld = 1028
+    assert _tp_calls(abi, p, prm, tp, grads=g)[2:] == (abi.DSPARK_ERR_ALIGNMENT,) * 2
+    g.dlogits_ld, g.dW2 = 4096, ctypes.c_void_p(0x80008)
+    assert _tp_calls(abi, pm, prm, tp, grads=g)[2:] == (abi.DSPARK_ERR_ALIGNMENT,) * 2
     # NULL params / tp / outputs
     out = abi.dspark_fwd_out_t()
     assert abi.dspark_tp_partials(ctypes.byref(p), None, ctypes.byref(tp), ctypes.c_void_p(0x200000),
@@ -318,7 +328,10 @@ def test_vocab_parallel_validation(abi):
                             ctypes.c_void_p(0x200000), ctypes.c_void_p(0x100000), 1 << 30,
                             None) == abi.DSPARK_ERR_INVALID_ARG
     assert abi.dspark_tp_finish(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), ctypes.c_void_p(0x200000),
-                                None, None, ctypes.c_void_p(0x100000), 1 << 30, None) == abi.DSPARK_ERR_INVALID_ARG
+                                None, None, None, ctypes.c_void_p(0x100000), 1 << 30,
+                                None) == abi.DSPARK_ERR_INVALID_ARG
+    assert abi.dspark_tp_heads_bwd(ctypes.byref(p), ctypes.byref(prm), ctypes.byref(tp), None, None,
+                                   ctypes.c_void_p(0x100000), 1 << 30, None) == abi.DSPARK_ERR_INVALID_ARG
     del out
 
 

@@ -17,7 +17,7 @@ import torch
 
 from oracle import dspark_oracle as O
 from speculative_decoding_draft_vocab_b200.synthetic import make_inputs
-from tests.parity_util import check_dlogit_row, compare, np32, oracle_run
+from tests.parity_util import check_dlogit_row, check_heads, compare, np32, oracle_run
 
 pytestmark = pytest.mark.gpu
 
@@ -29,9 +29,9 @@ def _built():
     assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
 
 
-def _group(inp, tp_size, grads=True):
+def _group(inp, tp_size, grads=True, mode=0):
     from speculative_decoding_draft_vocab_b200 import torch_api
-    ranks = torch_api.tp_group_emulated(inp, tp_size, grads=grads)
+    ranks = torch_api.tp_group_emulated(inp, tp_size, grads=grads, invalid_row_mode=mode)
     torch.cuda.synchronize()
     for r in ranks:
         assert r.check_status() == 0
@@ -42,7 +42,9 @@ def _as_call(rank):
     """The fields of one rank that the parity helpers read."""
     return SimpleNamespace(out=SimpleNamespace(
         num_tokens=rank.num_tokens, report=rank.report, loss_num=rank.loss_num, ce_rows=rank.ce_rows,
-        l1_rows=rank.l1_rows, accept_rows=rank.accept_rows, dconf=rank.dconf, dlogits=rank.dlogits))
+        l1_rows=rank.l1_rows, accept_rows=rank.accept_rows, conf_rows=rank.conf_rows, dconf=rank.dconf,
+        dlogits=rank.dlogits, dW1=rank.dW1, dW2=rank.dW2, dconf_w=rank.dconf_w, dconf_b=rank.dconf_b,
+        dhidden=rank.dhidden))
 
 
 def _check_group(inp, ranks, ref, **kw):
@@ -145,3 +147,47 @@ def test_tp_recipe_workload_every_row():
     assert torch.equal(fused.out.num_tokens, ranks[0].num_tokens)
     rel = (fused.out.report - ranks[0].report).abs() / fused.out.report.abs().clamp_min(1e-6)
     assert float(rel.max()) <= 2e-5
+
+
+HEADS = dict(B=2, N=4, K=7, V=8192, hidden=512, rank=64, target_vocab=3000, markov_std=0.3,
+             conf_bias=0.25, valid_p=0.7, mask_holes=True)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("T", [2, 4])
+def test_tp_heads_match_oracle(mode, T):
+    """Markov head with W2's rows split over the ranks and the confidence head fed the
+    Markov embedding: forward, dlogits and every weight gradient against the oracle, for
+    both invalid-row readings.  dW2 is assembled from the ranks' rows; dL/de is the sum of
+    the ranks' parts, so dW1, dproj, dbias and dh come out the same on every rank."""
+    inp = make_inputs("recipe_heads", device="cuda", seed=50 + mode + 2 * T, conf_with_markov=True, **HEADS)
+    inp.prev_ids = torch.where(inp.valid != 0, inp.prev_ids, torch.full_like(inp.prev_ids, -1))
+    ranks = _group(inp, T, mode=mode)
+    ref = oracle_run(inp, invalid_row_mode=mode)
+    _check_group(inp, ranks, ref)
+    check_heads(inp, _as_call(ranks[0]), ref, mode)
+    for r in ranks[1:]:
+        for name in ("dconf_w", "dconf_b", "dhidden", "conf_rows"):
+            assert torch.equal(getattr(r, name), getattr(ranks[0], name)), name
+        # dW1 is a scatter-add (atomics): the same values up to the order of the adds
+        assert torch.allclose(r.dW1, ranks[0].dW1, rtol=1e-5, atol=1e-9)
+
+
+def test_tp_markov_without_confidence_and_ragged_rank():
+    """rank 72 (a ragged tensor-core tile), three ranks over V = 5000 (uneven shards)."""
+    inp = make_inputs("recipe_heads", device="cuda", seed=57, B=3, N=5, K=6, V=5000, hidden=200, rank=72,
+                      target_vocab=777, markov_std=0.3, conf=None, valid_p=0.8)
+    ranks = _group(inp, 3)
+    ref = oracle_run(inp)
+    _check_group(inp, ranks, ref)
+    check_heads(inp, _as_call(ranks[0]), ref, 0)
+
+
+def test_tp_recipe_heads_workload_every_row():
+    """The C3 shape (4 x 16 x 7 rows, V = 151936, rank 256, hidden 4096) on 8 ranks."""
+    inp = make_inputs("recipe_heads", device="cuda")
+    ranks = _group(inp, 8)
+    ref = oracle_run(inp)
+    _check_group(inp, ranks, ref)
+    st = check_heads(inp, _as_call(ranks[0]), ref, 0)
+    assert st["dW2_frob_err"] <= 1.0 and st["dW1_frob_err"] <= 1.0
