@@ -165,12 +165,13 @@ def test_tp_heads_match_oracle(mode, T):
     ranks = _group(inp, T, mode=mode)
     ref = oracle_run(inp, invalid_row_mode=mode)
     _check_group(inp, ranks, ref)
-    check_heads(inp, _as_call(ranks[0]), ref, mode)
+    for r in ranks:
+        # dW1 is a scatter-add (atomics, in no fixed order): every rank's is checked
+        # against the oracle with the derived bound, not bit for bit against rank 0's
+        check_heads(inp, _as_call(r), ref, mode)
     for r in ranks[1:]:
         for name in ("dconf_w", "dconf_b", "dhidden", "conf_rows"):
             assert torch.equal(getattr(r, name), getattr(ranks[0], name)), name
-        # dW1 is a scatter-add (atomics): the same values up to the order of the adds
-        assert torch.allclose(r.dW1, ranks[0].dW1, rtol=1e-5, atol=1e-9)
 
 
 def test_tp_markov_without_confidence_and_ragged_rank():
