@@ -1,11 +1,12 @@
 """The vocabulary-parallel exchange protocol on CPU ranks (gloo): each rank holds one
 vocabulary shard of every row, reduces it to the records include/dspark.h defines
-(record 1: base-2 logsumexp partials and the target logit; record 2: L1 and S parts),
-and ``torch_api.tp_exchange`` (the binding's all-gather) hands every rank all ranks'
-records in rank order.  Merged in that order they give the full-row CE, L1 and S of
-the oracle, identically on every rank (NeMo RL design doc "DSpark Auxiliary Heads",
-Tensor Parallelism).  The per-shard arithmetic is the oracle's (no GPU here); the
-record layout, the exchange and the rank order are the product's."""
+(record 1: base-2 logsumexp partials and the target logit; record 2: L1 and S parts;
+with the Markov head, its part of dL/de), and ``torch_api.tp_exchange`` (the binding's
+all-gather) hands every rank all ranks' records in rank order.  Merged in that order
+they give the full-row CE, L1 and S and the embedding gradient of the oracle,
+identically on every rank (NeMo RL design doc "DSpark Auxiliary Heads", Tensor
+Parallelism).  The per-shard arithmetic is the oracle's (no GPU here); the record
+layout, the exchange and the rank order are the product's."""
 
 import math
 import os
@@ -93,3 +94,57 @@ def test_vocab_parallel_records_merge_to_full_rows(world):
             assert abs(lse_d - full["lse_d"]) <= 1e-12 and abs(lse_t - full["lse_t"]) <= 1e-12
             assert abs(ce - full["ce"]) <= 1e-12
             assert abs(l1 - full["l1"]) <= 1e-12 and abs(S - full["S"]) <= 1e-12
+
+
+def _heads_problem(seed=9, B=1, N=2, K=4, V=48, rank=8, H=6, Vt=11):
+    rng = np.random.default_rng(seed)
+    d = rng.normal(0, 1.5, (B, N, K, V))
+    t = 0.8 * d + rng.normal(0, 1.0, (B, N, K, V))
+    ids = rng.integers(0, V, (B, N, K))
+    ev = np.ones((B, N, K), dtype=np.uint8)
+    ev[0, 1, 3] = 0
+    kw = dict(target_logits=t, prev_ids=rng.integers(0, Vt, (B, N, K)),
+              valid=np.array([[[1, 1, 0, 1], [1, 1, 1, 1]]]), markov_w1=rng.normal(0, 0.4, (Vt, rank)),
+              markov_w2=rng.normal(0, 0.4, (V, rank)), draft_hidden=rng.normal(size=(B, N, K, H)),
+              conf_w=rng.normal(0, 0.3, (1, H + rank)), conf_b=np.array([0.1]), conf_with_markov=True)
+    return d, ids, ev, kw
+
+
+def _heads_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from speculative_decoding_draft_vocab_b200.torch_api import even_shards, tp_exchange
+    d, ids, ev, kw = _heads_problem()
+    res = O.dspark_loss(d, ids, ev, **kw)  # every rank holds the rows' dz (after the three steps)
+    R, V = ids.size, d.shape[-1]
+    w2 = kw["markov_w2"]
+    b = even_shards(V, world, 8)
+    lo, hi = b[rank], b[rank + 1]
+    # this rank's part of dL/de: its rows of W2 against its columns of dz
+    part = torch.zeros(R, w2.shape[1], dtype=torch.float64)
+    for r in res["dE"]:
+        part[r] = torch.from_numpy(w2[lo:hi].T @ res["dlogits"][r][lo:hi])
+    parts = tp_exchange(part)
+    proj_e = np.asarray(kw["conf_w"]).reshape(-1)[kw["draft_hidden"].shape[-1]:]  # proj's embedding slice
+    merged = {r: sum(parts[k, r].numpy() for k in range(world)) + res["dconf"][r] * proj_e for r in res["dE"]}
+    out[rank] = {r: v.tolist() for r, v in merged.items()}
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_vocab_parallel_embedding_gradient_reduced_across_ranks(world):
+    """dL/de = sum over ranks of W2_k^T dz_k (the reduce across tensor parallelism), plus
+    the replicated confidence head's dc * proj_e once: the oracle's dL/de on every rank."""
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_heads_worker, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+    d, ids, ev, kw = _heads_problem()
+    ref = O.dspark_loss(d, ids, ev, **kw)
+    assert len(ref["dE"]) > 0
+    for k in range(world):
+        assert out[k] == out[0]
+        for r, want in ref["dE"].items():
+            np.testing.assert_allclose(out[k][r], want, rtol=0, atol=1e-12)
