@@ -89,6 +89,14 @@ def algorithmic_bytes(inp, n_sup: int) -> int:
     return b
 
 
+def tp_algorithmic_bytes(inp, n_sup: int, width: int) -> int:
+    """One vocabulary-parallel rank's share of the single-pass bytes: its columns of the
+    supervised rows' draft and teacher logits read once, its columns of every row's
+    dlogits written once."""
+    es = 2 if inp.dtype == "bf16" else 4
+    return n_sup * width * es * (2 if inp.target_logits is not None else 1) + inp.R * width * es
+
+
 def algorithmic_flops(inp, n_sup: int) -> int:
     """Tensor-core work a perfect implementation must do: the Markov bias, dE and dW2
     contractions (2 * rows * V * rank each) and the teacher product (2 * rows * V * Ht)."""
@@ -428,11 +436,8 @@ def run_tp(args, inp, torch_api):
         raise SystemExit("device status after the timed steps")
     per_step = [s_.elapsed_time(e) for s_, e in zip(starts, ends)]
     mean_ms = statistics.mean(per_step)
-    es = 2 if inp.dtype == "bf16" else 4
     width = r0.width
-    # this rank's share of the single-pass bytes: its columns of the supervised rows'
-    # draft and teacher read once, its columns of every row's dlogits written once
-    alg = n_sup * width * es * 2 + inp.R * width * es
+    alg = tp_algorithmic_bytes(inp, n_sup, width)
     peak, peak_kind = hbm_peak()
     achieved = alg / (mean_ms / 1e3) / 1e9
     line = {

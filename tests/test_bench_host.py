@@ -1,0 +1,55 @@
+"""The roofline arithmetic of bench.py, pinned to sums written out by hand: the
+algorithmic bytes and tensor-core FLOPs of each workload's call and of one
+vocabulary-parallel rank.  Shapes only (meta tensors); no GPU."""
+
+from types import SimpleNamespace
+
+import torch
+
+import bench
+
+V = 151936
+
+
+def _inp(R=448, dtype="bf16", target=True, markov_rank=None, hidden=None, lm_hidden=None, Vt=V):
+    meta = dict(device="meta")
+    return SimpleNamespace(
+        dtype=dtype, V=V, R=R,
+        target_logits=torch.empty(R, V, **meta) if target else None,
+        markov_w2=torch.empty(V, markov_rank, **meta) if markov_rank else None,
+        markov_w1=torch.empty(Vt, markov_rank, **meta) if markov_rank else None,
+        conf_w=torch.empty(1, hidden, **meta) if hidden else None,
+        draft_hidden=torch.empty(R, hidden, **meta) if hidden else None,
+        lm_head=torch.empty(V, lm_hidden, **meta) if lm_hidden else None)
+
+
+def test_recipe_bytes():
+    """251 supervised rows of 448: draft and teacher read once (2 B each per logit),
+    dlogits written for every row."""
+    assert bench.algorithmic_bytes(_inp(), 251) == 251 * V * 2 * 2 + 448 * V * 2 == 288_678_400
+    assert bench.algorithmic_flops(_inp(), 251) == 0
+
+
+def test_heads_bytes_and_flops():
+    """Markov rank 256 (W2 read in bf16, dW2 written in fp32; the supervised rows'
+    embeddings and their dW1 rows) and the confidence head's hidden rows (read and
+    gradient written, bf16); three rank-256 contractions against the vocabulary."""
+    inp = _inp(markov_rank=256, hidden=4096)
+    want = (252 * V * 2 * 2 + 448 * V * 2) + V * 256 * (2 + 4) + 252 * 256 * (2 + 4) + 448 * 4096 * 2 * 2
+    assert bench.algorithmic_bytes(inp, 252) == want
+    assert bench.algorithmic_flops(inp, 252) == 3 * 2 * 252 * V * 256
+
+
+def test_teacher_from_hidden_bytes_and_flops():
+    """lm_head [V, 4096] and the supervised rows' hidden states read instead of teacher
+    logits; the teacher product is 2 * rows * V * 4096 FLOPs."""
+    inp = _inp(target=False, lm_hidden=4096)
+    assert bench.algorithmic_bytes(inp, 245) == 245 * V * 2 + 448 * V * 2 + V * 4096 * 2 + 245 * 4096 * 2
+    assert bench.algorithmic_flops(inp, 245) == 2 * 245 * V * 4096
+
+
+def test_tp_rank_bytes():
+    """One rank of eight: 18992 columns of the 251 supervised rows' draft and teacher,
+    and of all 448 rows' dlogits."""
+    assert bench.tp_algorithmic_bytes(_inp(), 251, 18992) == 251 * 18992 * 4 + 448 * 18992 * 2 == 36_084_800
+    assert bench.tp_algorithmic_bytes(_inp(target=False), 251, 18992) == 251 * 18992 * 2 + 448 * 18992 * 2
