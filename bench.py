@@ -92,9 +92,36 @@ def algorithmic_bytes(inp, n_sup: int) -> int:
 def tp_algorithmic_bytes(inp, n_sup: int, width: int) -> int:
     """One vocabulary-parallel rank's share of the single-pass bytes: its columns of the
     supervised rows' draft and teacher logits read once, its columns of every row's
-    dlogits written once."""
+    dlogits written once; with the heads, its rows of W2 read and of dW2 written, the
+    supervised rows' embeddings and dW1 rows, and the hidden states read and their
+    gradient written (the replicated heads' work is every rank's)."""
     es = 2 if inp.dtype == "bf16" else 4
-    return n_sup * width * es * (2 if inp.target_logits is not None else 1) + inp.R * width * es
+    b = n_sup * width * es * (2 if inp.target_logits is not None else 1) + inp.R * width * es
+    if inp.markov_w2 is not None:
+        r = inp.markov_w2.shape[1]
+        b += width * r * (2 + 4) + n_sup * r * (2 + 4)
+    if inp.conf_w is not None:
+        b += inp.draft_hidden.numel() * 2 * 2
+    return b
+
+
+def tp_algorithmic_flops(inp, n_sup: int, width: int) -> int:
+    """One rank's tensor-core work: the Markov bias, dE and dW2 contractions against its
+    columns (2 * rows * width * rank each)."""
+    return 3 * 2 * n_sup * width * inp.markov_w2.shape[1] if inp.markov_w2 is not None else 0
+
+
+def tp_launches_per_step(inp) -> int:
+    """Kernels one rank's calls launch per micro-batch."""
+    n = 4  # mask prologue, the three steps
+    markov, conf = inp.markov_w2 is not None, inp.conf_w is not None
+    if markov or conf:
+        n += 1  # embeddings and confidence logits
+    if markov:
+        n += 1 + 3 + 1  # bias GEMM; dE GEMM, dW2 GEMM, split sum; the merge of the ranks' parts
+    if conf:
+        n += 3  # dproj partials, dproj final, dhidden
+    return n
 
 
 def algorithmic_flops(inp, n_sup: int) -> int:
@@ -401,8 +428,9 @@ def main():
 
 
 def run_tp(args, inp, torch_api):
-    """One rank (rank 0) of a vocabulary-parallel group of args.tp ranks: its three calls
-    per step on its shard, L2 flushed before each step, CUDA events around the three."""
+    """One rank (rank 0) of a vocabulary-parallel group of args.tp ranks: its calls per step
+    on its shard (three, four with a head), L2 flushed before each step, CUDA events
+    around them; the other ranks' records come from one emulated group run before."""
     ranks = torch_api.tp_group_emulated(inp, args.tp, rows=False)
     torch.cuda.synchronize()
     for r in ranks:
@@ -410,6 +438,7 @@ def run_tp(args, inp, torch_api):
             raise SystemExit("device status after the emulated group")
     rec1_all = torch.stack([r.rec1 for r in ranks])
     rec2_all = torch.stack([r.rec2 for r in ranks])
+    de_all = torch.stack([r.de_part for r in ranks]) if ranks[0].de_part is not None else None
     r0 = ranks[0]
     del ranks[1:]
     n_sup = int(r0.num_tokens.item())
@@ -419,6 +448,8 @@ def run_tp(args, inp, torch_api):
         r0.partials()
         r0.l1(rec1_all)
         r0.finish(rec2_all)
+        if r0.has_heads:
+            r0.heads_bwd(de_all)
 
     for _ in range(args.warmup):
         step()
@@ -438,8 +469,22 @@ def run_tp(args, inp, torch_api):
     mean_ms = statistics.mean(per_step)
     width = r0.width
     alg = tp_algorithmic_bytes(inp, n_sup, width)
+    flops = tp_algorithmic_flops(inp, n_sup, width)
     peak, peak_kind = hbm_peak()
-    achieved = alg / (mean_ms / 1e3) / 1e9
+    tpeak, tpeak_kind = tensor_peak()
+    timed = ("one rank's dspark_tp_partials + dspark_tp_l1 + dspark_tp_finish"
+             + (" + dspark_tp_heads_bwd" if r0.has_heads else "")
+             + f" ({tp_launches_per_step(inp)} kernels), mean CUDA-event time")
+    if alg / (peak * 1e9) >= flops / (tpeak * 1e12):
+        achieved = alg / (mean_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                    "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
+    else:
+        achieved = flops / (mean_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": round(achieved / tpeak, 4), "peak_kind": tpeak_kind, "traffic": None,
+                    "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
     line = {
         "metric": METRIC, "value": round(n_sup / (mean_ms / 1e3), 1), "unit": "rows/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_ms, 5),
@@ -448,14 +493,10 @@ def run_tp(args, inp, torch_api):
         "config": {"workload": workload_desc(args.workload, inp), "parallelism": f"tp{args.tp} (one rank timed)",
                    "shard_columns": width, "supervised_rows": n_sup,
                    "l2": "flushed before every timed step (512 MiB write, untimed)",
-                   "not_timed": "the two all-gathers of per-row records between the calls"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None,
-                     "algorithmic_bytes": alg,
-                     "timed": "dspark_tp_partials + dspark_tp_l1 + dspark_tp_finish of one rank "
-                              "(mask prologue, three passes over the shard, report), mean CUDA-event time"},
+                   "not_timed": "the all-gathers of per-row records between the calls"},
+        "roofline": roofline,
         "cpu_baseline": None, "e2e": None,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": tp_launches_per_step(inp) * args.steps,
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

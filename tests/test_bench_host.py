@@ -53,3 +53,14 @@ def test_tp_rank_bytes():
     and of all 448 rows' dlogits."""
     assert bench.tp_algorithmic_bytes(_inp(), 251, 18992) == 251 * 18992 * 4 + 448 * 18992 * 2 == 36_084_800
     assert bench.tp_algorithmic_bytes(_inp(target=False), 251, 18992) == 251 * 18992 * 2 + 448 * 18992 * 2
+
+
+def test_tp_rank_heads_bytes_flops_and_launches():
+    """A rank's W2 rows (read bf16, gradient written fp32), the supervised embeddings and
+    dW1 rows, the hidden states; three rank-256 contractions against its columns."""
+    inp = _inp(markov_rank=256, hidden=4096)
+    want = 252 * 18992 * 4 + 448 * 18992 * 2 + 18992 * 256 * 6 + 252 * 256 * 6 + 448 * 4096 * 4
+    assert bench.tp_algorithmic_bytes(inp, 252, 18992) == want
+    assert bench.tp_algorithmic_flops(inp, 252, 18992) == 6 * 252 * 18992 * 256
+    assert bench.tp_launches_per_step(_inp()) == 4
+    assert bench.tp_launches_per_step(inp) == 4 + 1 + 5 + 3
