@@ -201,8 +201,8 @@ def even_shards(V: int, tp_size: int, align: int) -> list:
     """Bounds [0, v_1, ..., V] of tp_size contiguous vocabulary shards whose widths are
     multiples of ``align`` columns (8 bf16 / 4 fp32: the 16-byte rule), as even as
     that allows (the first shards take the remainder)."""
-    if V % align or tp_size < 1:
-        raise ValueError("V must be a multiple of align and tp_size >= 1")
+    if V % align or tp_size < 1 or V // align < tp_size:
+        raise ValueError("V must be a multiple of align, with at least one vector of align columns per rank")
     base, extra = divmod(V // align, tp_size)
     bounds = [0]
     for k in range(tp_size):

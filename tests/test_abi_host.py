@@ -343,3 +343,6 @@ def test_even_shards():
     assert max(y - x for x, y in zip(b, b[1:])) - min(y - x for x, y in zip(b, b[1:])) <= 8
     with pytest.raises(ValueError):
         even_shards(1001, 2, 8)
+    with pytest.raises(ValueError):  # an empty shard
+        even_shards(16, 3, 8)
+    assert even_shards(24, 3, 8) == [0, 8, 16, 24]
