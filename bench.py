@@ -42,6 +42,7 @@ METRIC = "supervised rows/s, DSpark loss fwd+bwd @V=151936; achieved HBM GB/s vs
 PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0  # the B200 data-sheet HBM3e bandwidth the loss target is quoted against
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sweep_recipe_traffic.md")
 KERNEL_SOURCES = ["speculative_decoding_draft_vocab_b200/csrc/sweep.cu",
                   "speculative_decoding_draft_vocab_b200/csrc/prologue.cu",
@@ -87,6 +88,36 @@ def algorithmic_bytes(inp, n_sup: int) -> int:
     if inp.conf_w is not None:
         b += inp.draft_hidden.numel() * 2 * 2
     return b
+
+
+def dense_bytes(inp) -> int:
+    """Every row's draft (and teacher) logits read and dlogits written, masked or not: the
+    dense "logits read plus dlogits written" figure."""
+    es = 2 if inp.dtype == "bf16" else 4
+    return inp.R * inp.V * es * (3 if inp.target_logits is not None else 2)
+
+
+def roofline_entry(alg: int, flops: int, mean_ms: float, hbm, tensor, timed: str, traffic=None,
+                   dense=None) -> dict:
+    """The roofline object of a JSON line: the bound is whichever of the algorithmic bytes
+    (at the measured HBM peak) and FLOPs (at the measured bf16 peak) takes longer; an HBM
+    bound also reports the fraction of the nominal bandwidth and, given ``dense``, the
+    dense figure's rate."""
+    (peak, peak_kind), (tpeak, tpeak_kind) = hbm, tensor
+    sec = mean_ms / 1e3
+    common = {"traffic": traffic, "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
+    if alg / (peak * 1e9) >= flops / (tpeak * 1e12):
+        achieved = alg / sec / 1e9
+        r = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+             "frac": round(achieved / peak, 4), "peak_kind": peak_kind, **common,
+             "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4)}
+        if dense is not None:
+            r["dense_bytes"] = dense
+            r["dense_achieved"] = round(dense / sec / 1e9, 1)
+        return r
+    achieved = flops / sec / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak, "unit": "TFLOP/s",
+            "frac": round(achieved / tpeak, 4), "peak_kind": tpeak_kind, **common}
 
 
 def tp_algorithmic_bytes(inp, n_sup: int, width: int) -> int:
@@ -375,25 +406,14 @@ def main():
     # needs; the bound is whichever takes longer at its measured peak
     alg = algorithmic_bytes(inp, n_sup)
     flops = algorithmic_flops(inp, n_sup)
-    peak, peak_kind = hbm_peak()
-    tpeak, tpeak_kind = tensor_peak()
     mean_ms = statistics.mean(per_step)
-    t_hbm, t_tc = alg / (peak * 1e9), flops / (tpeak * 1e12)
     n_launch = launches_per_call(inp)
     timed = (f"dspark_loss_fwd with fused backward ({n_launch} kernels: "
              + ("mask prologue + sweep" if n_launch == 2 else "prologue, heads, sweep, head gradients")
              + "), mean CUDA-event duration per call")
-    if t_hbm >= t_tc:
-        achieved = alg / (mean_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                    "traffic": recorded_traffic() if n_launch == 2 else None, "algorithmic_bytes": alg,
-                    "algorithmic_flops": flops, "timed": timed}
-    else:
-        achieved = flops / (mean_ms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak, "unit": "TFLOP/s",
-                    "frac": round(achieved / tpeak, 4), "peak_kind": tpeak_kind, "traffic": None,
-                    "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
+    roofline = roofline_entry(alg, flops, mean_ms, hbm_peak(), tensor_peak(), timed,
+                              traffic=recorded_traffic() if n_launch == 2 else None,
+                              dense=dense_bytes(inp) if n_launch == 2 else None)
 
     # ---- end to end from pinned host buffers
     e2e = run_e2e(inp, args.e2e_steps, torch_api)
@@ -470,21 +490,10 @@ def run_tp(args, inp, torch_api):
     width = r0.width
     alg = tp_algorithmic_bytes(inp, n_sup, width)
     flops = tp_algorithmic_flops(inp, n_sup, width)
-    peak, peak_kind = hbm_peak()
-    tpeak, tpeak_kind = tensor_peak()
     timed = ("one rank's dspark_tp_partials + dspark_tp_l1 + dspark_tp_finish"
              + (" + dspark_tp_heads_bwd" if r0.has_heads else "")
              + f" ({tp_launches_per_step(inp)} kernels), mean CUDA-event time")
-    if alg / (peak * 1e9) >= flops / (tpeak * 1e12):
-        achieved = alg / (mean_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None,
-                    "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
-    else:
-        achieved = flops / (mean_ms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tpeak, "unit": "TFLOP/s",
-                    "frac": round(achieved / tpeak, 4), "peak_kind": tpeak_kind, "traffic": None,
-                    "algorithmic_bytes": alg, "algorithmic_flops": flops, "timed": timed}
+    roofline = roofline_entry(alg, flops, mean_ms, hbm_peak(), tensor_peak(), timed)
     line = {
         "metric": METRIC, "value": round(n_sup / (mean_ms / 1e3), 1), "unit": "rows/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_ms, 5),

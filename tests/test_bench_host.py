@@ -64,3 +64,21 @@ def test_tp_rank_heads_bytes_flops_and_launches():
     assert bench.tp_algorithmic_flops(inp, 252, 18992) == 6 * 252 * 18992 * 256
     assert bench.tp_launches_per_step(_inp()) == 4
     assert bench.tp_launches_per_step(inp) == 4 + 1 + 5 + 3
+
+
+def test_roofline_entry_bound_and_fractions():
+    """The C2 call: 288,678,400 B in 0.0974 ms is 2963.8 GB/s, 0.459 of the measured
+    6458.1 GB/s and 0.370 of the nominal 8 TB/s; the dense figure counts every row's
+    draft, teacher and dlogits (448 x 151936 x 6 B)."""
+    hbm, tc = (6458.1, "measured"), (1590.0, "measured")
+    r = bench.roofline_entry(288_678_400, 0, 0.0974, hbm, tc, "t", traffic=1, dense=bench.dense_bytes(_inp()))
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 1
+    assert r["achieved"] == round(288_678_400 / 0.0974e-3 / 1e9, 1)
+    assert r["frac"] == round(288_678_400 / 0.0974e-3 / 1e9 / 6458.1, 4) == 0.4589
+    assert r["frac_of_nominal"] == round(288_678_400 / 0.0974e-3 / 1e9 / 8000.0, 4)
+    assert r["dense_bytes"] == 448 * V * 6 == 408_403_968
+    # the teacher product's FLOPs outweigh its bytes at these peaks: a tensor bound
+    t = bench.roofline_entry(1_000_000, 10**12, 1.0, hbm, tc, "t")  # 1 TFLOP in 1 ms: 1000 TFLOP/s
+    assert t["bound"] == "tensor" and t["unit"] == "TFLOP/s" and t["achieved"] == 1000.0
+    assert t["frac"] == round(1000.0 / 1590.0, 4)
+    assert "frac_of_nominal" not in t
