@@ -108,6 +108,7 @@ def test_teacher_from_prenorm_hidden(heads):
 
 
 def test_prenorm_teacher_config_every_row():
-    """The C4 shape with pre-norm 4096-wide hidden states."""
+    """The lm_head teacher shape (4 x 16 x 7 rows, lm_head 151936 x 4096) with pre-norm
+    4096-wide hidden states."""
     inp = make_inputs("lm_head_teacher", device="cuda", seed=53, target_prenorm=True)
     _run(inp)

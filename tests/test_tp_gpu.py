@@ -185,7 +185,8 @@ def test_tp_markov_without_confidence_and_ragged_rank():
 
 
 def test_tp_recipe_heads_workload_every_row():
-    """The C3 shape (4 x 16 x 7 rows, V = 151936, rank 256, hidden 4096) on 8 ranks."""
+    """The recipe shape with both heads (4 x 16 x 7 rows, V = 151936, rank 256, hidden 4096)
+    on 8 ranks."""
     inp = make_inputs("recipe_heads", device="cuda")
     ranks = _group(inp, 8)
     ref = oracle_run(inp)
