@@ -68,9 +68,9 @@ def test_tp_rank_heads_bytes_flops_and_launches():
 
 def test_roofline_entry_bound_and_fractions():
     """The recipe call (4 x 16 x 7 x 151936 bf16, 251 supervised rows): 288,678,400 B in
-    0.0974 ms is 2963.8 GB/s, 0.459 of the measured
-    6458.1 GB/s and 0.370 of the nominal 8 TB/s; the dense figure counts every row's
-    draft, teacher and dlogits (448 x 151936 x 6 B)."""
+    0.0974 ms is 2963.8 GB/s, 0.459 of the measured 6458.1 GB/s and 0.370 of the nominal
+    8 TB/s; the dense figure counts every row's draft, teacher and dlogits (448 x 151936
+    x 6 B)."""
     hbm, tc = (6458.1, "measured"), (1590.0, "measured")
     r = bench.roofline_entry(288_678_400, 0, 0.0974, hbm, tc, "t", traffic=1, dense=bench.dense_bytes(_inp()))
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 1
