@@ -318,6 +318,8 @@ class TPRank:
         return self.de_part
 
     def heads_bwd(self, de_all: Optional[torch.Tensor], stream=None) -> None:
+        if self.grads is None:
+            raise ValueError("this rank was built without gradients")
         _need(de_all, torch.float32, "de_all")
         st = abi.dspark_tp_heads_bwd(ctypes.byref(self.prob), ctypes.byref(self.prm), ctypes.byref(self.tp),
                                      _ptr(de_all), ctypes.byref(self.grads), self.ws_ptr, self.ws_len,
