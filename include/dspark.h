@@ -215,14 +215,22 @@ DSPARK_API dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, co
  * a service of this library).  For callers that cannot allocate device memory or pass
  * a workspace, e.g. an operator plugin whose host framework owns all device memory, or
  * a runtime that forbids cudaMalloc/cudaFree while serving because they synchronise the
- * device: the workspace is a fixed __device__ array inside this library, 467,200 bytes,
- * held on every GPU that loads the library until the process exits.  Same problem,
- * params, outputs and gradients as dspark_loss_fwd; nothing is allocated.
- *  - Serves micro-batches of at most 8192 rows (B*N*K) without the Markov head (whose
- *    corrected rows need 4*V bytes per row); others return DSPARK_ERR_WORKSPACE before
- *    anything is enqueued.
- *  - The first call on a device looks the array's device address up (once per device,
- *    with that device current); make that first call before any stream capture.
+ * device: the workspace is a fixed __device__ array inside this library,
+ * DSPARK_NOALLOC_BYTES bytes, held on every GPU that loads the library until the process
+ * exits.  Same problem, params, outputs and gradients as dspark_loss_fwd; nothing is
+ * allocated.
+ *  - Serves exactly the problems with at most DSPARK_NOALLOC_MAX_ROWS rows (B*N*K) and
+ *    dspark_workspace_size(prob) <= DSPARK_NOALLOC_BYTES; every other problem returns
+ *    DSPARK_ERR_WORKSPACE before anything is enqueued.  Without heads that is every
+ *    micro-batch of at most 8192 rows.  The Markov head (its FP32 bias rows take 4*V
+ *    bytes per supervised row) and the teacher from hidden states (its FP32 teacher chunk
+ *    takes 4*V bytes per chunk row) never fit at a real vocabulary.  A confidence head
+ *    adds ceil(R/16)*(hidden_size [+ markov_rank])*4 bytes of partial sums, so with
+ *    hidden_size 4096 it fits only up to about 430 rows (the 448-row recipe micro-batch
+ *    with a confidence head is refused).
+ *  - The first call on a device (and the first after that device's context was torn down
+ *    and created again) looks the array's device address up, with that device current;
+ *    make that first call before any stream capture.
  *  - Every call on a device shares the one array and leaves its contents behind; the
  *    next call clears what must start at zero.  Calls that overlap on the GPU (other
  *    streams, other threads) race on the array: serialise them.
@@ -230,6 +238,8 @@ DSPARK_API dspark_status_t dspark_acceptance(int64_t B, int64_t N, int64_t K, co
  *    is no workspace pointer to pass to dspark_check_status); rows with out-of-range ids
  *    are still skipped.
  */
+enum { DSPARK_NOALLOC_MAX_ROWS = 8192, DSPARK_NOALLOC_BYTES = 467200 };
+
 DSPARK_API dspark_status_t dspark_loss_fwd_noalloc(const dspark_problem_t* prob,
                                                    const dspark_params_t* params,
                                                    const dspark_fwd_out_t* out,

@@ -49,7 +49,7 @@ forms, invariants, brute force and finite differences.
 from __future__ import annotations
 
 import math
-from typing import Callable, Optional
+from typing import Optional
 
 import numpy as np
 
@@ -240,13 +240,6 @@ def target_final_norm(hidden_rows, weight, eps) -> np.ndarray:
     w = np.asarray(weight, dtype=np.float64).reshape(-1)
     y = w * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + float(eps))
     return torch.from_numpy(y).to(torch.bfloat16).double().numpy()
-
-
-def teacher_rows_from_hidden(hidden_rows, lm_head) -> np.ndarray:
-    """t = lm_head @ h per row: [TS-PR] scope list, the teacher distribution comes
-    from the target model's output projection applied to its last hidden state
-    (taken here as already passed through the final norm)."""
-    return np.asarray(hidden_rows, dtype=np.float64) @ np.asarray(lm_head, dtype=np.float64).T
 
 
 def confidence_head_logits(hidden_rows, e_rows, proj, bias, valid_rows) -> np.ndarray:

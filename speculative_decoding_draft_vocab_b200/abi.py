@@ -129,8 +129,10 @@ dspark_workspace_size = lib.dspark_workspace_size
 dspark_loss_fwd = lib.dspark_loss_fwd
 dspark_loss_bwd = lib.dspark_loss_bwd
 dspark_loss_fwd_noalloc = lib.dspark_loss_fwd_noalloc
-# Rows (B*N*K) the fixed scratch of dspark_loss_fwd_noalloc serves.
+# The fixed scratch of dspark_loss_fwd_noalloc: the rows (B*N*K) and the workspace bytes
+# it serves (DSPARK_NOALLOC_MAX_ROWS, DSPARK_NOALLOC_BYTES of dspark.h).
 NOALLOC_MAX_ROWS = 8192
+NOALLOC_BYTES = 467200
 dspark_acceptance = lib.dspark_acceptance
 dspark_tp_partials = lib.dspark_tp_partials
 dspark_tp_l1 = lib.dspark_tp_l1

@@ -346,3 +346,39 @@ def test_even_shards():
     with pytest.raises(ValueError):  # an empty shard
         even_shards(16, 3, 8)
     assert even_shards(24, 3, 8) == [0, 8, 16, 24]
+
+
+def test_no_alloc_limits_match_header_and_workspace_rule(abi):
+    """The fixed scratch of dspark_loss_fwd_noalloc: the header's constants are the
+    binding's, and which problems fit follows dspark_workspace_size alone."""
+    src = ('#include <stdio.h>\n#include "dspark.h"\n'
+           'int main(void) { printf("%d %d\\n", (int)DSPARK_NOALLOC_MAX_ROWS, (int)DSPARK_NOALLOC_BYTES); return 0; }\n')
+    with tempfile.TemporaryDirectory() as d:
+        with open(os.path.join(d, "n.c"), "w") as f:
+            f.write(src)
+        subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), os.path.join(d, "n.c"), "-o",
+                        os.path.join(d, "n")], check=True)
+        rows, nbytes = map(int, subprocess.run([os.path.join(d, "n")], check=True, capture_output=True,
+                                               text=True).stdout.split())
+    assert (rows, nbytes) == (abi.NOALLOC_MAX_ROWS, abi.NOALLOC_BYTES)
+    size = lambda p: abi.dspark_workspace_size(ctypes.byref(p))
+    # without heads every micro-batch up to the row limit fits
+    p = _problem(abi, V=151936)
+    p.B, p.N, p.K = 8, 64, 16
+    assert size(p) <= nbytes
+    # the Markov head and the teacher from hidden states never fit at a real vocabulary
+    assert size(_with_markov(abi, _problem(abi, V=151936), rank=256)) > nbytes
+    assert size(_with_lm_head(abi, _problem(abi, V=151936), Ht=4096)) > nbytes
+    # a confidence head with hidden size 4096: a few hundred rows fit, the 448-row recipe
+    # micro-batch does not
+    p = _with_conf_head(abi, _problem(abi, V=151936), H=4096)
+    p.B, p.N, p.K = 4, 16, 7
+    assert size(p) > nbytes
+    p.B, p.N, p.K = 2, 16, 7
+    assert size(p) <= nbytes
+    # more rows than the limit are refused before any CUDA call
+    p = _problem(abi)
+    p.B, p.N, p.K = 1, rows // 4 + 1, 4
+    out = abi.dspark_fwd_out_t()
+    assert abi.dspark_loss_fwd_noalloc(ctypes.byref(p), ctypes.byref(_params(abi)), ctypes.byref(out), None,
+                                       None) == abi.DSPARK_ERR_WORKSPACE
