@@ -7,8 +7,13 @@
 
 namespace dspark {
 
-// A bounded wait gives up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// A bounded wait gives up after this many nanoseconds of %globaltimer: 2 s unless the
+// build defines DSPARK_WAIT_LIMIT_NS (a test harness shortens it to a few milliseconds to
+// make a wait run out on purpose).
+#ifndef DSPARK_WAIT_LIMIT_NS
+#define DSPARK_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = DSPARK_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

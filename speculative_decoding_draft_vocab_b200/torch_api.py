@@ -196,6 +196,28 @@ def acceptance(l1_rows: torch.Tensor, eval_mask: torch.Tensor, block_keep: Optio
     return ap, tp, ar
 
 
+# ------------------------------------------------------- data-parallel reduction
+REPORT_VECTOR_LEN = 2 + 2 * abi.DSPARK_REP_COUNT
+
+
+def reduce_report(loss_num: torch.Tensor, num_tokens: torch.Tensor, report: torch.Tensor, group=None):
+    """Sum one micro-batch's forward outputs over the data-parallel ranks of ``group``:
+    the numerator, the supervised-token count and the report pairs, packed into one FP64
+    vector [loss_num, num_tokens, num_0, den_0, ..., num_5, den_5] and all-reduced (SUM)
+    in a single collective.  Nothing is divided: the caller forms each ratio once, from
+    the sums (the Megatron-Bridge API doc's Return contract).  Counts and denominators
+    are integers below 2^53, so their FP64 sums are exact.  Works on CUDA tensors over
+    NCCL and on CPU tensors over gloo; returns (loss_num [1] f64, num_tokens [1] i64,
+    report [DSPARK_REP_COUNT, 2] f64) on the inputs' device."""
+    import torch.distributed as dist
+    if report.numel() != 2 * abi.DSPARK_REP_COUNT:
+        raise ValueError(f"report must hold {2 * abi.DSPARK_REP_COUNT} values")
+    vec = torch.cat([loss_num.reshape(1).to(torch.float64), num_tokens.reshape(1).to(torch.float64),
+                     report.reshape(-1).to(torch.float64)])
+    dist.all_reduce(vec, op=dist.ReduceOp.SUM, group=group)
+    return vec[:1], vec[1:2].to(torch.int64), vec[2:].reshape(abi.DSPARK_REP_COUNT, 2)
+
+
 # ------------------------------------------------------- vocabulary-parallel path
 def even_shards(V: int, tp_size: int, align: int) -> list:
     """Bounds [0, v_1, ..., V] of tp_size contiguous vocabulary shards whose widths are

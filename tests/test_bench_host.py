@@ -83,3 +83,53 @@ def test_roofline_entry_bound_and_fractions():
     assert t["bound"] == "tensor" and t["unit"] == "TFLOP/s" and t["achieved"] == 1000.0
     assert t["frac"] == round(1000.0 / 1590.0, 4)
     assert "frac_of_nominal" not in t
+
+
+def test_oracle_pool_baseline_on_the_tiny_workload():
+    """The CPU baseline: whole blocks of the workload drawn on the CPU, the oracle run in
+    worker processes forked before any CUDA call, on one core and on every core."""
+    inp = bench.cpu_inputs("tiny")
+    pool = bench.OraclePool({"tiny": bench.oracle_view(inp)}, procs=2)
+    try:
+        res = bench.cpu_baseline(pool, "tiny", 0.05)
+        # one task over both blocks reproduces the whole micro-batch's supervised rows
+        rows, _ = pool.run([("tiny", 0, 2)])[0]
+    finally:
+        pool.close()
+    assert rows == int(inp.eval_mask.sum())
+    assert res["one_core"]["cores"] == 1 and res["all_cores"]["cores"] == 2
+    assert res["one_core"]["value"] > 0 and res["all_cores"]["value"] > 0
+
+
+def test_block_ranges_wrap_and_stay_in_bounds():
+    r = bench._block_ranges(5, 8, 3, 4)
+    assert r == [(5, 8), (0, 3), (3, 6), (6, 8)]
+    assert all(0 <= a < b <= 8 for a, b in r)
+
+
+def test_gpus_flag_starts_one_process_per_gpu(monkeypatch):
+    """Without a launcher, --gpus N re-runs the script under torch.distributed.run with N
+    processes on 127.0.0.1; under a launcher the world size must match --gpus."""
+    seen = {}
+
+    class FakeProc:
+        pid = 0
+
+        def __init__(self, cmd, env=None, start_new_session=False):
+            seen["cmd"], seen["env"] = cmd, env
+
+        def wait(self, timeout=None):
+            return 0
+
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench.subprocess, "Popen", FakeProc)
+    assert bench.main(["--gpus", "4", "--steps", "5", "--warmup", "3"]) == 0
+    cmd = seen["cmd"]
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd and cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-6:] == ["--gpus", "4", "--steps", "5", "--warmup", "3"]
+    assert seen["env"]["NCCL_DEBUG"]
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    import pytest
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "4"])
