@@ -179,6 +179,7 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
     }
     fence_mbar_init();
   }
+  __syncwarp();  // warp 0 is whole again (thread 0 set the barriers up) for the aligned alloc
   if (warp == 0) tm_alloc(smem_u32(&ctrl->tmem_base), TCOLS);
   tm_fence_before();
   __syncthreads();
@@ -227,8 +228,10 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
       // a wait ran out above): the latest use of each slot, each wait bounded again
       for (int slot = 0; slot < S && slot < g; ++slot) {
         const int64_t last_use = (g - 1 - slot) / S;
-        if (!mbar_wait_bounded(smem_u32(&ctrl->full[slot]), uint32_t(last_use) & 1u))
+        if (!mbar_wait_bounded(smem_u32(&ctrl->full[slot]), uint32_t(last_use) & 1u)) {
           atomicOr(&hdr->status, kFlagTimeout);
+          break;
+        }
       }
     }
     __syncwarp();
@@ -326,6 +329,7 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
 #pragma unroll
             for (int e = 0; e < EPV; ++e) et[e] = 0.f;
           }
+          __syncwarp();  // the TMEM store is warp-collective
           tm_st8(taddr(par, i * EPV), et);
           __syncwarp();
           if (lane == 0) mbar_arrive_local(smem_u32(&ctrl->empty[slot]));
@@ -375,12 +379,14 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
           const float k0 = cce - cl1 * S_;
           const int tv = ptok / EPV - v0, te = ptok % EPV;
           uint8_t* out = static_cast<uint8_t*>(a.dlogits) + (size_t(prow) * a.ld_g + size_t(v0) * EPV) * 2;
+          __syncwarp();  // TMEM accesses are warp-collective
           tm_wait_st();  // u of row j-1 (stored in its pass 2) is in TMEM
           uint32_t rb[2][EPV];
           tm_ld8(taddr(pp, 0), rb[0]);
 #pragma unroll
           for (int i = 0; i < NV; ++i) {
             uint32_t* r = rb[i & 1];
+            __syncwarp();
             tm_wait_ld8(r);
             if (i + 1 < NV) tm_ld8(taddr(pp, (i + 1) * EPV), rb[(i + 1) & 1]);  // in flight meanwhile
             const int v = tid + i * NTC;
@@ -439,6 +445,7 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
       const float az = hz ? ex2(oz - lz2) : 0.f;  // p = e * az
       const float at = ht ? ex2(ot - lt2) : 0.f;  // q = e * at
       float l4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
+      __syncwarp();  // TMEM accesses are warp-collective
       tm_wait_st();  // this row's teacher exponentials are in TMEM
       uint32_t rb[2][EPV];
       tm_ld8(taddr(par, 0), rb[0]);
@@ -478,6 +485,7 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
     }
     // what is left of this cluster's zero rows (all of them if it had no row)
     if (bwd) write_zeros(my_n * zslice, ztot);
+    __syncwarp();
     tm_wait_st();
   }
 
