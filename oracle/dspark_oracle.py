@@ -320,7 +320,12 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
     valid dz_j where sign(p_j - q_j) is undecided, 0 elsewhere), per-row sums over
     every supervised row ``dz_norm2`` [R] (sum_j dlogits_j^2) and ``swing_sum`` [R],
     ``dconf`` [R], and for the heads ``dW2``,
-    ``dE`` (row -> dL/de), ``dW1`` (id -> row), ``dconf_w``, ``dconf_b``, ``dhidden``.
+    ``dE`` (row -> dL/de), ``dW1`` (id -> row), ``dconf_w``, ``dconf_b``, ``dhidden``,
+    plus the sums a tolerance on the weight gradients needs, over every row the Markov
+    contractions take (so no caller has to keep every row's dlogits):
+    ``tol_dW2_rss2`` = sum_r dz_r^2 (x) e_r^2 and ``tol_dW2_swing`` = sum_r swing_r (x) |e_r|
+    ([V, rank]), and per row ``tol_dE_rss2`` = (dz_r^2) . (W2^2) and ``tol_dE_swing`` =
+    swing_r . |W2| ([rank]); swing_r is the ``dlogit_swing`` row.
 
     The loss is sum_r w_r (ce_alpha*CE_r + l1_alpha*L1_r + conf_alpha*BCE_r) where
     the BCE term exists only with a confidence source, and the L1 and BCE terms need
@@ -369,6 +374,12 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
     dlogits, amb, swing, dE = {}, {}, {}, {}
     dz_norm2, swing_sum = np.zeros(R), np.zeros(R)
     dW2 = np.zeros_like(w2) if (has_markov and want_grads) else None
+    # tolerance helpers of the head weight gradients (sums over every row the contractions
+    # take, so no caller needs every row's dlogits): sum_r dz_r^2 (x) e_r^2 and
+    # sum_r swing_r (x) |e_r| for dW2; per row (dz_r^2) . (W2^2) and swing_r . |W2| for dE
+    tol_dw2_rss2 = np.zeros_like(w2) if dW2 is not None else None
+    tol_dw2_swing = np.zeros_like(w2) if dW2 is not None else None
+    tol_de_rss2, tol_de_swing = {}, {}
 
     for c0 in range(0, len(sup), row_chunk):
         rr = sup[c0:c0 + row_chunk]
@@ -404,9 +415,10 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
             if has_markov and not markov_live and invalid_row_mode == 0:
                 row_grad = np.zeros(V)             # the corrected row is the constant 0
             dz_norm2[r] = float(np.dot(row_grad, row_grad))
+            sw_row = np.zeros(V)
             if rt["q"] is not None and row_grad is dz:
-                swing_sum[r] = float(np.sum(np.where(sign_ambiguity(rt["p"], rt["q"]),
-                                                     2.0 * grad_scale * w_r[r] * l1_alpha * rt["p"], 0.0)))
+                sw_row = np.where(sign_ambiguity(rt["p"], rt["q"]), 2.0 * grad_scale * w_r[r] * l1_alpha * rt["p"], 0.0)
+                swing_sum[r] = float(np.sum(sw_row))
             if r in keep:
                 dlogits[r] = row_grad
                 amb[r] = (sign_ambiguity(rt["p"], rt["q"]) if rt["q"] is not None
@@ -416,14 +428,20 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
                 swing[r] = (np.where(amb[r], 2.0 * grad_scale * w_r[r] * l1_alpha * rt["p"], 0.0)
                             if row_grad is dz else np.zeros(V))
             if markov_live:
-                dz_live.append((r, dz))
+                dz_live.append((r, dz, sw_row))
         if dz_live:
-            Dz = np.stack([d for _, d in dz_live])              # [n, V]
-            Er = e_all[[r for r, _ in dz_live]]                 # [n, rank]
+            Dz = np.stack([d for _, d, _ in dz_live])           # [n, V]
+            Sw = np.stack([x for _, _, x in dz_live])           # [n, V]
+            Er = e_all[[r for r, _, _ in dz_live]]              # [n, rank]
             dW2 += Dz.T @ Er                                     # dW2 = sum_r dz_r (x) e_r
             dEr = Dz @ w2                                        # dE_r = W2^T dz_r
-            for j, (r, _) in enumerate(dz_live):
+            tol_dw2_rss2 += (Dz ** 2).T @ (Er ** 2)
+            tol_dw2_swing += Sw.T @ np.abs(Er)
+            de_rss2 = (Dz ** 2) @ (w2 ** 2)
+            de_swing = Sw @ np.abs(w2)
+            for j, (r, _, _) in enumerate(dz_live):
                 dE[r] = dEr[j]
+                tol_de_rss2[r], tol_de_swing[r] = de_rss2[j], de_swing[j]
 
     # confidence / BCE
     y = acceptance_label(l1) if fixed_label is None else np.asarray(fixed_label, dtype=np.float64).reshape(R)
@@ -471,5 +489,6 @@ def dspark_loss(draft_logits, target_ids, eval_mask, *, target_logits=None, bloc
         pids = np.asarray(prev_ids, dtype=np.int64).reshape(R)
         for r in sorted(dE):
             dW1[int(pids[r])] = dW1.get(int(pids[r]), 0.0) + dE[r]
-        res.update(dW2=dW2, dE=dE, dW1=dW1)
+        res.update(dW2=dW2, dE=dE, dW1=dW1, tol_dW2_rss2=tol_dw2_rss2, tol_dW2_swing=tol_dw2_swing,
+                   tol_dE_rss2=tol_de_rss2, tol_dE_swing=tol_de_swing)
     return res

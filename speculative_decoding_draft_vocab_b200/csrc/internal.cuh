@@ -274,10 +274,10 @@ enum : int {
 };
 // False if V exceeds every build of that kind.
 bool sweep_supported(int kind, int64_t V, bool has_target);
-// The bf16 sweep with a teacher whose exponentials are held in TMEM (sweep_tm.cu):
-// false if V exceeds its builds.
-bool sweep_tm_supported(int64_t V);
-cudaError_t launch_sweep_tm(const SweepArgs& a, cudaStream_t s);
+// The sweep with a teacher whose exponentials are held in TMEM (sweep_tm.cu), for the
+// bf16 kinds with a teacher: false if the kind has no such build or V exceeds its builds.
+bool sweep_tm_supported(int kind, int64_t V);
+cudaError_t launch_sweep_tm(int kind, const SweepArgs& a, cudaStream_t s);
 cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s);
 cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
                               const uint8_t* eval_mask, const uint8_t* block_keep,

@@ -138,9 +138,16 @@ struct CtrlTm {
   int last;
 };
 
-template <int CL, int NWC, int NV>
+// TT: the teacher rows' type (bf16 logits, or FP32 rows of the teacher computed from
+// hidden states, compact by supervised position); HAS_B: the Markov head's FP32 bias rows
+// (compact by supervised position) are added to the base rows on chip, z = keep*base +
+// bias, keep = 0 only on an invalid slot whose corrected row is all zero.
+template <typename TT, bool HAS_B, int CL, int NWC, int NV>
 __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const int S) {
-  constexpr int EPV = 8;              // bf16 logits per 16-byte vector
+  constexpr int EPV = 8;              // logits per 16-byte bf16 vector
+  constexpr int BB = HAS_B ? 32 : 0;  // bytes of a vector's bias values
+  constexpr int TB = EPV * int(sizeof(TT));  // bytes of a vector's teacher values
+  constexpr bool kT32 = sizeof(TT) == 4;
   constexpr int NTC = NWC * 32;       // compute threads
   constexpr int NE = NV * EPV;        // logits per compute thread
   constexpr int NP = CL * NWC;
@@ -154,7 +161,10 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
   const uint32_t rank = cluster_ctarank();
   const uint32_t cid = cluster_id_x();
   const uint32_t G = nclusters_x();
-  const uint32_t slab_bytes = uint32_t(NTC) * 32u;  // draft + teacher vectors
+  // slab: NTC draft vectors, NTC bias vectors (HAS_B), NTC teacher vectors
+  const uint32_t slab_bytes = uint32_t(NTC) * uint32_t(16 + BB + TB);
+  constexpr uint32_t kOffB = uint32_t(NTC) * 16u;
+  constexpr uint32_t kOffT = uint32_t(NTC) * uint32_t(16 + BB);
   CtrlT* ctrl = reinterpret_cast<CtrlT*>(smem + size_t(S) * slab_bytes);
   WsHeader* hdr = a.ws.hdr;
   const int v0 = int(rank) * a.seg_vec;
@@ -206,21 +216,26 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
         ctrl->rrow[j % kRowRing] = row;
         ctrl->rtok[j % kRowRing] = a.ws.sup_tok[si];
         ctrl->rw[j % kRowRing] = a.ws.sup_w[si];
+        // the teacher chunk's rows are compact by supervised position
+        const int64_t trow = (kT32 && a.target_compact) ? si - a.row0 : row;
         const uint8_t* zr = draft + (size_t(row) * a.ld_d + size_t(v0) * EPV) * 2;
-        const uint8_t* tr = target + (size_t(row) * a.ld_t + size_t(v0) * EPV) * 2;
+        const uint8_t* br = HAS_B ? reinterpret_cast<const uint8_t*>(a.bias + size_t(si) * a.ld_b + size_t(v0) * EPV)
+                                  : nullptr;
+        const uint8_t* tr = target + (size_t(trow) * a.ld_t + size_t(v0) * EPV) * sizeof(TT);
         for (int i = 0; i < NV; ++i, ++g) {
           const int slot = int(g % S);
           const uint32_t use = uint32_t(g / S);
           if (use > 0) wait(smem_u32(&ctrl->empty[slot]), (use - 1) & 1u);
           const int nv_i = max(0, min(NTC, nvec - i * NTC));
-          const uint32_t bytes = uint32_t(nv_i) * 16u;
           const uint32_t full = smem_u32(&ctrl->full[slot]);
           // the arrive releases the row scalars written above to the compute warps
-          mbar_arrive_expect_tx(full, 2 * bytes);
-          if (bytes) {
+          mbar_arrive_expect_tx(full, uint32_t(nv_i) * uint32_t(16 + BB + TB));
+          if (nv_i) {
             const uint32_t dst = smem_u32(smem + size_t(slot) * slab_bytes);
-            bulk_g2s(dst, zr + size_t(i) * NTC * 16, bytes, full, policy);
-            bulk_g2s(dst + uint32_t(NTC) * 16u, tr + size_t(i) * NTC * 16, bytes, full, policy);
+            bulk_g2s(dst, zr + size_t(i) * NTC * 16, uint32_t(nv_i) * 16u, full, policy);
+            if constexpr (HAS_B)
+              bulk_g2s(dst + kOffB, br + size_t(i) * NTC * BB, uint32_t(nv_i) * uint32_t(BB), full, policy);
+            bulk_g2s(dst + kOffT, tr + size_t(i) * NTC * TB, uint32_t(nv_i) * uint32_t(TB), full, policy);
           }
         }
       }
@@ -270,24 +285,46 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
       int32_t tok = 0;
       if (cur) {
         const int64_t g0 = g;
-        uint32_t tmax2 = 0xff80ff80u;  // two bf16 -inf
+        uint32_t tmax2 = 0xff80ff80u;  // two bf16 -inf (bf16 teacher)
+        float mt32 = -INFINITY;        // FP32 teacher
         float mz = -INFINITY;
+        float keep = 1.f;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
           const int slot = int((g0 + i) % S);
           wait(smem_u32(&ctrl->full[slot]), uint32_t((g0 + i) / S) & 1u);
-          if (i == 0) tok = ctrl->rtok[j % kRowRing] & 0x7fffffff;
+          if (i == 0) {
+            const int32_t tokf = ctrl->rtok[j % kRowRing];
+            tok = tokf & 0x7fffffff;
+            if (HAS_B && tokf < 0) keep = 0.f;  // the corrected row is all zero
+          }
           const int v = tid + i * NTC;
           const uint8_t* sb = smem + size_t(slot) * slab_bytes;
           if (v < nvec) {
             const uint4 qz = *reinterpret_cast<const uint4*>(sb + size_t(tid) * 16);
-            const uint4 qt = *reinterpret_cast<const uint4*>(sb + size_t(NTC + tid) * 16);
             float x[EPV];
             x[0] = bf16lo(qz.x); x[1] = bf16hi(qz.x); x[2] = bf16lo(qz.y); x[3] = bf16hi(qz.y);
             x[4] = bf16lo(qz.z); x[5] = bf16hi(qz.z); x[6] = bf16lo(qz.w); x[7] = bf16hi(qz.w);
+            if constexpr (HAS_B) {  // z = keep * base + bias
+              const uint4 b0 = *reinterpret_cast<const uint4*>(sb + kOffB + size_t(tid) * 32);
+              const uint4 b1 = *reinterpret_cast<const uint4*>(sb + kOffB + size_t(tid) * 32 + 16);
+              x[0] = fmaf(x[0], keep, __uint_as_float(b0.x)); x[1] = fmaf(x[1], keep, __uint_as_float(b0.y));
+              x[2] = fmaf(x[2], keep, __uint_as_float(b0.z)); x[3] = fmaf(x[3], keep, __uint_as_float(b0.w));
+              x[4] = fmaf(x[4], keep, __uint_as_float(b1.x)); x[5] = fmaf(x[5], keep, __uint_as_float(b1.y));
+              x[6] = fmaf(x[6], keep, __uint_as_float(b1.z)); x[7] = fmaf(x[7], keep, __uint_as_float(b1.w));
+            }
             mz = fmax3(mz, fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]));
             mz = fmax3(mz, x[6], x[7]);
-            tmax2 = bf2max(bf2max(tmax2, bf2max(qt.x, qt.y)), bf2max(qt.z, qt.w));
+            if constexpr (kT32) {
+              const uint4 t0 = *reinterpret_cast<const uint4*>(sb + kOffT + size_t(tid) * 32);
+              const uint4 t1 = *reinterpret_cast<const uint4*>(sb + kOffT + size_t(tid) * 32 + 16);
+              mt32 = fmax3(mt32, fmax3(__uint_as_float(t0.x), __uint_as_float(t0.y), __uint_as_float(t0.z)),
+                           fmax3(__uint_as_float(t0.w), __uint_as_float(t1.x), __uint_as_float(t1.y)));
+              mt32 = fmax3(mt32, __uint_as_float(t1.z), __uint_as_float(t1.w));
+            } else {
+              const uint4 qt = *reinterpret_cast<const uint4*>(sb + kOffT + size_t(tid) * 16);
+              tmax2 = bf2max(bf2max(tmax2, bf2max(qt.x, qt.y)), bf2max(qt.z, qt.w));
+            }
             const bool own = v == tok / EPV - v0;
             const int te = tok % EPV;
 #pragma unroll
@@ -300,7 +337,7 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
             for (int e = 0; e < EPV; ++e) xz[i * EPV + e] = -INFINITY;
           }
         }
-        const float mt = fmaxf(bf16lo(tmax2), bf16hi(tmax2));
+        const float mt = kT32 ? mt32 : fmaxf(bf16lo(tmax2), bf16hi(tmax2));
         hz = mz != -INFINITY;
         ht = mt != -INFINITY;
         oz = hz ? mz * kLog2e : 0.f;
@@ -317,9 +354,18 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
           const int v = tid + i * NTC;
           float et[EPV];
           if (v < nvec) {
-            const uint4 qt = *reinterpret_cast<const uint4*>(smem + size_t(slot) * slab_bytes + size_t(NTC + tid) * 16);
-            et[0] = bf16lo(qt.x); et[1] = bf16hi(qt.x); et[2] = bf16lo(qt.y); et[3] = bf16hi(qt.y);
-            et[4] = bf16lo(qt.z); et[5] = bf16hi(qt.z); et[6] = bf16lo(qt.w); et[7] = bf16hi(qt.w);
+            const uint8_t* tp = smem + size_t(slot) * slab_bytes + kOffT + size_t(tid) * TB;
+            if constexpr (kT32) {
+              const uint4 t0 = *reinterpret_cast<const uint4*>(tp);
+              const uint4 t1 = *reinterpret_cast<const uint4*>(tp + 16);
+              et[0] = __uint_as_float(t0.x); et[1] = __uint_as_float(t0.y); et[2] = __uint_as_float(t0.z);
+              et[3] = __uint_as_float(t0.w); et[4] = __uint_as_float(t1.x); et[5] = __uint_as_float(t1.y);
+              et[6] = __uint_as_float(t1.z); et[7] = __uint_as_float(t1.w);
+            } else {
+              const uint4 qt = *reinterpret_cast<const uint4*>(tp);
+              et[0] = bf16lo(qt.x); et[1] = bf16hi(qt.x); et[2] = bf16lo(qt.y); et[3] = bf16hi(qt.y);
+              et[4] = bf16lo(qt.z); et[5] = bf16hi(qt.z); et[6] = bf16lo(qt.w); et[7] = bf16hi(qt.w);
+            }
 #pragma unroll
             for (int e = 0; e < EPV; ++e) {
               et[e] = ex2(fmaf(et[e], kLog2e, -ot));
@@ -373,8 +419,10 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
           st_row[kStS] = S_;
         }
         if (bwd) {
-          const int32_t ptok = ctrl->rtok[jr] & 0x7fffffff;
-          const float gw = g_scale * ctrl->rw[jr];
+          const int32_t ptokf = ctrl->rtok[jr];
+          const int32_t ptok = ptokf & 0x7fffffff;
+          // an invalid Markov slot's corrected row is a constant: nothing flows to the base
+          const float gw = (HAS_B && ptokf < 0) ? 0.f : g_scale * ctrl->rw[jr];
           const float cce = gw * a.ce_alpha, cl1 = gw * a.l1_alpha;
           const float k0 = cce - cl1 * S_;
           const int tv = ptok / EPV - v0, te = ptok % EPV;
@@ -523,13 +571,13 @@ struct TmCache {
   int clusters = 0;
 };
 
-template <int CL, int NWC, int NV>
+template <typename TT, bool HAS_B, int CL, int NWC, int NV>
 cudaError_t launch_tm(const SweepArgs& a0, cudaStream_t s) {
   constexpr int NTC = NWC * 32, NT = NTC + 32;
   SweepArgs a = a0;
   a.vvec = int32_t(a.V / 8);
   a.seg_vec = (a.vvec + CL - 1) / CL;
-  const size_t slab = size_t(NTC) * 32;
+  const size_t slab = size_t(NTC) * (16 + (HAS_B ? 32 : 0) + 8 * sizeof(TT));
   const int S = int(std::min<size_t>(kMaxSlabs, kRingBudget / slab));
   if (S < NV) return cudaErrorInvalidValue;
   const size_t ctrl = sizeof(CtrlTm<CL * NWC>);
@@ -537,7 +585,7 @@ cudaError_t launch_tm(const SweepArgs& a0, cudaStream_t s) {
   smem = std::max(smem, size_t(NT / 32) * kNAcc * sizeof(double));
   smem = std::max(smem, kOneCtaPerSm);
   if (smem > kMaxSmemTm) return cudaErrorInvalidValue;
-  auto kern = sweep_tm_kernel<CL, NWC, NV>;
+  auto kern = sweep_tm_kernel<TT, HAS_B, CL, NWC, NV>;
   static TmCache cache;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -553,6 +601,10 @@ cudaError_t launch_tm(const SweepArgs& a0, cudaStream_t s) {
     if (cache.dev != dev || cache.smem != smem) {
       err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxSmemTm));
       if (err != cudaSuccess) return err;
+      if (CL > 8) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (err != cudaSuccess) return err;
+      }
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(CL, 1, 1);
       q.blockDim = dim3(NT, 1, 1);
@@ -573,7 +625,7 @@ cudaError_t launch_tm(const SweepArgs& a0, cudaStream_t s) {
     }
     clusters = cache.clusters;
   }
-  // programmatic dependent launch: scheduled while the prologue runs, waits for it
+  // programmatic dependent launch: scheduled while the kernel before it runs, waits for it
   at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
@@ -590,26 +642,47 @@ cudaError_t launch_tm(const SweepArgs& a0, cudaStream_t s) {
 struct TmBuild {
   int cl, nwc, nv;
 };
-constexpr TmBuild kTmBuilds[] = {{1, 4, 1}, {2, 8, 2}, {4, 16, 2}, {8, 16, 3}, {8, 16, 5}};
-constexpr int kNumTmBuilds = int(sizeof(kTmBuilds) / sizeof(kTmBuilds[0]));
+constexpr int kNumTmBuilds = 5;
+// bf16 draft and teacher: 32 bytes per vector in the ring
+constexpr TmBuild kTmBuilds[kNumTmBuilds] = {{1, 4, 1}, {2, 8, 2}, {4, 16, 2}, {8, 16, 3}, {8, 16, 5}};
+// with bias rows and/or an FP32 teacher (48 to 80 bytes per vector): the largest rows over
+// 16-CTA clusters of 8 compute warps, so that the ring still holds more than a row
+constexpr TmBuild kTmHeadBuilds[kNumTmBuilds] = {{1, 4, 1}, {2, 8, 2}, {4, 16, 2}, {8, 16, 3}, {16, 8, 5}};
 
-int pick_tm(int64_t V) {
+int pick_tm(int kind, int64_t V) {
+  const TmBuild* b = kind == kSweepBf16 ? kTmBuilds : kTmHeadBuilds;
   for (int i = 0; i < kNumTmBuilds; ++i)
-    if (int64_t(kTmBuilds[i].cl) * kTmBuilds[i].nwc * 32 * kTmBuilds[i].nv * 8 >= V) return i;
+    if (int64_t(b[i].cl) * b[i].nwc * 32 * b[i].nv * 8 >= V) return i;
   return -1;
+}
+
+template <typename TT, bool HB>
+cudaError_t dispatch_tm(int i, bool heads_table, const SweepArgs& a, cudaStream_t s) {
+  switch (i) {
+    case 0: return launch_tm<TT, HB, 1, 4, 1>(a, s);
+    case 1: return launch_tm<TT, HB, 2, 8, 2>(a, s);
+    case 2: return launch_tm<TT, HB, 4, 16, 2>(a, s);
+    case 3: return launch_tm<TT, HB, 8, 16, 3>(a, s);
+    case 4: return heads_table ? launch_tm<TT, HB, 16, 8, 5>(a, s) : launch_tm<TT, HB, 8, 16, 5>(a, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool sweep_tm_supported(int64_t V) { return pick_tm(V) >= 0; }
+bool sweep_tm_supported(int kind, int64_t V) {
+  return (kind == kSweepBf16 || kind == kSweepZ32 || kind == kSweepT32 || kind == kSweepZT32) &&
+         pick_tm(kind, V) >= 0;
+}
 
-cudaError_t launch_sweep_tm(const SweepArgs& a, cudaStream_t s) {
-  switch (pick_tm(a.V)) {
-    case 0: return launch_tm<1, 4, 1>(a, s);
-    case 1: return launch_tm<2, 8, 2>(a, s);
-    case 2: return launch_tm<4, 16, 2>(a, s);
-    case 3: return launch_tm<8, 16, 3>(a, s);
-    case 4: return launch_tm<8, 16, 5>(a, s);
+cudaError_t launch_sweep_tm(int kind, const SweepArgs& a, cudaStream_t s) {
+  const int i = pick_tm(kind, a.V);
+  if (i < 0) return cudaErrorInvalidValue;
+  switch (kind) {
+    case kSweepBf16: return dispatch_tm<__nv_bfloat16, false>(i, false, a, s);
+    case kSweepZ32: return dispatch_tm<__nv_bfloat16, true>(i, true, a, s);
+    case kSweepT32: return dispatch_tm<float, false>(i, true, a, s);
+    case kSweepZT32: return dispatch_tm<float, true>(i, true, a, s);
   }
   return cudaErrorInvalidValue;
 }

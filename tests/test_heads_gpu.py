@@ -130,9 +130,12 @@ def test_recipe_heads_visible_correction():
 
 def test_large_config():
     """8 x 64 x 16 rows (8192), V = 151936, heads on, ragged prefixes with empty blocks.
-    The oracle runs on every row (report, per-row terms, dL/dc, every weight
-    gradient); dlogits are compared on 256 sampled supervised rows plus every row of
-    the first four blocks, and every unsupervised row must be exactly zero."""
+    The oracle runs on every row (report, per-row terms, dL/dc, every weight gradient,
+    dW2 and dW1 checked element-wise); dlogits are compared on every row of 64 whole
+    blocks drawn at random and on 1024 more supervised rows drawn at random (the oracle
+    run a chunk of rows at a time: rows are independent), and every unsupervised row must
+    be exactly zero."""
+    from tests.parity_util import check_dlogit_row
     inp = make_inputs("large", device="cuda")
     call = _call(inp, 0)
     call.launch()
@@ -141,9 +144,21 @@ def test_large_config():
     m = O.prefix_supervision_mask(np32(inp.eval_mask), np32(inp.block_keep)).reshape(-1)
     sup = np.nonzero(m)[0]
     rng = np.random.default_rng(5)
-    sample = sorted(set(rng.choice(sup, size=min(256, len(sup)), replace=False).tolist())
-                    | {int(r) for r in sup if r < 4 * inp.K})
-    ref = oracle_run(inp, keep_rows=sample)
+    blocks = rng.choice(inp.B * inp.N, size=64, replace=False)
+    in_blocks = {int(b) * inp.K + k for b in blocks for k in range(inp.K)}
+    extra = set(rng.choice(sup, size=min(1024, len(sup)), replace=False).tolist())
+    rows = sorted(r for r in (in_blocks | extra) if m[r])
+    ref = oracle_run(inp, keep_rows=rows[:64])
     compare(inp, call, ref)
-    check_heads(inp, call, ref, 0, elementwise=False)
+    check_heads(inp, call, ref, 0, elementwise=True)
+    g = call.out.dlogits.view(inp.R, inp.V)
+    for c0 in range(64, len(rows), 128):
+        chunk = rows[c0:c0 + 128]
+        part = oracle_run(inp, rows=np.array(chunk), keep_rows=chunk)
+        for r in chunk:
+            check_dlogit_row(g[r].float().cpu().double().numpy(), part["dlogits"][r], part["sign_amb"][r],
+                             inp.dtype, tag=f"row {r}")
+    unsup_in_blocks = [r for r in in_blocks if not m[r]]
+    if unsup_in_blocks:
+        assert bool((g[torch.tensor(unsup_in_blocks, device=g.device)] == 0).all())
     assert ref["report"]["tau"][1] < inp.B * inp.N  # some blocks are empty

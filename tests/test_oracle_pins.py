@@ -593,3 +593,41 @@ def test_subgradient_swing_on_ties_and_none_elsewhere():
     res = O.dspark_loss(d, ids, ev, target_logits=t)
     assert all(not sw.any() for sw in res["dlogit_swing"].values())
     assert np.all(res["swing_sum"] == 0.0)
+
+
+def test_weight_gradient_tolerance_sums_equal_their_definitions():
+    """The sums the weight-gradient tolerances are built from, written out per element from
+    the rows' own dlogits, swings and embeddings: sum over the Markov-live rows of
+    dz^2 (x) e^2 and swing (x) |e| for dW2, and per row (dz^2) . W2^2 and swing . |W2| for dE.
+    Rows tie on purpose (the teacher equals the draft on one block) so the swing terms
+    are not all zero."""
+    rng = np.random.default_rng(31)
+    B, N, K, V, r = 1, 2, 3, 11, 4
+    d, t, ids, ev = _rand_problem(rng, B, N, K, V, scale=1.5)
+    prev = rng.integers(1, 6, ids.shape)
+    valid = np.array([[[1, 0, 1], [1, 1, 1]]])
+    w1, w2 = rng.normal(0, 0.4, (6, r)), rng.normal(0, 0.4, (V, r))
+    # block 0: a zero embedding (no bias) and a teacher equal to the draft, so every sign
+    # there is undecided
+    w1[0] = 0.0
+    prev[0, 0] = 0
+    t[0, 0] = d[0, 0]
+    res = O.dspark_loss(d, ids, ev, target_logits=t, prev_ids=prev, valid=valid, markov_w1=w1, markov_w2=w2,
+                        grad_scale=0.8, gamma=4.0)
+    live = [int(x) for x in res["rows"] if valid.reshape(-1)[int(x)]]
+    assert live and any(res["dlogit_swing"][x].any() for x in live)
+    rss2 = np.zeros((V, r))
+    swing = np.zeros((V, r))
+    for x in live:
+        e = w1[prev.reshape(-1)[x]]
+        for j in range(V):
+            for c in range(r):
+                rss2[j, c] += res["dlogits"][x][j] ** 2 * e[c] ** 2
+                swing[j, c] += res["dlogit_swing"][x][j] * abs(e[c])
+        de_rss2 = [sum(res["dlogits"][x][j] ** 2 * w2[j, c] ** 2 for j in range(V)) for c in range(r)]
+        de_swing = [sum(res["dlogit_swing"][x][j] * abs(w2[j, c]) for j in range(V)) for c in range(r)]
+        np.testing.assert_allclose(res["tol_dE_rss2"][x], de_rss2, rtol=1e-12, atol=1e-300)
+        np.testing.assert_allclose(res["tol_dE_swing"][x], de_swing, rtol=1e-12, atol=1e-300)
+    assert set(res["tol_dE_rss2"]) == set(live)
+    np.testing.assert_allclose(res["tol_dW2_rss2"], rss2, rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(res["tol_dW2_swing"], swing, rtol=1e-12, atol=1e-300)
