@@ -337,6 +337,12 @@ DSPARK_API dspark_status_t dspark_check_status(const void* ws, dspark_stream_t s
 /* Static English text for a status code. */
 DSPARK_API const char* dspark_status_string(dspark_status_t status);
 
+/* Name of the CUDA runtime error behind the most recent DSPARK_ERR_CUDA returned by any
+ * call of this library in the process ("cudaSuccess" if there was none).  A library
+ * service with no counterpart on the source pages: it tells the caller which CUDA call
+ * failed without a debugger.  Static storage; never NULL. */
+DSPARK_API const char* dspark_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -123,6 +123,8 @@ lib.dspark_check_status.argtypes = [c_vp, c_vp]
 lib.dspark_check_status.restype = ctypes.c_int
 lib.dspark_status_string.argtypes = [ctypes.c_int]
 lib.dspark_status_string.restype = ctypes.c_char_p
+lib.dspark_last_cuda_error.argtypes = []
+lib.dspark_last_cuda_error.restype = ctypes.c_char_p
 
 # The C entry points under their own names.
 dspark_workspace_size = lib.dspark_workspace_size
@@ -140,12 +142,14 @@ dspark_tp_finish = lib.dspark_tp_finish
 dspark_tp_heads_bwd = lib.dspark_tp_heads_bwd
 dspark_check_status = lib.dspark_check_status
 dspark_status_string = lib.dspark_status_string
+dspark_last_cuda_error = lib.dspark_last_cuda_error
 
 
 class DSparkError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {dspark_status_string(status).decode()} (status {status})")
+        detail = f", {dspark_last_cuda_error().decode()}" if status == DSPARK_ERR_CUDA else ""
+        super().__init__(f"{where}: {dspark_status_string(status).decode()} (status {status}{detail})")
 
 
 def check(status: int, where: str) -> None:

@@ -2,6 +2,7 @@
 // launch sequence of each entry point.  No allocation, no synchronisation (except
 // dspark_check_status, whose job it is).
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -121,7 +122,14 @@ dspark_status_t check_problem(const dspark_problem_t* p, const dspark_params_t* 
   return DSPARK_OK;
 }
 
-inline dspark_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+// The CUDA error behind the most recent DSPARK_ERR_CUDA of any call in this process.
+std::atomic<int> g_last_cuda_error{0};
+
+inline dspark_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DSPARK_OK;
+  g_last_cuda_error.store(int(e), std::memory_order_relaxed);
+  return DSPARK_ERR_CUDA;
+}
 
 dspark_status_t check_ws(const dspark_problem_t* p, const void* ws, size_t ws_bytes) {
   if (ws == nullptr) return DSPARK_ERR_WORKSPACE;
@@ -275,6 +283,10 @@ const char* dspark_status_string(dspark_status_t s) {
     case DSPARK_ERR_CUDA: return "CUDA runtime error";
   }
   return "unknown status";
+}
+
+const char* dspark_last_cuda_error(void) {
+  return cudaGetErrorName(static_cast<cudaError_t>(g_last_cuda_error.load(std::memory_order_relaxed)));
 }
 
 size_t dspark_workspace_size(const dspark_problem_t* prob) {
@@ -526,10 +538,11 @@ dspark_status_t dspark_tp_heads_bwd(const dspark_problem_t* prob, const dspark_p
 dspark_status_t dspark_check_status(const void* ws, dspark_stream_t stream) {
   if (ws == nullptr) return DSPARK_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
   uint32_t flags = 0;
-  if (cudaMemcpy(&flags, ws, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return DSPARK_ERR_CUDA;
+  e = cudaMemcpy(&flags, ws, sizeof(flags), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e);
   if (flags & kFlagIdOutOfRange) return DSPARK_ERR_ID_OUT_OF_RANGE;
   if (flags & kFlagTimeout) return DSPARK_ERR_DEVICE_TIMEOUT;
   return DSPARK_OK;

@@ -622,7 +622,9 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at2;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  err = cudaLaunchKernelEx(&cfg, kern, a);
+  if (err != cudaSuccess) cudaGetLastError();  // a refused launch leaves no error for later calls
+  return err;
 }
 
 // Builds, smallest first.  A build covers rows of up to CL * NT * NV * (elements per

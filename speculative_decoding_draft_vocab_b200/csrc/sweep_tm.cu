@@ -119,7 +119,11 @@ constexpr uint32_t pow2_cols(int n) {
 }
 
 constexpr int kMaxSlabs = 16;  // ring slots
-constexpr int kTmRegs = 120;   // registers per thread: 17 warps x 32 x 120 <= 65536
+// Registers per thread.  The register file is split over the SM's four schedulers
+// (16384 registers each) and a CTA's warps are dealt round-robin to them, so a build with
+// at most 13 warps (NWC <= 12 plus the producer) puts at most 4 warps on one scheduler:
+// 4 x 32 x 128 = 16384.
+constexpr int kTmRegs = 128;
 constexpr int kRowRing = 32;   // row scalars in flight (> kMaxSlabs + 3 rows)
 
 // Control block; NP = CL * NWC partials per exchange.
@@ -154,6 +158,7 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
   constexpr int COLS = (NWC / 4) * NE;  // TMEM columns of one row (per lane quarter)
   constexpr uint32_t TCOLS = pow2_cols(2 * COLS);
   static_assert(NWC % 4 == 0 && 2 * COLS <= 512, "TMEM layout");
+  static_assert(NWC + 1 <= 13, "at most 4 warps of kTmRegs registers per scheduler");
   using CtrlT = CtrlTm<NP>;
   extern __shared__ __align__(128) uint8_t smem[];
 
@@ -635,7 +640,9 @@ cudaError_t launch_tm(const SweepArgs& a0, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, a, S);
+  err = cudaLaunchKernelEx(&cfg, kern, a, S);
+  if (err != cudaSuccess) cudaGetLastError();  // a refused launch leaves no error for later calls
+  return err;
 }
 
 // Builds, smallest first: a build covers rows of up to CL * NWC * 32 * NV * 8 logits.
@@ -644,10 +651,10 @@ struct TmBuild {
 };
 constexpr int kNumTmBuilds = 5;
 // bf16 draft and teacher: 32 bytes per vector in the ring
-constexpr TmBuild kTmBuilds[kNumTmBuilds] = {{1, 4, 1}, {2, 8, 2}, {4, 16, 2}, {8, 16, 3}, {8, 16, 5}};
+constexpr TmBuild kTmBuilds[kNumTmBuilds] = {{1, 4, 1}, {2, 8, 2}, {4, 12, 3}, {8, 12, 4}, {8, 12, 7}};
 // with bias rows and/or an FP32 teacher (48 to 80 bytes per vector): the largest rows over
 // 16-CTA clusters of 8 compute warps, so that the ring still holds more than a row
-constexpr TmBuild kTmHeadBuilds[kNumTmBuilds] = {{1, 4, 1}, {2, 8, 2}, {4, 16, 2}, {8, 16, 3}, {16, 8, 5}};
+constexpr TmBuild kTmHeadBuilds[kNumTmBuilds] = {{1, 4, 1}, {2, 8, 2}, {4, 12, 3}, {8, 12, 4}, {16, 8, 5}};
 
 int pick_tm(int kind, int64_t V) {
   const TmBuild* b = kind == kSweepBf16 ? kTmBuilds : kTmHeadBuilds;
@@ -661,9 +668,9 @@ cudaError_t dispatch_tm(int i, bool heads_table, const SweepArgs& a, cudaStream_
   switch (i) {
     case 0: return launch_tm<TT, HB, 1, 4, 1>(a, s);
     case 1: return launch_tm<TT, HB, 2, 8, 2>(a, s);
-    case 2: return launch_tm<TT, HB, 4, 16, 2>(a, s);
-    case 3: return launch_tm<TT, HB, 8, 16, 3>(a, s);
-    case 4: return heads_table ? launch_tm<TT, HB, 16, 8, 5>(a, s) : launch_tm<TT, HB, 8, 16, 5>(a, s);
+    case 2: return launch_tm<TT, HB, 4, 12, 3>(a, s);
+    case 3: return launch_tm<TT, HB, 8, 12, 4>(a, s);
+    case 4: return heads_table ? launch_tm<TT, HB, 16, 8, 5>(a, s) : launch_tm<TT, HB, 8, 12, 7>(a, s);
   }
   return cudaErrorInvalidValue;
 }
