@@ -330,12 +330,13 @@ __global__ void __maxnreg__(kTmRegs) sweep_tm_kernel(const SweepArgs a, const in
               const uint4 qt = *reinterpret_cast<const uint4*>(sb + kOffT + size_t(tid) * 16);
               tmax2 = bf2max(bf2max(tmax2, bf2max(qt.x, qt.y)), bf2max(qt.z, qt.w));
             }
-            const bool own = v == tok / EPV - v0;
-            const int te = tok % EPV;
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) {
-              if (own && e == te) zt = x[e];
-              xz[i * EPV + e] = x[e];
+            for (int e = 0; e < EPV; ++e) xz[i * EPV + e] = x[e];
+            if (v == tok / EPV - v0) {  // one thread of the cluster holds the target id
+              const int te = tok % EPV;
+#pragma unroll
+              for (int e = 0; e < EPV; ++e)
+                if (e == te) zt = x[e];
             }
           } else {
 #pragma unroll
