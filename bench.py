@@ -65,6 +65,7 @@ KERNEL_SOURCES = ["speculative_decoding_draft_vocab_b200/csrc/sweep.cu",
 EXTRA_WORKLOADS = ("recipe_heads", "lm_head_teacher", "large")
 CPU_BASELINE_WORKLOADS = ("recipe", "large")
 WEIGHTS = ("markov_w1", "markov_w2", "conf_w", "conf_b", "lm_head", "target_norm_weight")  # resident
+HOST_SLACK_CYCLES = 200_000  # device spin before each timed call: about 100 us at 1965 MHz
 
 
 def workload_desc(name: str, inp) -> str:
@@ -452,6 +453,10 @@ def time_calls(call, steps: int, warmup: int, flush, clk_device: int):
         wall0 = time.perf_counter()
         for i in range(steps):
             flush.zero_()
+            # a spin of about 100 us on the device after the flush: the host enqueues the
+            # start event and the call meanwhile, so the device never waits for the host
+            # between the two events (host launch latency is not device time)
+            torch.cuda._sleep(HOST_SLACK_CYCLES)
             starts[i].record()
             call.launch()
             ends[i].record()
@@ -681,7 +686,8 @@ def main(argv=None):
                        "supervised_rows_all_ranks": int(rows_all), "rows_per_rank": inp.R,
                        "global_batch": inp.B * world, "parallelism": f"dp{world}",
                        "l2": "flushed before every timed call (512 MiB write, untimed)",
-                       "timing": "median per-call CUDA-event time, maximum over ranks",
+                       "timing": "median per-call CUDA-event time, maximum over ranks; a ~100 us device "
+                                 "spin after each flush keeps host launch latency out of the events",
                        "ms_mean": round(statistics.mean(per_step), 5)},
             "roofline": roofline,
             "cpu_baseline": cpu,
@@ -749,6 +755,7 @@ def run_tp(args, inp, torch_api):
     with ClockSampler(0) as clk:
         for i in range(args.steps):
             flush.zero_()
+            torch.cuda._sleep(HOST_SLACK_CYCLES)  # the host enqueues the step meanwhile
             starts[i].record()
             step()
             ends[i].record()

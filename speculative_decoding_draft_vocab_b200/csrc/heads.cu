@@ -35,12 +35,6 @@ __global__ void __launch_bounds__(256) heads_prep_kernel(const HeadsArgs a) {
     const int64_t pv = a.prev_ids ? a.prev_ids[r] : -1;
     const bool has_e = a.w1 != nullptr && valid && pv >= 0 && pv < a.Vt;
     float edot = 0.f;
-    if (a.w1 != nullptr && r >= a.ws.hdr->n_sup) {
-      // position r of the compact list holds no row: zeros (the dW2 GEMM contracts the
-      // compact embeddings over whole 64-position chunks)
-      uint16_t* dpos = a.ws.esup + size_t(r) * a.rank;
-      for (int j = lane * 8; j < a.rank; j += 256) *reinterpret_cast<uint4*>(dpos + j) = make_uint4(0u, 0u, 0u, 0u);
-    }
     if (a.w1 != nullptr) {
       const uint16_t* src = a.w1 + size_t(has_e ? pv : 0) * a.rank;
       uint16_t* dall = a.ws.eall + size_t(r) * a.rank;
@@ -114,18 +108,16 @@ struct WeightEpi {
 };
 
 // ---- dE = sum of the partials (+ dc proj_e), then dW1[prev] += dE.  The partials are
-// [splits][R][rank]: the K splits of the dE GEMM (rows indexed by supervised position), or
-// the vocabulary-parallel ranks' parts in rank order (indexed by row).
-__global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const float* parts, const int splits,
-                                                        const int by_position) {
+// [splits][R][rank]: the K splits of the dE GEMM, or the vocabulary-parallel ranks' parts
+// in rank order.
+__global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const float* parts, const int splits) {
   const int64_t n = a.R * a.rank;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t r = i / a.rank, j = i - r * a.rank;
     const bool live = a.ws.m[r] != 0 && a.valid[r] != 0;
     float acc = 0.f;
     if (live) {
-      const int64_t pr = by_position ? int64_t(a.ws.sup_index[r]) : r;
-      const float* dp = parts + size_t(pr) * a.rank + j;
+      const float* dp = parts + size_t(r) * a.rank + j;
       const size_t stride = size_t(a.R) * a.rank;
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;  // loads in flight together; fixed order
       int s = 0;
@@ -146,16 +138,15 @@ __global__ void __launch_bounds__(256) de_reduce_kernel(const HeadsArgs a, const
   }
 }
 
-// ---- one vocabulary-parallel rank's part of dE by row: the K splits of its dE GEMM (by
-// supervised position) summed in the order de_reduce_kernel uses (0 on rows without a
-// gradient)
+// ---- one vocabulary-parallel rank's part of dE: the K splits of its dE GEMM summed in
+// the order de_reduce_kernel uses (0 on rows without a gradient)
 __global__ void __launch_bounds__(256) de_split_sum_kernel(const HeadsArgs a, const int splits, float* out) {
   const int64_t n = a.R * a.rank;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t r = i / a.rank, j = i - r * a.rank;
     float acc = 0.f;
     if (a.ws.m[r] != 0 && a.valid[r] != 0) {
-      const float* dp = a.ws.dep + size_t(a.ws.sup_index[r]) * a.rank + j;  // partials by supervised position
+      const float* dp = a.ws.dep + size_t(r) * a.rank + j;
       const size_t stride = size_t(a.R) * a.rank;
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
       int s = 0;
@@ -333,11 +324,8 @@ cudaError_t launch_teacher_chunk(const TeacherArgs& a, int64_t row0, cudaStream_
   if (!tc::make_map(&mb, a.lm_head, a.V, a.Ht, a.Ht, 64, 256)) return cudaErrorInvalidValue;
   CUtensorMap mo;
   if (!tc::make_out_map(&mo, a.ws.tchunk, rows, a.V, a.V)) return cudaErrorInvalidValue;
-  tc::GemmOpts o;
-  o.m_bound = &a.ws.hdr->n_sup;
-  o.m_base = int(row0);
   return tc::gemm<256, false, false, 4>(ma, mb, int(rows), int(a.V), int(a.Ht), 1, TeacherEpi{}, &a.ws.hdr->status,
-                                        s, o, &mo);
+                                        s, &a.ws.hdr->n_sup, int(row0), &mo);
 }
 
 cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
@@ -347,59 +335,42 @@ cudaError_t launch_markov_bias(const HeadsArgs& a, cudaStream_t s) {
   CUtensorMap mo;
   if (!tc::make_out_map(&mo, a.ws.bias, a.R, a.V, a.V)) return cudaErrorInvalidValue;
   BiasEpi epi{a.ws.sup_list, a.ws.hdr, a.valid};
-  tc::GemmOpts o;
-  o.m_bound = &a.ws.hdr->n_sup;
-  return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s, o,
-                                        &mo);
+  return tc::gemm<256, false, false, 4>(ma, mb, int(a.R), int(a.V), int(a.rank), 1, epi, &a.ws.hdr->status, s,
+                                        &a.ws.hdr->n_sup, 0, &mo);
 }
 
 namespace {
 
-// dE split partials into ws.dep and dW2 (its rows of the vocabulary) from the bf16
-// dlogits of the supervised rows only: the GEMMs gather those rows by the supervised list
-// (every other row's dlogits are zero and contribute nothing).
+// dE split partials into ws.dep and dW2 (its rows of the vocabulary) from the bf16 dlogits
 cudaError_t markov_grad_gemms(const HeadsArgs& a, int splits, cudaStream_t s) {
-  // dlogits rows, fetched one row at a time in 64-column boxes
-  CUtensorMap mrow;
-  if (!tc::make_row_map(&mrow, a.dlogits, a.R, a.V, a.ld_g, 64)) return cudaErrorInvalidValue;
-  tc::GemmOpts o;
-  o.list = a.ws.sup_list;
-  o.list_len = &a.ws.hdr->n_sup;
-  o.zero_row = int(a.R);  // past the tensor map: zeros
-  // dE partials by supervised position: A = gathered dlogits [positions][V] (K-major),
-  // B = W2 as [V][rank] (MN-major); M bounded by the supervised count
-  CUtensorMap mb;
+  // dE partials: A = dlogits [R][V] (K-major), B = W2 as [V][rank] (MN-major)
+  CUtensorMap ma, mb;
+  if (!tc::make_map(&ma, a.dlogits, a.R, a.V, a.ld_g, 64, 128)) return cudaErrorInvalidValue;
   if (!tc::make_map(&mb, a.w2, a.V, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
   CUtensorMap mo;
   if (!tc::make_out_map(&mo, a.ws.dep, a.R, a.rank, a.rank, splits, a.R * a.rank)) return cudaErrorInvalidValue;
-  tc::GemmOpts oe = o;
-  oe.m_bound = &a.ws.hdr->n_sup;
-  cudaError_t e = tc::gemm<256, false, true, 4, PartialEpi, true>(mrow, mb, int(a.R), int(a.rank),
-                                                                   int(a.V), splits, PartialEpi{}, &a.ws.hdr->status,
-                                                                   s, oe, &mo);
+  cudaError_t e = tc::gemm<256, false, true, 4>(ma, mb, int(a.R), int(a.rank), int(a.V), splits, PartialEpi{},
+                                                &a.ws.hdr->status, s, nullptr, 0, &mo);
   if (e != cudaSuccess) return e;
-  // dW2 = dlogits^T . E over the supervised positions: A = gathered dlogits as [positions][V]
-  // (MN-major, M = vocabulary), B = the compact embeddings [positions][rank] (MN-major,
-  // zero past the last supervised position); K bounded by the supervised count
+  // dW2 = dlogits^T . E: A = dlogits as [R][V] (MN-major, M = vocabulary),
+  // B = E by row [R][rank] (MN-major)
   if (a.dw2 != nullptr) {
-    CUtensorMap mb2;
-    if (!tc::make_map(&mb2, a.ws.esup, a.R, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
+    CUtensorMap ma2, mb2;
+    if (!tc::make_map(&ma2, a.dlogits, a.R, a.V, a.ld_g, 64, 64)) return cudaErrorInvalidValue;
+    if (!tc::make_map(&mb2, a.ws.eall, a.R, a.rank, a.rank, 64, 64)) return cudaErrorInvalidValue;
     CUtensorMap mo2;
     if (!tc::make_out_map(&mo2, a.dw2, a.V, a.rank, a.rank)) return cudaErrorInvalidValue;
-    tc::GemmOpts ow = o;
-    ow.k_bound = &a.ws.hdr->n_sup;
-    e = tc::gemm<256, true, true, 4, WeightEpi, true>(mrow, mb2, int(a.V), int(a.rank), int(a.R), 1,
-                                                      WeightEpi{a.accumulate}, &a.ws.hdr->status, s, ow, &mo2);
+    e = tc::gemm<256, true, true, 4>(ma2, mb2, int(a.V), int(a.rank), int(a.R), 1, WeightEpi{a.accumulate},
+                                     &a.ws.hdr->status, s, nullptr, 0, &mo2);
   }
   return e;
 }
 
 // dE from its partials, dW1, then the confidence head's gradients
-cudaError_t merge_and_conf_grads(const HeadsArgs& a, const float* parts, int nparts, int by_position,
-                                 cudaStream_t s) {
+cudaError_t merge_and_conf_grads(const HeadsArgs& a, const float* parts, int nparts, cudaStream_t s) {
   cudaError_t e = cudaSuccess;
   if (a.w1 != nullptr) {
-    de_reduce_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, parts, nparts, by_position);
+    de_reduce_kernel<<<grid_for(a.R * a.rank, 256), 256, 0, s>>>(a, parts, nparts);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.conf_w != nullptr) {
@@ -426,7 +397,7 @@ cudaError_t launch_heads_bwd(const HeadsArgs& a, cudaStream_t s) {
     const cudaError_t e = markov_grad_gemms(a, splits, s);
     if (e != cudaSuccess) return e;
   }
-  return merge_and_conf_grads(a, a.ws.dep, splits, 1, s);
+  return merge_and_conf_grads(a, a.ws.dep, splits, s);
 }
 
 cudaError_t launch_markov_bwd_shard(const HeadsArgs& a, float* de_part, cudaStream_t s) {
@@ -438,7 +409,7 @@ cudaError_t launch_markov_bwd_shard(const HeadsArgs& a, float* de_part, cudaStre
 }
 
 cudaError_t launch_heads_bwd_merge(const HeadsArgs& a, const float* de_all, int nranks, cudaStream_t s) {
-  return merge_and_conf_grads(a, de_all, nranks, 0, s);
+  return merge_and_conf_grads(a, de_all, nranks, s);
 }
 
 }  // namespace dspark

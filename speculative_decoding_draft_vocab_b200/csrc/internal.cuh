@@ -55,7 +55,7 @@ struct WsView {
   float* bias;         // [R][V] Markov bias rows W2.e (0 on invalid slots), compact by supervised position
   uint16_t* esup;      // [R][rank] bf16 Markov embeddings, compact (0 on invalid slots)
   uint16_t* eall;      // [R][rank] bf16 Markov embeddings by row (0 unless supervised+valid)
-  float* dep;          // [splits][R][rank] split-K partials of dE, by supervised position
+  float* dep;          // [splits][R][rank] split-K partials of dE
   float* de;           // [R][rank] dL/de
   // teacher from hidden states (present when the problem has it)
   uint16_t* hsup;      // [R][Ht] bf16 target hidden rows, compact by supervised position
@@ -253,11 +253,10 @@ struct HeadsArgs {
 };
 
 // K splits of the dE contraction (a fixed count for a given shape, so the workspace
-// size does not depend on the device).  The contraction runs over the supervised rows
-// only, whose count the host does not know: the splits are sized for half of the rows.
+// size does not depend on the device).
 constexpr int kHeadsSlots = 148;
 constexpr int heads_splits(int64_t R, int64_t V) {
-  const int64_t m_tiles = R / 2 > 128 ? (R / 2 + 127) / 128 : 1, kchunks = (V + 63) / 64;
+  const int64_t m_tiles = (R + 127) / 128, kchunks = (V + 63) / 64;
   const int64_t s = kHeadsSlots / m_tiles;
   return int(s < 1 ? 1 : (s > kchunks ? kchunks : s));
 }
@@ -274,10 +273,7 @@ enum : int {
 };
 // False if V exceeds every build of that kind.
 bool sweep_supported(int kind, int64_t V, bool has_target);
-// The sweep with a teacher whose exponentials are held in TMEM (sweep_tm.cu), for the
-// bf16 kinds with a teacher: false if the kind has no such build or V exceeds its builds.
-bool sweep_tm_supported(int kind, int64_t V);
-cudaError_t launch_sweep_tm(int kind, const SweepArgs& a, cudaStream_t s);
+
 cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s);
 cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
                               const uint8_t* eval_mask, const uint8_t* block_keep,

@@ -49,28 +49,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// The same test, the thread suspended (issuing nothing) until the phase completes or
-// about `ns` nanoseconds have passed.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t ns) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done) : "r"(bar), "r"(parity), "r"(ns) : "memory");
-  return done != 0;
-}
-
-// How long one suspended test may sleep; waiting threads then leave the issue slots to
-// the warps that have work.
-constexpr uint32_t kSuspendNs = 1000000;  // 1 ms
-
-// Waits for phase `parity` of the mbarrier; false if the wait limit ran out.
+// Waits for phase `parity` of the mbarrier; false if the wait limit ran out.  The test
+// spins: a suspended test (try_wait with a time hint) was measured to add its wake-up
+// latency to every pipeline and exchange wait of the sweep and the GEMMs.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }

@@ -721,17 +721,9 @@ cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-// Kinds the TMEM-resident, row-pipelined sweep runs (the rest take sweep_kernel).
-constexpr bool kTmKinds[5] = {true, false, false, false, false};
-
-bool sweep_supported(int kind, int64_t V, bool has_target) {
-  if (has_target && kTmKinds[kind] && sweep_tm_supported(kind, V)) return true;
-  return pick_build(kind, V, has_target) >= 0;
-}
+bool sweep_supported(int kind, int64_t V, bool has_target) { return pick_build(kind, V, has_target) >= 0; }
 
 cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s) {
-  // rows with a teacher: the TMEM-resident, row-pipelined sweep
-  if (has_target && kTmKinds[kind] && sweep_tm_supported(kind, a.V)) return launch_sweep_tm(kind, a, s);
   const int i = pick_build(kind, a.V, has_target);
   if (i < 0) return cudaErrorInvalidValue;
   switch (kind) {

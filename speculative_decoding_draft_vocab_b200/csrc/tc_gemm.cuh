@@ -102,18 +102,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
 }
 
-// Four rows y0..y3 of a 2-D tensor map whose box is one row high, columns x .. x + box
-// width, written one after another at dst (the 128-byte swizzle follows the shared-
-// memory address, so 32 such loads fill a 128-row tile exactly as one 128-row box does).
-// Rows outside the tensor read as zeros.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
-                                            int y3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
-      ::"r"(dst), "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar) : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -161,44 +149,30 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, fl
 // large operand of the row-skinny products) through L2 instead of each m-tile
 // streaming all of B from HBM again.  With a device-side row bound (rows m_base + m
 // at or past *m_bound are not needed) only the first m_eff() m-tiles take part.
-// With a gather list, the rows of A are fetched by index: operand row i (an M index of a
-// K-major A, a K index of an MN-major A) is row list[i] of the tensor, for i below
-// *list_len, and a zero row past it.  With a device-side K bound only the first
-// ceil(*k_bound / BK) chunks of K take part (a work item with none stores zeros).
 struct WorkMap {
   int m_tiles, n_tiles, ksplit, kchunks;
   const int32_t* m_bound;
   int m_base;
-  const int32_t* k_bound;
-  const int32_t* list;
-  const int32_t* list_len;
-  int zero_row;  // a row index outside A's tensor map (reads as zeros)
   __device__ __forceinline__ int m_eff() const {
     if (m_bound == nullptr) return m_tiles;
     const int rem = *m_bound - m_base;
     return rem <= 0 ? 0 : min(m_tiles, (rem + BM - 1) / BM);
   }
-  __device__ __forceinline__ int k_eff() const {
-    if (k_bound == nullptr) return kchunks;
-    const int k = *k_bound;
-    return k <= 0 ? 0 : min(kchunks, (k + BK - 1) / BK);
-  }
   __device__ __forceinline__ int items(int me) const { return me * n_tiles * ksplit; }
-  __device__ __forceinline__ void decode(int w, int me, int ke, int& mt, int& nt, int& s, int& kc0, int& kc1) const {
+  __device__ __forceinline__ void decode(int w, int me, int& mt, int& nt, int& s, int& kc0, int& kc1) const {
     mt = w % me;
     const int t = w / me;
     s = t % ksplit;
     nt = t / ksplit;
-    kc0 = int((int64_t(s) * ke) / ksplit);
-    kc1 = int((int64_t(s + 1) * ke) / ksplit);
+    kc0 = int((int64_t(s) * kchunks) / ksplit);
+    kc1 = int((int64_t(s + 1) * kchunks) / ksplit);
   }
-  __device__ __forceinline__ int row_of(int i, int len) const { return i < len ? list[i] : zero_row; }
 };
 
 // A_MN / B_MN: operand stored MN-major (the M or N index is the contiguous one).
 // Tensor maps: K-major A = [M rows][K] box {64, 128}; MN-major A = [K rows][M] box
 // {64, 64}; K-major B = [N rows][K] box {64, BN}; MN-major B = [K rows][N] box {64, 64}.
-template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi, bool GA = false>
+template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmO, const WorkMap wm, const Epi epi, uint32_t* status) {
@@ -217,7 +191,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ME = wm.m_eff();  // the same in every role
-  const int KE = wm.k_eff();
   const int W = wm.items(ME);
 
   if (threadIdx.x == 0) {
@@ -238,45 +211,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t tmem_base = *tmem_slot;
   bool timed_out = false;
 
-  if (warp == 0 && (GA || lane == 0)) {
-    // ---------------- TMA producer (with a gather list the whole warp issues the
-    // 32 four-row loads of A's tile, one per lane)
-    const int glen = GA ? *wm.list_len : 0;
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
     int it = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x) {
       int mt, nt, s, kc0, kc1;
-      wm.decode(w, ME, KE, mt, nt, s, kc0, kc1);
+      wm.decode(w, ME, mt, nt, s, kc0, kc1);
       for (int kc = kc0; kc < kc1; ++kc, ++it) {
         const int st = it % STAGES;
         const uint32_t round = uint32_t(it / STAGES);
-        if (lane == 0 && !mbar_wait_bounded(empty0 + 8 * st, (round & 1u) ^ 1u)) timed_out = true;
+        if (!mbar_wait_bounded(empty0 + 8 * st, (round & 1u) ^ 1u)) timed_out = true;
         const uint32_t fb = full0 + 8 * st;
+        mbar_arrive_expect_tx(fb, SS);
         const uint32_t sa = smem_u32(smem + size_t(st) * SS), sb = sa + SA;
         const int k0 = kc * BK;
-        if constexpr (GA) {
-          __syncwarp();  // the stage is free for every lane
-          // K-major A: lane l fetches tile rows 4l .. 4l+3 (M indices);
-          // MN-major A: lane l fetches K rows 4(l % 16) .. +3 of column box l / 16
-          const int i0 = A_MN ? k0 + 4 * (lane & 15) : mt * BM + 4 * lane;
-          const int y0 = wm.row_of(i0, glen), y1 = wm.row_of(i0 + 1, glen);
-          const int y2 = wm.row_of(i0 + 2, glen), y3 = wm.row_of(i0 + 3, glen);
-          if (lane == 0) mbar_arrive_expect_tx(fb, SS);
-          __syncwarp();
-          if constexpr (!A_MN) {
-            tma_gather4(sa + uint32_t(lane) * 512u, &tmA, k0, y0, y1, y2, y3, fb);
-          } else {
-            tma_gather4(sa + uint32_t(lane >> 4) * 8192u + uint32_t(lane & 15) * 512u, &tmA,
-                        mt * BM + (lane >> 4) * 64, y0, y1, y2, y3, fb);
-          }
-          if (lane != 0) continue;
+        if constexpr (!A_MN) {
+          tma_load_2d(sa, &tmA, k0, mt * BM, fb);
         } else {
-          mbar_arrive_expect_tx(fb, SS);
-          if constexpr (!A_MN) {
-            tma_load_2d(sa, &tmA, k0, mt * BM, fb);
-          } else {
 #pragma unroll
-            for (int c = 0; c < BM / 64; ++c) tma_load_2d(sa + c * 8192, &tmA, mt * BM + c * 64, k0, fb);
-          }
+          for (int c = 0; c < BM / 64; ++c) tma_load_2d(sa + c * 8192, &tmA, mt * BM + c * 64, k0, fb);
         }
         if constexpr (!B_MN) {
           tma_load_2d(sb, &tmB, k0, nt * BN, fb);
@@ -291,7 +244,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     int it = 0, tl = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x, ++tl) {
       int mt, nt, s, kc0, kc1;
-      wm.decode(w, ME, KE, mt, nt, s, kc0, kc1);
+      wm.decode(w, ME, mt, nt, s, kc0, kc1);
       const int b = tl & 1;
       const uint32_t use = uint32_t(tl >> 1);
       if (!mbar_wait_bounded(acce0 + 8 * b, (use & 1u) ^ 1u)) timed_out = true;
@@ -324,14 +277,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     int tl = 0;
     for (int w = blockIdx.x; w < W; w += gridDim.x, ++tl) {
       int mt, nt, s, kc0, kc1;
-      wm.decode(w, ME, KE, mt, nt, s, kc0, kc1);
+      wm.decode(w, ME, mt, nt, s, kc0, kc1);
       const int b = tl & 1;
       const uint32_t use = uint32_t(tl >> 1);
       if (!mbar_wait_bounded(accf0 + 8 * b, use & 1u)) timed_out = true;
       fence_after_sync();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(b * BN);
       const int m0 = mt * BM + q * 32;
-      const bool no_k = kc1 <= kc0;  // no MMA ran: the tile is zero
       if constexpr (Epi::kTma) {
         const float scale = epi.row_scale(m0 + lane);  // this thread's row, once per tile
 #pragma unroll 1
@@ -339,10 +291,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           float v[32];
           __syncwarp();  // the TMEM load is warp-collective
           tmem_ld32(taddr + uint32_t(c * 32), v);
-          if (no_k) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          }
           const uint32_t buf = tbuf0 + uint32_t(blk & 1) * 4096u;
           if (lane == 0) bulk_wait_read<1>();  // the store that last used this buffer has read it
           __syncwarp();
@@ -371,7 +319,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           __syncwarp();  // the TMEM load is warp-collective
           tmem_ld32(taddr + uint32_t(c * 32), v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) tile[lane * kTileLd + i] = no_k ? 0.f : v[i];  // row lane, column i
+          for (int i = 0; i < 32; ++i) tile[lane * kTileLd + i] = v[i];  // row lane, column i
           __syncwarp();
           // rows m0 .. m0 + 31, columns n0 .. n0 + 31: element (r, j) at tile[r * kTileLd + j]
           epi(m0, nt * BN + c * 32, s, static_cast<const float*>(tile), lane, rs);

@@ -46,13 +46,6 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A bf16 matrix of `rows` x `cols` (row stride `ld` elements) read by gathers of single
-// rows: boxes of box_cols x 1 (box_cols * 2 = 128 bytes), 128-byte swizzle.
-inline bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
-                         uint32_t box_cols) {
-  return make_map(m, base, rows, cols, ld, box_cols, 1);
-}
-
 // An FP32 output seen by tensor stores of 32 x 32 blocks (128-byte swizzle): a matrix
 // of `rows` x `cols` (row stride `ld` elements), or `planes` such matrices `plane`
 // elements apart (3-D).  Blocks reaching past the matrix are clipped.
@@ -76,43 +69,24 @@ inline int sm_count() {
   return n > 0 ? n : 1;
 }
 
-// Device-side bounds and the row gather of a GEMM launch (all optional):
-//  - m_bound: rows m with m_base + m >= *m_bound (a count the device holds) are skipped;
-//  - k_bound: only K values below *k_bound take part (rounded up to a 64-wide chunk);
-//  - list / list_len / zero_row: A's rows are gathered, operand row i being tensor row
-//    list[i] for i < *list_len and `zero_row` (a row outside A's tensor map, read as
-//    zeros) past it; A's tensor map must then have boxes one row high (make_row_map).
-struct GemmOpts {
-  const int32_t* m_bound = nullptr;
-  int m_base = 0;
-  const int32_t* k_bound = nullptr;
-  const int32_t* list = nullptr;
-  const int32_t* list_len = nullptr;
-  int zero_row = 0;
-};
-
 // D[M, N] = A . B^T over K (A is M x K, B is N x K in the math), operands as described
-// by their tensor maps; work split into `ksplit` slices of K.  GA: A's rows are gathered
-// (see GemmOpts).  Returns the launch error.
-template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi, bool GA = false>
+// by their tensor maps; work split into `ksplit` slices of K.  With `m_bound`, rows m
+// with m_base + m >= *m_bound (a count the device holds) are skipped.  Returns the
+// launch error.
+template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi>
 cudaError_t gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int ksplit, const Epi& epi,
-                 uint32_t* status, cudaStream_t s, const GemmOpts& o = GemmOpts{},
+                 uint32_t* status, cudaStream_t s, const int32_t* m_bound = nullptr, int m_base = 0,
                  const CUtensorMap* out = nullptr) {
   if (Epi::kTma && out == nullptr) return cudaErrorInvalidValue;
-  if (GA && (o.list == nullptr || o.list_len == nullptr)) return cudaErrorInvalidValue;
   WorkMap wm;
-  wm.m_bound = o.m_bound;
-  wm.m_base = o.m_base;
-  wm.k_bound = o.k_bound;
-  wm.list = o.list;
-  wm.list_len = o.list_len;
-  wm.zero_row = o.zero_row;
+  wm.m_bound = m_bound;
+  wm.m_base = m_base;
   wm.m_tiles = (M + BM - 1) / BM;
   wm.n_tiles = (N + BN - 1) / BN;
   wm.kchunks = (K + BK - 1) / BK;
   wm.ksplit = std::max(1, std::min(ksplit, wm.kchunks));
   const int W = wm.m_tiles * wm.n_tiles * wm.ksplit;
-  auto kern = gemm_kernel<BN, A_MN, B_MN, STAGES, Epi, GA>;
+  auto kern = gemm_kernel<BN, A_MN, B_MN, STAGES, Epi>;
   constexpr size_t smem = gemm_smem_bytes<BN, STAGES>();
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;

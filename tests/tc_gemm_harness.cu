@@ -45,31 +45,3 @@ extern "C" int tc_gemm_test(const void* a, const void* b, float* d, int M, int N
   }
   return -2;
 }
-
-// Gathered A: the rows of the bf16 matrix `src` [src_rows][src_cols] listed in `list`
-// (`*len` of them, a device count) form A, fetched by four-row gathers.  a_mn = 0: A's
-// rows are M indices (D[M = positions, N] = sum over K = src_cols); a_mn = 1: A's rows are
-// K indices (D[M = src_cols, N] = sum over K = positions, bounded on the device by *len).
-// b is [N][K] (K-major) for a_mn = 0 and [K][N] (MN-major) for a_mn = 1.
-extern "C" int tc_gemm_gather_test(const void* src, int src_rows, int src_cols, const int32_t* list,
-                                   const int32_t* len, int positions, const void* b, int N, float* d, int a_mn,
-                                   int ksplit, uint32_t* status) {
-  CUtensorMap ma, mb;
-  if (!tc::make_row_map(&ma, src, src_rows, src_cols, src_cols, 64)) return -1;
-  tc::GemmOpts o;
-  o.list = list;
-  o.list_len = len;
-  o.zero_row = src_rows;
-  if (!a_mn) {
-    if (!tc::make_map(&mb, b, N, src_cols, src_cols, 64, 256)) return -1;
-    o.m_bound = len;
-    SplitStoreEpi epi{d, positions, N};
-    return int(tc::gemm<256, false, false, 4, SplitStoreEpi, true>(ma, mb, positions, N, src_cols, ksplit, epi,
-                                                                    status, nullptr, o));
-  }
-  if (!tc::make_map(&mb, b, positions, N, N, 64, 64)) return -1;
-  o.k_bound = len;
-  SplitStoreEpi epi{d, src_cols, N};
-  return int(tc::gemm<256, true, true, 4, SplitStoreEpi, true>(ma, mb, src_cols, N, positions, 1, epi, status,
-                                                                nullptr, o));
-}
