@@ -286,8 +286,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const int m0 = mt * BM + q * 32;
       if constexpr (Epi::kTma) {
         const float scale = epi.row_scale(m0 + lane);  // this thread's row, once per tile
+        // a 32-row block wholly past the device-side row bound is not needed: not stored
+        const bool needed = wm.m_bound == nullptr || wm.m_base + m0 < *wm.m_bound;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c, ++blk) {
+        for (int c = 0; needed && c < BN / 32; ++c, ++blk) {
           float v[32];
           __syncwarp();  // the TMEM load is warp-collective
           tmem_ld32(taddr + uint32_t(c * 32), v);

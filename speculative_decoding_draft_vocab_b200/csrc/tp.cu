@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
     const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
     const float keep = (HAS_B && a.ws.sup_tok[idx] < 0) ? 0.f : 1.f;
     float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
-#pragma unroll 2
+#pragma unroll 4
     for (int v = threadIdx.x; v < nvec; v += kTpThreads) {
       float x[VT::N];
       VT::load(zr + size_t(v) * 16, x);
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
       const uint8_t* tr = row_ptr<T>(a.target, row, a.ld_t);
       const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
       const float keep = (HAS_B && a.ws.sup_tok[idx] < 0) ? 0.f : 1.f;
-#pragma unroll 2
+#pragma unroll 4
       for (int v = threadIdx.x; v < nvec; v += kTpThreads) {
         float x[VT::N], y[VT::N];
         VT::load(zr + size_t(v) * 16, x);
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
       const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
       const float keep = zero_row ? 0.f : 1.f;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * size_t(a.ld_g) * sizeof(T);
-#pragma unroll 2
+#pragma unroll 4
       for (int v = threadIdx.x; v < nvec; v += kTpThreads) {
         float x[VT::N], o[VT::N];
         VT::load(zr + size_t(v) * 16, x);
