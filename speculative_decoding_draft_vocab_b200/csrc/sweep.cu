@@ -300,10 +300,6 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     const uint8_t* zb = zbuf(j);
     const uint8_t* bb = bbuf(j);
     const uint8_t* tb = tbuf(j);
-    // rows j + kRingFill .. j + kRing - 1 into the half of the ring that row j is not in
-    // (read from row j + kRingFill - 1 on, many barriers later)
-    if (j >= kRingFill && j % kRingFill == 0) fill_ring(j + kRingFill, kRingFill);
-
     if (!mbar_wait_bounded((j & 1) ? bar_d1 : bar_d0, phase) && tid == 0) flag_timeout();
 
     // ---- draft segment -> registers
@@ -331,6 +327,11 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
       ctrl->ztid = zt;
     }
     __syncthreads();  // the draft buffer is free again
+    // rows j + kRingFill .. j + kRing - 1 into the half of the ring that row j is not in.
+    // Only past this barrier: the slots hold rows j - kRingFill .. j - 1, and a warp still
+    // in pass 3 of row j - 1 reads that row's weight (its entries are read from row
+    // j + kRingFill on, many barriers later).
+    if (j >= kRingFill && j % kRingFill == 0) fill_ring(j + kRingFill, kRingFill);
     if (tid == 0) {
       // HAS_T: draft buffer + the teacher buffer of row j-1 (its pass 2 is done).
       // Without a teacher the draft buffers alternate.
