@@ -388,10 +388,7 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
         st_async_f4(dst, make_float4(m1, s1, m2, s2), dsmem_map(bar_ga, uint32_t(lane)));
       }
     }
-    // with a teacher, half of this row's slice of zero rows is stored during the (L1, S)
-    // exchange below; without one, all of it now
-    const int zmid = HAS_T ? min(ztot, j * zslice + zslice / 2) : min(ztot, (j + 1) * zslice);
-    write_zeros(j * zslice, zmid);
+    write_zeros(j * zslice, min(ztot, (j + 1) * zslice));
     if (warp == 0) {
       if (!mbar_wait_bounded(bar_ga, gphase) && lane == 0) flag_timeout();
       // NP partials, in the same order in every CTA: lane l merges l, l + 32, ...
@@ -462,7 +459,6 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
           st_async_f4(dst, make_float4(x, y, 0.f, 0.f), dsmem_map(bar_gb, uint32_t(lane)));
         }
       }
-      write_zeros(zmid, min(ztot, (j + 1) * zslice));
       if (!mbar_wait_bounded(bar_gb, gphase) && tid == 0) flag_timeout();
 #pragma unroll
       for (int i = 0; i < CL; ++i) {  // same order in every CTA
