@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, 1-D bulk async copies (TMA, no
-// multicast), thread-block-cluster barriers and distributed shared memory, and the
-// bounded waits every spin in this library uses.
+// multicast), thread-block-cluster barriers and distributed shared memory, per-thread
+// tensor-memory staging, and the bounded waits every spin in this library uses.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -201,5 +201,67 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+
+// ---------------------------------------------------------------- tensor memory
+// Per-thread staging of FP32 values in TMEM (no MMA).  A warp reaches only the 32 TMEM
+// lanes of its quarter (warp index mod 4); an address is (lane << 16) | column.  All of
+// these are warp-collective (.sync.aligned): the caller keeps the warp converged.
+namespace tm {
+
+__device__ __forceinline__ void alloc(uint32_t slot_saddr, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(slot_saddr), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// N consecutive columns of this thread's lane <- v[0 .. N-1]  (N = 4 or 8)
+template <int N> __device__ __forceinline__ void st(uint32_t taddr, const float* v);
+template <> __device__ __forceinline__ void st<8>(uint32_t taddr, const float* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]),
+                 "f"(v[6]), "f"(v[7]) : "memory");
+}
+template <> __device__ __forceinline__ void st<4>(uint32_t taddr, const float* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+               ::"r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]) : "memory");
+}
+// every tcgen05.st of this thread has completed
+__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// v[0 .. N-1] <- N consecutive columns of this thread's lane, waited for: the wait names
+// the destination registers, so no use of them is scheduled before it.
+template <int N> __device__ __forceinline__ void ld(uint32_t taddr, float* v);
+template <> __device__ __forceinline__ void ld<8>(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+                 "=f"(v[7]) : "r"(taddr) : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+                 "+f"(v[7]) :: "memory");
+}
+template <> __device__ __forceinline__ void ld<4>(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(taddr) : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]) :: "memory");
+}
+
+// Columns to allocate: a power of two, at least 32.
+__host__ __device__ constexpr uint32_t alloc_cols(uint32_t n) {
+  uint32_t c = 32;
+  while (c < n) c <<= 1;
+  return c;
+}
+
+}  // namespace tm
 
 }  // namespace dspark

@@ -5,7 +5,8 @@
 // of the next rows is streamed into shared memory by 1-D bulk async copies (TMA,
 // no multicast) while the current row is processed from registers, so every logit
 // is read from HBM exactly once.  The exponentials are taken once per element and
-// kept in registers for the rest of the row; the three row-wide reductions
+// kept on chip for the rest of the row (the draft's in registers, the teacher's in
+// tensor memory); the three row-wide reductions
 // (logsumexp; L1 and S; nothing else) combine per-CTA partials through distributed
 // shared memory, in the same fixed order in every CTA, so every CTA sees bitwise
 // the same row scalars.  dlogits are written in the same sweep.
@@ -15,7 +16,8 @@
 //   lse_d = log sum exp z,  lse_t = log sum exp t,  CE = lse_d - z[id]
 //   p = exp(z - lse_d), q = exp(t - lse_t), L1 = sum |p - q| (raw), S = sum p*sign(p-q)
 //   dL/dz_j = g*w*[ce_alpha*(p_j - [j = id]) + l1_alpha*p_j*(sign(p_j - q_j) - S)]
-// Everything is computed in base 2: offsets are kept as x*log2(e).
+// Everything is computed in base 2: offsets are kept as x*log2(e).  Each logit costs
+// one ex2 for the draft and one for the teacher.
 #include <cuda_bf16.h>
 #include <algorithm>
 #include <mutex>
@@ -112,7 +114,8 @@ struct Ctrl {
   float4 bcast;           // row logsumexps (base 2)
   float ztid;             // raw draft logit at the target id (owner only)
   int last;               // this CTA finished last and writes the report
-  float pad[2];
+  uint32_t tmem;          // TMEM base address of the teacher's exponentials
+  float pad;
   // ring of the cluster's upcoming rows: row id, target id, loss weight
   int32_t rrow[64];
   int32_t rtok[64];
@@ -141,11 +144,12 @@ __device__ __forceinline__ void lse_pair_merge(float& m1, float& s1, float& m2, 
 
 // One cluster of CL CTAs owns one supervised row at a time; CTA `rank` owns the
 // rank-th contiguous segment of the vocabulary.  Draft values live in registers
-// (NV 16-byte vectors per thread, as FP32 exponentials); the teacher segment stays
-// in shared memory as loaded and is re-read, so a CTA holds 6 bytes per logit pair
-// on chip and a row fits in 4 SMs of a 148-SM part.  Shared memory holds one draft
-// landing buffer and two teacher buffers: the next row's copy is issued as soon as
-// the current draft segment is in registers, one full row ahead of its use.
+// (NV 16-byte vectors per thread, as FP32 exponentials); the teacher segment is read
+// twice from shared memory in pass 1 (maximum, then exponentials), and its FP32
+// exponentials wait in tensor memory (TMEM, staging only: no MMA) for pass 2, so each
+// teacher value costs one ex2.  Shared memory holds one draft landing buffer and two
+// teacher buffers: the next row's copy is issued as soon as the current draft segment
+// is in registers, one full row ahead of its use.
 // TZ is the draft logits' type; TT the teacher rows' type (the logits type, or FP32
 // rows of the teacher computed from hidden states); TO the type of the dlogits.  With
 // HAS_B (the Markov head) the corrected row z = keep * base + bias is formed on chip
@@ -171,6 +175,10 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   static_assert(NW <= 32 && CL <= 16, "control block sizes");
   static_assert(NE % 4 == 0, "whole groups of four elements");
   using CtrlT = Ctrl<NP>;
+  // With a teacher, pass 1 keeps the teacher's exponentials in TMEM for pass 2: warp w
+  // owns columns [(w / 4) * NE, (w / 4 + 1) * NE) of the 32 lanes of quarter w mod 4.
+  constexpr uint32_t kTmCols = HAS_T ? tm::alloc_cols(uint32_t(NW / 4) * NE) : 0u;
+  static_assert(!HAS_T || (NW % 4 == 0 && kTmCols <= 256), "TMEM columns of a teacher build");
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -233,9 +241,21 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     mbar_init(bar_gb, 1);
     fence_mbar_init();
   }
+  if constexpr (HAS_T) {
+    if (warp == 0) {
+      __syncwarp();
+      tm::alloc(smem_u32(&ctrl->tmem), kTmCols);
+    }
+    tm::fence_before_sync();
+  }
   // every CTA's barriers exist before any peer signals them
   __syncthreads();
   cluster_sync();
+  uint32_t taddr = 0;  // this warp's first TMEM column
+  if constexpr (HAS_T) {
+    tm::fence_after_sync();
+    taddr = ctrl->tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t((warp >> 2) * NE);
+  }
   // the mask prologue has finished and its writes are visible past this point
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // this launch's supervised rows: list positions [row0, min(row1, n_sup))
@@ -344,7 +364,18 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     float mz = -INFINITY, mt = -INFINITY;
 #pragma unroll
     for (int e = 0; e < NE; e += 2) mz = fmax3(mz, xz[e], xz[e + 1]);
-    if constexpr (HAS_T) {
+    if constexpr (HAS_T && sizeof(TT) == 2) {  // bf16 pairs compared packed (exact)
+      uint32_t mp = 0xff80ff80u;  // (-inf, -inf)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int v = tid + i * NT;
+        if (v < nvec) {
+          const uint4 q = *reinterpret_cast<const uint4*>(tb + size_t(v) * TB);
+          mp = bf2max(mp, bf2max(bf2max(q.x, q.y), bf2max(q.z, q.w)));
+        }
+      }
+      mt = fmaxf(bf16lo(mp), bf16hi(mp));
+    } else if constexpr (HAS_T) {
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int v = tid + i * NT;
@@ -364,16 +395,25 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
       xz[e] = ex2(fmaf(xz[e], kLog2e, -oz));
       sz += xz[e];
     }
-    if constexpr (HAS_T) {
+    if constexpr (HAS_T) {  // the teacher's exponentials, summed and kept in TMEM
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int v = tid + i * NT;
+        float e8[EPV];
         if (v < nvec) {
           float t8[EPV];
           load_group<TT, EPV>(tb + size_t(v) * TB, t8);
 #pragma unroll
-          for (int e = 0; e < EPV; ++e) st += ex2(fmaf(t8[e], kLog2e, -ot));
+          for (int e = 0; e < EPV; ++e) {
+            e8[e] = ex2(fmaf(t8[e], kLog2e, -ot));
+            st += e8[e];
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) e8[e] = 0.f;
         }
+        __syncwarp();
+        tm::st<EPV>(taddr + uint32_t(i * EPV), e8);
       }
     }
 
@@ -411,21 +451,23 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     const float az = (mz == -INFINITY) ? 0.f : ex2(oz - lz2);  // p = e * az
     const float at = (!HAS_T || mt == -INFINITY) ? 0.f : ex2(ot - lt2);
 
-    // ---- pass 2: L1 and S.  q is rebuilt exactly as pass 1 formed it, so equal
-    // draft and teacher rows give p == q bit for bit.  xz <- u = p * sign(p - q)
-    // (an exact tie takes the sub-gradient +p).
+    // ---- pass 2: L1 and S.  q is formed from pass 1's own exponentials (read back
+    // from TMEM) exactly as p is, so equal draft and teacher rows give p == q bit for
+    // bit.  xz <- u = p * sign(p - q) (an exact tie takes the sub-gradient +p).
     float L1 = 0.f, S = 0.f;
     if constexpr (HAS_T) {
+      tm::wait_st();
       float l4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int v = tid + i * NT;
+        float e8[EPV];
+        __syncwarp();
+        tm::ld<EPV>(taddr + uint32_t(i * EPV), e8);
         if (v < nvec) {
-          float t8[EPV];
-          load_group<TT, EPV>(tb + size_t(v) * TB, t8);
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
-            const float q = __fmul_rn(ex2(fmaf(t8[e], kLog2e, -ot)), at);
+            const float q = __fmul_rn(e8[e], at);
             const float p = __fmul_rn(xz[i * EPV + e], az);
             const float d = __fsub_rn(p, q);
             const float u = copysignf(p, d);
@@ -515,9 +557,17 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
 
   // ---- what is left of this cluster's zero rows (all of them if it had no row)
   write_zeros(my_n * zslice, ztot);
+  if constexpr (HAS_T) tm::fence_before_sync();
   // no CTA leaves while a peer may still signal or read its shared memory
   __syncthreads();
   cluster_sync();
+  if constexpr (HAS_T) {
+    if (warp == 0) {  // every warp's TMEM reads completed before the barrier
+      tm::fence_after_sync();
+      __syncwarp();
+      tm::dealloc(ctrl->tmem, kTmCols);
+    }
+  }
 
   // ---- the last CTA to finish writes the per-row epilogue and the report (in the
   // launch that covers the last rows)
