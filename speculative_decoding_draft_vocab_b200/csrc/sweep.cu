@@ -431,17 +431,31 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
     write_zeros(j * zslice, min(ztot, (j + 1) * zslice));
     if (warp == 0) {
       if (!mbar_wait_bounded(bar_ga, gphase) && lane == 0) flag_timeout();
-      // NP partials, in the same order in every CTA: lane l merges l, l + 32, ...
-      float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
+      // NP partials, in the same order in every CTA: the maxima first, then one
+      // rescaled sum (lane l holds partials l, l + 32, ...; independent ex2s)
+      constexpr int KP = (NP + 31) / 32;
+      float4 q4[KP];
+      float m1 = -INFINITY, m2 = -INFINITY;
 #pragma unroll
-      for (int k = lane; k < NP; k += 32) {
-        const float4 q4 = ctrl->ga[k];
-        const float n1 = fmaxf(m1, q4.x), n2 = fmaxf(m2, q4.z);
-        s1 = (n1 == -INFINITY) ? 0.f : s1 * ex2(m1 - n1) + (q4.x == -INFINITY ? 0.f : q4.y * ex2(q4.x - n1));
-        s2 = (n2 == -INFINITY) ? 0.f : s2 * ex2(m2 - n2) + (q4.z == -INFINITY ? 0.f : q4.w * ex2(q4.z - n2));
-        m1 = n1, m2 = n2;
+      for (int kk = 0; kk < KP; ++kk) {
+        const int k = lane + 32 * kk;
+        q4[kk] = k < NP ? ctrl->ga[k] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        m1 = fmaxf(m1, q4[kk].x);
+        m2 = fmaxf(m2, q4[kk].z);
       }
-      lse_pair_merge(m1, s1, m2, s2);
+      m1 = warp_max_f32(m1);
+      m2 = warp_max_f32(m2);
+      float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KP; ++kk) {
+        s1 += q4[kk].x == -INFINITY ? 0.f : q4[kk].y * ex2(q4[kk].x - m1);
+        s2 += q4[kk].z == -INFINITY ? 0.f : q4[kk].w * ex2(q4[kk].z - m2);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      }
       if (lane == 0) ctrl->bcast = make_float4(m1 + log2f(s1), HAS_T ? m2 + log2f(s2) : 0.f, 0.f, 0.f);
     }
     __syncthreads();
