@@ -192,8 +192,8 @@ def algorithmic_flops(inp, n_sup: int) -> int:
 
 def launches_per_call(inp) -> int:
     """Kernels one fused call launches (the launch sequence of dspark_loss_fwd)."""
-    n = 2  # mask prologue, sweep
     markov, conf_head, lm = inp.markov_w2 is not None, inp.conf_w is not None, inp.lm_head is not None
+    n = 2 if lm else 3  # mask prologue, sweep (and, without lm_head, the zero-row fill behind it)
     if markov or conf_head:
         n += 1  # gather of embeddings and confidence logits
     if markov:
@@ -471,7 +471,7 @@ def time_calls(call, steps: int, warmup: int, flush, clk_device: int):
 def timed_label(inp) -> str:
     n = launches_per_call(inp)
     return (f"dspark_loss_fwd with fused backward ({n} kernels: "
-            + ("mask prologue + sweep" if n == 2 else "prologue, heads, sweep, head gradients")
+            + ("mask prologue, sweep, zero-row fill" if n == 3 else "prologue, heads, sweep, head gradients")
             + "), median CUDA-event duration per call")
 
 

@@ -350,7 +350,12 @@ dspark_status_t dspark_loss_fwd(const dspark_problem_t* prob, const dspark_param
   fa.dconf = grads ? grads->dconf : nullptr;
   const int kind = sweep_kind(prob);
   if (!sh.has_lm_head) {
-    e = launch_sweep(kind, sh.has_teacher, sa, s);
+    // the zero rows are filled on the SMs the sweep leaves idle, by its dependent grid
+    const bool side_zero = sa.dlogits != nullptr;
+    sa.do_zero = side_zero ? 0 : 1;
+    int ctas = 0;
+    e = launch_sweep(kind, sh.has_teacher, sa, s, &ctas);
+    if (e == cudaSuccess && side_zero) e = launch_zero_rows(kind, sa, ctas, s);
     if (e != cudaSuccess) return cuda_status(e);
   } else {
     // teacher rows a chunk of supervised rows at a time, each chunk swept right after

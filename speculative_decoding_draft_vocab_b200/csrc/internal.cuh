@@ -274,7 +274,12 @@ enum : int {
 // False if V exceeds every build of that kind.
 bool sweep_supported(int kind, int64_t V, bool has_target);
 
-cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s);
+// `ctas` (if non-null) receives the number of CTAs the sweep launched.
+cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s, int* ctas = nullptr);
+// The unsupervised rows' zero dlogits, launched right behind a sweep that leaves them out
+// (do_zero = 0) as its programmatic dependent: it runs on the SMs the sweep leaves idle
+// (`sweep_ctas` of them taken) and finishes only after the sweep has.
+cudaError_t launch_zero_rows(int kind, const SweepArgs& a, int sweep_ctas, cudaStream_t s);
 cudaError_t launch_acceptance(int64_t B, int64_t N, int64_t K, const float* l1_rows,
                               const uint8_t* eval_mask, const uint8_t* block_keep,
                               float* accept_pair, float* tau_pair, float* accept_rows,

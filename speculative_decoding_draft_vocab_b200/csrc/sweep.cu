@@ -258,6 +258,8 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   }
   // the mask prologue has finished and its writes are visible past this point
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // a programmatic dependent (the zero-row fill) may start once every CTA is here
+  asm volatile("griddepcontrol.launch_dependents;");
   // this launch's supervised rows: list positions [row0, min(row1, n_sup))
   const int n_sup = max(0, min(hdr->n_sup, a.row1) - a.row0);
   const int my_n = (int(cid) < n_sup) ? (n_sup - 1 - int(cid)) / int(G) + 1 : 0;
@@ -623,7 +625,7 @@ size_t smem_bytes(int64_t V, bool has_t, bool has_b, int nt) {
 }
 
 template <typename TZ, typename TT, typename TO, int CL, int NT, int NV, bool HAS_T, bool HAS_B>
-cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
+cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s, int* ctas) {
   constexpr int EPV = VecTraits<TO>::EPV;
   SweepArgs a = a0;
   a.vvec = int32_t(a.V / EPV);
@@ -689,6 +691,7 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s) {
   cfg.numAttrs = 2;
   err = cudaLaunchKernelEx(&cfg, kern, a);
   if (err != cudaSuccess) cudaGetLastError();  // a refused launch leaves no error for later calls
+  if (ctas) *ctas = clusters * CL;
   return err;
 }
 
@@ -747,38 +750,38 @@ int pick_build(int kind, int64_t V, bool has_t) {
 }
 
 template <typename TZ, typename TT, typename TO, bool HT, bool HB>
-cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
+cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s, int* ctas) {
   if constexpr (sizeof(TZ) == 4) {
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 8, HT, HB>(a, s);
-      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 10, HT, HB>(a, s);
-      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 5, HT, HB>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s, ctas);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s, ctas);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 8, HT, HB>(a, s, ctas);
+      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 10, HT, HB>(a, s, ctas);
+      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 5, HT, HB>(a, s, ctas);
     }
   } else if constexpr (sizeof(TT) == 2 && !HB) {
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s);
-      case 3: return launch_cfg<TZ, TT, TO, 5, 640, 6, HT, HB>(a, s);
-      case 4: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT, HB>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s, ctas);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s, ctas);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s, ctas);
+      case 3: return launch_cfg<TZ, TT, TO, 5, 640, 6, HT, HB>(a, s, ctas);
+      case 4: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT, HB>(a, s, ctas);
     }
   } else if constexpr (sizeof(TT) == 4 && HB) {  // kTeacherBiasBuilds
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s);
-      case 3: return launch_cfg<TZ, TT, TO, 10, 512, 4, HT, HB>(a, s);
-      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 3, HT, HB>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s, ctas);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s, ctas);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s, ctas);
+      case 3: return launch_cfg<TZ, TT, TO, 10, 512, 4, HT, HB>(a, s, ctas);
+      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 3, HT, HB>(a, s, ctas);
     }
   } else {  // kHeadBuilds
     switch (i) {
-      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s);
-      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s);
-      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s);
-      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT, HB>(a, s);
-      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 3, HT, HB>(a, s);
+      case 0: return launch_cfg<TZ, TT, TO, 1, 256, 1, HT, HB>(a, s, ctas);
+      case 1: return launch_cfg<TZ, TT, TO, 2, 512, 2, HT, HB>(a, s, ctas);
+      case 2: return launch_cfg<TZ, TT, TO, 4, 512, 4, HT, HB>(a, s, ctas);
+      case 3: return launch_cfg<TZ, TT, TO, 8, 512, 5, HT, HB>(a, s, ctas);
+      case 4: return launch_cfg<TZ, TT, TO, 16, 512, 3, HT, HB>(a, s, ctas);
     }
   }
   return cudaErrorInvalidValue;
@@ -788,25 +791,63 @@ cudaError_t dispatch(int i, const SweepArgs& a, cudaStream_t s) {
 
 bool sweep_supported(int kind, int64_t V, bool has_target) { return pick_build(kind, V, has_target) >= 0; }
 
-cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s) {
+cudaError_t launch_sweep(int kind, bool has_target, const SweepArgs& a, cudaStream_t s, int* ctas) {
   const int i = pick_build(kind, a.V, has_target);
   if (i < 0) return cudaErrorInvalidValue;
   switch (kind) {
     case kSweepBf16:
-      return has_target ? dispatch<bf16, bf16, bf16, true, false>(i, a, s)
-                        : dispatch<bf16, bf16, bf16, false, false>(i, a, s);
+      return has_target ? dispatch<bf16, bf16, bf16, true, false>(i, a, s, ctas)
+                        : dispatch<bf16, bf16, bf16, false, false>(i, a, s, ctas);
     case kSweepF32:
-      return has_target ? dispatch<float, float, float, true, false>(i, a, s)
-                        : dispatch<float, float, float, false, false>(i, a, s);
+      return has_target ? dispatch<float, float, float, true, false>(i, a, s, ctas)
+                        : dispatch<float, float, float, false, false>(i, a, s, ctas);
     case kSweepZ32:
-      return has_target ? dispatch<bf16, bf16, bf16, true, true>(i, a, s)
-                        : dispatch<bf16, bf16, bf16, false, true>(i, a, s);
+      return has_target ? dispatch<bf16, bf16, bf16, true, true>(i, a, s, ctas)
+                        : dispatch<bf16, bf16, bf16, false, true>(i, a, s, ctas);
     case kSweepT32:
-      return dispatch<bf16, float, bf16, true, false>(i, a, s);
+      return dispatch<bf16, float, bf16, true, false>(i, a, s, ctas);
     case kSweepZT32:
-      return dispatch<bf16, float, bf16, true, true>(i, a, s);
+      return dispatch<bf16, float, bf16, true, true>(i, a, s, ctas);
   }
   return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------ zero-row fill
+// One CTA per unsupervised row at a time, 16-byte zero stores over the whole row.  It
+// reads the prologue's list, complete before any sweep CTA passed its own dependency
+// wait, which is where the sweep releases this grid; it waits for the sweep at its end.
+constexpr int kZeroThreads = 1024;
+
+__global__ void __launch_bounds__(kZeroThreads) zero_rows_kernel(const SweepArgs a, int vvec, int osize) {
+  const int n_zero = a.ws.hdr->n_zero;
+  for (int k = blockIdx.x; k < n_zero; k += gridDim.x) {
+    uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(a.ws.zero_list[k]) * a.ld_g * size_t(osize);
+    for (int v = threadIdx.x; v < vvec; v += kZeroThreads)
+      *reinterpret_cast<uint4*>(out + size_t(v) * 16) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  // whatever follows on the stream waits for this grid: it must find the sweep done too
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+cudaError_t launch_zero_rows(int kind, const SweepArgs& a, int sweep_ctas, cudaStream_t s) {
+  const int osize = kind == kSweepF32 ? 4 : 2;
+  const int vvec = int(a.V * osize / 16);
+  int dev = 0, sms = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(std::max(sms - sweep_ctas, 8)), 1, 1);
+  cfg.blockDim = dim3(kZeroThreads, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, zero_rows_kernel, a, vvec, osize);
+  if (err != cudaSuccess) cudaGetLastError();
+  return err;
 }
 
 // ------------------------------------------------------- backward-only stream
