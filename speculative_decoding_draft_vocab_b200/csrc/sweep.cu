@@ -595,7 +595,8 @@ __global__ void __launch_bounds__(NT, 1) sweep_kernel(const SweepArgs a) {
   __syncthreads();
   if (ctrl->last) {
     __threadfence();
-    finalize_rows(a.fin, reinterpret_cast<double*>(smem));
+    if (a.fin.K <= NT) finalize_rows_smem(a.fin, reinterpret_cast<double*>(smem));
+    else finalize_rows(a.fin, reinterpret_cast<double*>(smem));
     if (tid == 0) hdr->done = 0;
   }
 }
@@ -631,9 +632,9 @@ cudaError_t launch_cfg(const SweepArgs& a0, cudaStream_t s, int* ctas) {
   a.vvec = int32_t(a.V / EPV);
   a.seg_vec = (a.vvec + CL - 1) / CL;
   a.nbuf = 2;
-  // at least the report's reduction scratch (reused at the end)
+  // at least the report's scratch (reused at the end)
   const size_t smem = std::max<size_t>(smem_bytes<TZ, TT, TO, CL>(a.V, HAS_T, HAS_B, NT),
-                                       size_t(NT / 32) * kNAcc * sizeof(double));
+                                       (size_t(kNAcc + 1) * NT + kNAcc) * sizeof(double));
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
 
   auto kern = sweep_kernel<TZ, TT, TO, CL, NT, NV, HAS_T, HAS_B>;

@@ -113,6 +113,35 @@ def test_disjoint_rows_l1_two():
     assert call.out.report[5].tolist() == [2.0, 2.0]
 
 
+@pytest.mark.parametrize("B,N,K,V", [(8, 40, 7, 4096), (8, 128, 8, 1024), (4, 257, 8, 1024), (2, 9, 3, 2048)])
+def test_many_rows_dropped_blocks_and_bad_ids(B, N, K, V):
+    """Up to 8224 rows of small vocabularies (many rows per cluster, the row-scalar ring
+    refilled several times), masks with holes, blocks dropped at random, then a few
+    out-of-range ids on supervised positions: flagged, and their rows dropped from the
+    supervised list (zero dlogits)."""
+    inp = make_inputs("recipe", device="cuda", B=B, N=N, K=K, V=V, mask_holes=True, seed=31 + B * N * K)
+    gen = torch.Generator(device="cpu").manual_seed(B * N)
+    drop = (torch.rand(inp.block_keep.shape, generator=gen) < 0.2).to(inp.block_keep.device)
+    inp.block_keep[drop] = 0
+    call = run_gpu(inp)
+    from speculative_decoding_draft_vocab_b200 import abi
+    assert call.check_status() == 0
+    compare(inp, call, oracle_run(inp))
+    # out-of-range ids on supervised positions
+    flat = inp.target_ids.view(-1)
+    sup = (torch.cumprod(inp.eval_mask.long(), dim=-1) * inp.block_keep.long().unsqueeze(-1)).view(-1)
+    cand = torch.nonzero(sup.cpu()).view(-1)
+    bad = cand[torch.randperm(cand.numel(), generator=gen)[:3]].to(flat.device)
+    flat[bad] = V + 3
+    call = run_gpu(inp)
+    assert call.check_status() == abi.DSPARK_ERR_ID_OUT_OF_RANGE
+    flat[bad] = 0
+    for r in bad.tolist():
+        b, rest = divmod(r, N * K)
+        n, k = divmod(rest, K)
+        assert bool((call.out.dlogits[b, n, k] == 0).all())
+
+
 def test_all_masked_batch():
     inp = make_inputs("recipe", device="cuda", B=2, N=3, K=7, V=4096, prefix=(0, 0), seed=9)
     call, ref, _ = _run_and_compare(inp)
