@@ -459,6 +459,13 @@ dspark_status_t dspark_tp_partials(const dspark_problem_t* prob, const dspark_pa
   }
   TpArgs a = tp_args(prob, params, tp, v);
   a.rec1 = rec1;
+  if (!sh.has_markov && !sh.has_conf_head) {  // nothing between the prologue and step 1
+    a.own_rows = 1;
+    a.eval_mask = prob->eval_mask;
+    a.block_keep = prob->block_keep;
+    a.K = prob->K;
+    a.vocab_size = tp->vocab_size;
+  }
   return cuda_status(launch_tp_partials(prob->logits_dtype == DSPARK_F32, a, s));
 }
 

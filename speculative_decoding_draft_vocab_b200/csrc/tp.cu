@@ -160,12 +160,31 @@ template <typename T, bool HAS_T, bool HAS_B>
 __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[2 * kTpWarps];
-  // launched behind the mask prologue: its row lists are complete past this point
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int row_sup;
   const int nvec = int(a.V / VT::N);
-  const int n_sup = a.ws.hdr->n_sup;
-  for (int idx = blockIdx.x; idx < n_sup; idx += gridDim.x) {
-    const int64_t row = a.ws.sup_list[idx];
+  // own_rows: every row, supervised or not by the prologue's rule (prefix of eval_mask
+  // within the block, block_keep, target id in range), decided here; otherwise the
+  // prologue's list of supervised rows, complete past the dependency wait
+  if (!a.own_rows) asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int n_rows = a.own_rows ? int(a.R) : a.ws.hdr->n_sup;
+  for (int idx = blockIdx.x; idx < n_rows; idx += gridDim.x) {
+    int64_t row;
+    if (a.own_rows) {
+      row = idx;
+      if (threadIdx.x == 0) {
+        const int64_t blk = row / a.K, k = row - blk * a.K;
+        bool run = a.block_keep == nullptr || a.block_keep[blk] != 0;
+        for (int64_t j = 0; j <= k; ++j) run &= a.eval_mask[blk * a.K + j] != 0;
+        const int64_t t = a.tids[row];
+        row_sup = run && t >= 0 && t < a.vocab_size;
+      }
+      __syncthreads();
+      const bool sup = row_sup != 0;
+      __syncthreads();  // read by every thread before thread 0 rewrites it
+      if (!sup) continue;
+    } else {
+      row = a.ws.sup_list[idx];
+    }
     const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
     const uint8_t* tr = HAS_T ? row_ptr<T>(a.target, row, a.ld_t) : nullptr;
     const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
@@ -196,6 +215,9 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
       rec[1] = make_float4(zt, 0.f, 0.f, 0.f);
     }
   }
+  // what follows on the stream reads the prologue's lists: it must find the prologue
+  // finished too
+  if (a.own_rows) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- step 2

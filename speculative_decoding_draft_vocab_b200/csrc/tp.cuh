@@ -23,6 +23,14 @@ struct TpArgs {
   float* rec2;               // [R][4] this shard's (L1, S) partials
   const float* rec2_all;     // [tp_size][R][4]
   const float* bias;         // Markov bias rows of the shard (compact by supervised position), or null
+  // Step 1 straight behind the mask prologue (no heads): it takes every row and decides
+  // by the prologue's own rule whether the row is supervised, so it need not wait for
+  // the prologue's lists
+  int32_t own_rows;
+  const uint8_t* eval_mask;
+  const uint8_t* block_keep;
+  int64_t K;
+  int64_t vocab_size;        // global vocabulary (the target ids' range)
   float ce_alpha, l1_alpha;
   WsView ws;
   FinalizeArgs fin;          // the per-row epilogue and report the last CTA of step 3 runs

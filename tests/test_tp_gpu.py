@@ -63,6 +63,18 @@ def test_tp_group_matches_oracle(dtype, V, T):
     _check_group(inp, ranks, oracle_run(inp))
 
 
+def test_tp_dropped_blocks_and_many_rows():
+    """Blocks dropped at random (block_keep 0 on blocks whose masks are set) and more rows
+    than the step kernels have CTAs: step 1 decides itself which rows are supervised, by
+    the prologue's rule, and must agree with the prologue's lists that steps 2 and 3 use."""
+    inp = make_inputs("recipe", device="cuda", B=4, N=80, K=7, V=4096, mask_holes=True, seed=48)
+    gen = torch.Generator(device="cpu").manual_seed(48)
+    drop = (torch.rand(inp.block_keep.shape, generator=gen) < 0.25).to(inp.block_keep.device)
+    inp.block_keep[drop] = 0
+    ranks = _group(inp, 3)
+    _check_group(inp, ranks, oracle_run(inp))
+
+
 def test_tp_given_confidence_gamma_none_grad_scale():
     inp = make_inputs("recipe", device="cuda", B=2, N=4, K=7, V=8192, conf="given", gamma=None,
                       grad_scale=0.37, seed=41)
