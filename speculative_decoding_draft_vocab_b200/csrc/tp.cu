@@ -290,7 +290,8 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float rowS;
   __shared__ int last;
-  __shared__ double scratch[kTpWarps * kNAcc];
+  // the report's scratch: per-thread partials, one acceptance per thread, the totals
+  __shared__ double scratch[(kNAcc + 1) * kTpThreads + kNAcc];
   const int nvec = int(a.V / VT::N);
   const int n_sup = a.ws.hdr->n_sup;
   const int total = n_sup + (a.dlogits ? a.ws.hdr->n_zero : 0);
@@ -368,7 +369,8 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
   __syncthreads();
   if (last) {
     __threadfence();
-    finalize_rows(a.fin, scratch);
+    if (a.fin.K <= kTpThreads) finalize_rows_smem(a.fin, scratch);
+    else finalize_rows(a.fin, scratch);
     if (threadIdx.x == 0) a.ws.hdr->done = 0;
   }
 }
