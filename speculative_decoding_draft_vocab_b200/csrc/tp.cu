@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
   // within the block, block_keep, target id in range), decided here; otherwise the
   // prologue's list of supervised rows, complete past the dependency wait
   if (!a.own_rows) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next step may be scheduled now; it waits for this grid before reading anything
+  asm volatile("griddepcontrol.launch_dependents;");
   const int n_rows = a.own_rows ? int(a.R) : a.ws.hdr->n_sup;
   for (int idx = blockIdx.x; idx < n_rows; idx += gridDim.x) {
     int64_t row;
@@ -226,6 +228,9 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[kTpWarps];
   __shared__ float2 lse2;  // the row's base-2 logsumexps, as every step uses them
+  // launched behind the previous step (or the exchange): its results are visible past here
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   const int nvec = int(a.V / VT::N);
   const int n_sup = a.ws.hdr->n_sup;
   for (int idx = blockIdx.x; idx < n_sup; idx += gridDim.x) {
@@ -292,6 +297,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
   __shared__ int last;
   // the report's scratch: per-thread partials, one acceptance per thread, the totals
   __shared__ double scratch[(kNAcc + 1) * kTpThreads + kNAcc];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int nvec = int(a.V / VT::N);
   const int n_sup = a.ws.hdr->n_sup;
   const int total = n_sup + (a.dlogits ? a.ws.hdr->n_zero : 0);
@@ -406,36 +412,42 @@ cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s) {
                   : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, false>, a);
 }
 
+// steps 2 and 3: programmatic dependent launches (scheduled early, waiting for the work
+// before them on the stream before reading anything)
+template <typename K>
+cudaError_t launch_pdl(K kern, const TpArgs& a, cudaStream_t s) {
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tp_grid(a.R), 1, 1);
+  cfg.blockDim = dim3(kTpThreads, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a);
+  if (err != cudaSuccess) cudaGetLastError();
+  return err;
+}
+
 cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s) {
-  const unsigned g = tp_grid(a.R);
   using bf16 = __nv_bfloat16;
-  if (f32) {
-    if (a.target) tp_l1_kernel<float, true, false><<<g, kTpThreads, 0, s>>>(a);
-    else tp_l1_kernel<float, false, false><<<g, kTpThreads, 0, s>>>(a);
-  } else if (a.bias) {
-    if (a.target) tp_l1_kernel<bf16, true, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_l1_kernel<bf16, false, true><<<g, kTpThreads, 0, s>>>(a);
-  } else {
-    if (a.target) tp_l1_kernel<bf16, true, false><<<g, kTpThreads, 0, s>>>(a);
-    else tp_l1_kernel<bf16, false, false><<<g, kTpThreads, 0, s>>>(a);
-  }
-  return cudaGetLastError();
+  if (f32) return a.target ? launch_pdl(tp_l1_kernel<float, true, false>, a, s)
+                           : launch_pdl(tp_l1_kernel<float, false, false>, a, s);
+  if (a.bias) return a.target ? launch_pdl(tp_l1_kernel<bf16, true, true>, a, s)
+                              : launch_pdl(tp_l1_kernel<bf16, false, true>, a, s);
+  return a.target ? launch_pdl(tp_l1_kernel<bf16, true, false>, a, s)
+                  : launch_pdl(tp_l1_kernel<bf16, false, false>, a, s);
 }
 
 cudaError_t launch_tp_finish(bool f32, const TpArgs& a, cudaStream_t s) {
-  const unsigned g = tp_grid(a.R);
   using bf16 = __nv_bfloat16;
-  if (f32) {
-    if (a.target) tp_finish_kernel<float, true, false><<<g, kTpThreads, 0, s>>>(a);
-    else tp_finish_kernel<float, false, false><<<g, kTpThreads, 0, s>>>(a);
-  } else if (a.bias) {
-    if (a.target) tp_finish_kernel<bf16, true, true><<<g, kTpThreads, 0, s>>>(a);
-    else tp_finish_kernel<bf16, false, true><<<g, kTpThreads, 0, s>>>(a);
-  } else {
-    if (a.target) tp_finish_kernel<bf16, true, false><<<g, kTpThreads, 0, s>>>(a);
-    else tp_finish_kernel<bf16, false, false><<<g, kTpThreads, 0, s>>>(a);
-  }
-  return cudaGetLastError();
+  if (f32) return a.target ? launch_pdl(tp_finish_kernel<float, true, false>, a, s)
+                           : launch_pdl(tp_finish_kernel<float, false, false>, a, s);
+  if (a.bias) return a.target ? launch_pdl(tp_finish_kernel<bf16, true, true>, a, s)
+                              : launch_pdl(tp_finish_kernel<bf16, false, true>, a, s);
+  return a.target ? launch_pdl(tp_finish_kernel<bf16, true, false>, a, s)
+                  : launch_pdl(tp_finish_kernel<bf16, false, false>, a, s);
 }
 
 }  // namespace dspark
