@@ -644,13 +644,15 @@ def main(argv=None):
 
     # ---- roofline of the call: HBM bytes and tensor FLOPs a perfect implementation
     # needs; the bound is whichever takes longer at its measured peak
-    n_launch = launches_per_call(inp)
-    traffic = recorded_traffic() if n_launch == 2 else None
+    plain = inp.markov_w2 is None and inp.conf_w is None and inp.lm_head is None
+    traffic = recorded_traffic() if plain else None
     roofline = roofline_entry(algorithmic_bytes(inp, n_sup), algorithmic_flops(inp, n_sup), med, hbm_peak(),
                               tensor_peak(), timed_label(inp), traffic=traffic,
-                              dense=dense_bytes(inp) if n_launch == 2 else None)
-    roofline["traffic_source"] = ("recorded: the ncu DRAM bytes of profiles/sweep_recipe_traffic.md, taken on the "
-                                  "same kernel sources" if traffic is not None else None)
+                              dense=dense_bytes(inp) if plain else None)
+    roofline["traffic_source"] = ("recorded: the ncu DRAM bytes of the sweep kernel in "
+                                  "profiles/sweep_recipe_traffic.md, taken on the same kernel sources (the "
+                                  "zero-row fill beside it writes the unsupervised rows)" if traffic is not None
+                                  else None)
 
     # ---- end to end from pinned host buffers, the report summed over the ranks
     e2e = run_e2e(inp_cpu, inp, args.e2e_steps, torch_api, dist)
@@ -694,7 +696,7 @@ def main(argv=None):
             "e2e": {"value": round(e2e_value, 1), "unit": "rows/s", "h2d_bytes_per_step": e2e["h2d"],
                     "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"], 4),
                     "reduced_num_tokens": int(e2e["tokens"])},
-            "gpu_launches": n_launch * args.steps,
+            "gpu_launches": launches_per_call(inp) * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": round(wall, 3),
         }
