@@ -275,8 +275,12 @@ DSPARK_API dspark_status_t dspark_loss_fwd_noalloc(const dspark_problem_t* prob,
  * written for this shard's rows, and the embedding gradient dL/de is the sum of the
  * ranks' parts (the reduce across tensor parallelism) before dW1 is scattered and the
  * confidence head's own term dc*proj_e is added once.  dW1, dconf_w, dconf_b and dhidden
- * come out the same on every rank.  The teacher from hidden states is not taken on this
- * path (DSPARK_ERR_UNSUPPORTED).  Sum the forward outputs and the replicated gradients
+ * come out the same on every rank.  The teacher from hidden states is taken on this path
+ * with lm_head split like the logits: lm_head points at this shard's rows [V,
+ * target_hidden_size] and target_hidden (with target_norm_weight) is replicated;
+ * dspark_tp_partials computes the shard's FP32 teacher rows of every supervised row into
+ * the workspace, where the next two calls read them, so a micro-batch may hold at most 512
+ * rows (DSPARK_ERR_UNSUPPORTED above that).  Sum the forward outputs and the replicated gradients
  * over data-parallel ranks only: every tensor-parallel rank holds the same values.  The
  * calls of a micro-batch take the same problem, params, tp and workspace
  * (dspark_workspace_size(prob) bytes), in stream order.

@@ -234,7 +234,10 @@ dspark_status_t check_tp(const dspark_problem_t* p, const dspark_params_t* prm, 
   if (prm == nullptr || tp == nullptr) return DSPARK_ERR_INVALID_ARG;
   dspark_status_t st = check_problem(p, prm, sh, false);
   if (st != DSPARK_OK) return st;
-  if (sh->has_lm_head) return DSPARK_ERR_UNSUPPORTED;
+  // the teacher from hidden states: the shard's teacher rows of every supervised row are
+  // kept in the workspace's teacher chunk through the three calls, so all rows must fit
+  // one chunk
+  if (sh->has_lm_head && sh->R > kTeacherChunk) return DSPARK_ERR_UNSUPPORTED;
   if (tp->tp_size < 1 || tp->tp_size > 1024) return DSPARK_ERR_INVALID_ARG;
   if (tp->vocab_size <= 0 || tp->vocab_size > (int64_t(1) << 30) || tp->vocab_begin < 0 ||
       tp->vocab_begin > tp->vocab_size - p->V)
@@ -260,8 +263,13 @@ TpArgs tp_args(const dspark_problem_t* p, const dspark_params_t* prm, const dspa
   a.vocab_begin = tp->vocab_begin;
   a.tp_size = int32_t(tp->tp_size);
   a.ce_alpha = prm->ce_alpha;
-  a.l1_alpha = p->target_logits ? prm->l1_alpha : 0.f;
+  a.l1_alpha = (p->target_logits || lm_present(p)) ? prm->l1_alpha : 0.f;
   a.bias = markov_present(p) ? ws.bias : nullptr;
+  if (lm_present(p)) {  // the shard's teacher rows, computed by dspark_tp_partials
+    a.target = ws.tchunk;
+    a.ld_t = p->V;
+    a.t_compact = 1;
+  }
   a.ws = ws;
   return a;
 }
@@ -457,9 +465,16 @@ dspark_status_t dspark_tp_partials(const dspark_problem_t* prob, const dspark_pa
     if ((e = launch_heads_prep(ha, s)) != cudaSuccess) return cuda_status(e);
     if (sh.has_markov && (e = launch_markov_bias(ha, s)) != cudaSuccess) return cuda_status(e);
   }
+  if (sh.has_lm_head) {
+    // the supervised rows' hidden states (with the final norm if pre-norm), then the
+    // shard's teacher rows: hidden x lm_head rows of the shard, FP32, on the tensor cores
+    const TeacherArgs ta = teacher_args(prob, v);
+    if ((e = launch_gather_hidden(ta, s)) != cudaSuccess) return cuda_status(e);
+    if ((e = launch_teacher_chunk(ta, 0, s)) != cudaSuccess) return cuda_status(e);
+  }
   TpArgs a = tp_args(prob, params, tp, v);
   a.rec1 = rec1;
-  if (!sh.has_markov && !sh.has_conf_head) {  // nothing between the prologue and step 1
+  if (!sh.has_markov && !sh.has_conf_head && !sh.has_lm_head) {  // nothing between the prologue and step 1
     a.own_rows = 1;
     a.eval_mask = prob->eval_mask;
     a.block_keep = prob->block_keep;

@@ -155,8 +155,27 @@ __device__ __forceinline__ const uint8_t* row_ptr(const void* base, int64_t row,
   return static_cast<const uint8_t*>(base) + size_t(row) * size_t(ld) * sizeof(T);
 }
 
+// The teacher row of a supervised row: the logits' own rows (type T, by row), or with TF
+// the FP32 teacher rows computed from hidden states (compact by list position idx).
+template <typename T, bool TF>
+__device__ __forceinline__ const uint8_t* teacher_row(const TpArgs& a, int64_t row, int64_t idx) {
+  if constexpr (TF) return row_ptr<float>(a.target, idx, a.ld_t);
+  else return row_ptr<T>(a.target, row, a.ld_t);
+}
+// Vector v of a teacher row, as floats: the same columns as vector v of the draft row.
+template <typename T, bool TF>
+__device__ __forceinline__ void load_teacher(const uint8_t* tr, int v, float* y) {
+  if constexpr (TF) {
+    constexpr int N = Vec<T>::N;
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) Vec<float>::load(tr + (size_t(v) * N + 4 * q) * 4, y + 4 * q);
+  } else {
+    Vec<T>::load(tr + size_t(v) * 16, y);
+  }
+}
+
 // ---------------------------------------------------------------- step 1
-template <typename T, bool HAS_T, bool HAS_B>
+template <typename T, bool HAS_T, bool HAS_B, bool TF>
 __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[2 * kTpWarps];
@@ -188,7 +207,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
       row = a.ws.sup_list[idx];
     }
     const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
-    const uint8_t* tr = HAS_T ? row_ptr<T>(a.target, row, a.ld_t) : nullptr;
+    const uint8_t* tr = HAS_T ? teacher_row<T, TF>(a, row, idx) : nullptr;
     const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
     const float keep = (HAS_B && a.ws.sup_tok[idx] < 0) ? 0.f : 1.f;
     float mz = -INFINITY, sz = 0.f, mt = -INFINITY, st = 0.f;
@@ -199,7 +218,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
       if constexpr (HAS_B) add_bias<VT::N>(x, br, v, keep);
       if constexpr (HAS_T) {
         float y[VT::N];
-        VT::load(tr + size_t(v) * 16, y);
+        load_teacher<T, TF>(tr, v, y);
         lse_add<VT::N>(mt, st, y);
       }
       lse_add<VT::N>(mz, sz, x);
@@ -223,7 +242,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_partials_kernel(const TpArgs a)
 }
 
 // ---------------------------------------------------------------- step 2
-template <typename T, bool HAS_T, bool HAS_B>
+template <typename T, bool HAS_T, bool HAS_B, bool TF>
 __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float2 sh[kTpWarps];
@@ -264,7 +283,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
     if constexpr (HAS_T) {
       const float lz = lse2.x, lt = lse2.y;
       const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
-      const uint8_t* tr = row_ptr<T>(a.target, row, a.ld_t);
+      const uint8_t* tr = teacher_row<T, TF>(a, row, idx);
       const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
       const float keep = (HAS_B && a.ws.sup_tok[idx] < 0) ? 0.f : 1.f;
 #pragma unroll 4
@@ -272,7 +291,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
         float x[VT::N], y[VT::N];
         VT::load(zr + size_t(v) * 16, x);
         if constexpr (HAS_B) add_bias<VT::N>(x, br, v, keep);
-        VT::load(tr + size_t(v) * 16, y);
+        load_teacher<T, TF>(tr, v, y);
 #pragma unroll
         for (int e = 0; e < VT::N; ++e) {
           const float p = ex2(fmaf(x[e], kLog2e, -lz));
@@ -290,7 +309,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_l1_kernel(const TpArgs a) {
 }
 
 // ---------------------------------------------------------------- step 3
-template <typename T, bool HAS_T, bool HAS_B>
+template <typename T, bool HAS_T, bool HAS_B, bool TF>
 __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
   using VT = Vec<T>;
   __shared__ float rowS;
@@ -334,7 +353,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
       const float lz = st[kStLseD] * kLog2e, lt = st[kStLseT] * kLog2e;
       const int64_t col = a.tids[row] - a.vocab_begin;
       const uint8_t* zr = row_ptr<T>(a.draft, row, a.ld_d);
-      const uint8_t* tr = HAS_T ? row_ptr<T>(a.target, row, a.ld_t) : nullptr;
+      const uint8_t* tr = HAS_T ? teacher_row<T, TF>(a, row, idx) : nullptr;
       const float* br = HAS_B ? a.bias + size_t(idx) * size_t(a.V) : nullptr;
       const float keep = zero_row ? 0.f : 1.f;
       uint8_t* out = static_cast<uint8_t*>(a.dlogits) + size_t(row) * size_t(a.ld_g) * sizeof(T);
@@ -345,7 +364,7 @@ __global__ void __launch_bounds__(kTpThreads) tp_finish_kernel(const TpArgs a) {
         if constexpr (HAS_B) add_bias<VT::N>(x, br, v, keep);
         if constexpr (HAS_T) {
           float y[VT::N];
-          VT::load(tr + size_t(v) * 16, y);
+          load_teacher<T, TF>(tr, v, y);
 #pragma unroll
           for (int e = 0; e < VT::N; ++e) {
             const float p = ex2(fmaf(x[e], kLog2e, -lz));
@@ -401,15 +420,19 @@ cudaError_t launch_tp_partials(bool f32, const TpArgs& a, cudaStream_t s) {
   cfg.numAttrs = 1;
   using bf16 = __nv_bfloat16;
   if (f32) {
-    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, true, false>, a)
-                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, false, false>, a);
+    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, true, false, false>, a)
+                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<float, false, false, false>, a);
+  }
+  if (a.t_compact) {  // the teacher from hidden states (bf16 logits)
+    return a.bias ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, true, true>, a)
+                  : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, false, true>, a);
   }
   if (a.bias) {  // the Markov head needs bf16 logits
-    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, true>, a)
-                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, true>, a);
+    return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, true, false>, a)
+                    : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, true, false>, a);
   }
-  return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, false>, a)
-                  : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, false>, a);
+  return a.target ? cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, true, false, false>, a)
+                  : cudaLaunchKernelEx(&cfg, tp_partials_kernel<bf16, false, false, false>, a);
 }
 
 // steps 2 and 3: programmatic dependent launches (scheduled early, waiting for the work
@@ -432,22 +455,26 @@ cudaError_t launch_pdl(K kern, const TpArgs& a, cudaStream_t s) {
 
 cudaError_t launch_tp_l1(bool f32, const TpArgs& a, cudaStream_t s) {
   using bf16 = __nv_bfloat16;
-  if (f32) return a.target ? launch_pdl(tp_l1_kernel<float, true, false>, a, s)
-                           : launch_pdl(tp_l1_kernel<float, false, false>, a, s);
-  if (a.bias) return a.target ? launch_pdl(tp_l1_kernel<bf16, true, true>, a, s)
-                              : launch_pdl(tp_l1_kernel<bf16, false, true>, a, s);
-  return a.target ? launch_pdl(tp_l1_kernel<bf16, true, false>, a, s)
-                  : launch_pdl(tp_l1_kernel<bf16, false, false>, a, s);
+  if (f32) return a.target ? launch_pdl(tp_l1_kernel<float, true, false, false>, a, s)
+                           : launch_pdl(tp_l1_kernel<float, false, false, false>, a, s);
+  if (a.t_compact) return a.bias ? launch_pdl(tp_l1_kernel<bf16, true, true, true>, a, s)
+                                 : launch_pdl(tp_l1_kernel<bf16, true, false, true>, a, s);
+  if (a.bias) return a.target ? launch_pdl(tp_l1_kernel<bf16, true, true, false>, a, s)
+                              : launch_pdl(tp_l1_kernel<bf16, false, true, false>, a, s);
+  return a.target ? launch_pdl(tp_l1_kernel<bf16, true, false, false>, a, s)
+                  : launch_pdl(tp_l1_kernel<bf16, false, false, false>, a, s);
 }
 
 cudaError_t launch_tp_finish(bool f32, const TpArgs& a, cudaStream_t s) {
   using bf16 = __nv_bfloat16;
-  if (f32) return a.target ? launch_pdl(tp_finish_kernel<float, true, false>, a, s)
-                           : launch_pdl(tp_finish_kernel<float, false, false>, a, s);
-  if (a.bias) return a.target ? launch_pdl(tp_finish_kernel<bf16, true, true>, a, s)
-                              : launch_pdl(tp_finish_kernel<bf16, false, true>, a, s);
-  return a.target ? launch_pdl(tp_finish_kernel<bf16, true, false>, a, s)
-                  : launch_pdl(tp_finish_kernel<bf16, false, false>, a, s);
+  if (f32) return a.target ? launch_pdl(tp_finish_kernel<float, true, false, false>, a, s)
+                           : launch_pdl(tp_finish_kernel<float, false, false, false>, a, s);
+  if (a.t_compact) return a.bias ? launch_pdl(tp_finish_kernel<bf16, true, true, true>, a, s)
+                                 : launch_pdl(tp_finish_kernel<bf16, true, false, true>, a, s);
+  if (a.bias) return a.target ? launch_pdl(tp_finish_kernel<bf16, true, true, false>, a, s)
+                              : launch_pdl(tp_finish_kernel<bf16, false, true, false>, a, s);
+  return a.target ? launch_pdl(tp_finish_kernel<bf16, true, false, false>, a, s)
+                  : launch_pdl(tp_finish_kernel<bf16, false, false, false>, a, s);
 }
 
 }  // namespace dspark

@@ -23,6 +23,8 @@ struct TpArgs {
   float* rec2;               // [R][4] this shard's (L1, S) partials
   const float* rec2_all;     // [tp_size][R][4]
   const float* bias;         // Markov bias rows of the shard (compact by supervised position), or null
+  int32_t t_compact;         // teacher rows: FP32, compact by supervised position, ld_t columns
+                             // (the teacher computed from hidden states on the shard)
   // Step 1 straight behind the mask prologue (no heads): it takes every row and decides
   // by the prologue's own rule whether the row is supervised, so it need not wait for
   // the prologue's lists

@@ -240,8 +240,9 @@ class TPRank:
     ``inp`` holds rows that contain this rank's shard at columns [col0, col0 + width):
     the full rows (single-device emulation of a group) or just the shard (one rank per
     GPU, col0 = 0).  The shard is addressed in place, with the rows' stride; so are the
-    shard's rows of ``inp.markov_w2`` (rows col0 .. col0 + width).  dlogits of the shard
-    go to the same columns of ``dlogits`` (rows shaped like ``inp``'s), and dW2 of the
+    shard's rows of ``inp.markov_w2`` and ``inp.lm_head`` (rows col0 .. col0 + width).
+    dlogits of the shard go to the same columns of ``dlogits`` (rows shaped like
+    ``inp``'s), and dW2 of the
     shard to the same rows of ``dW2`` (shaped like ``inp.markov_w2``), or to buffers this
     rank allocates.  Every rank writes its own copy of the forward outputs and of the
     replicated gradients (dW1, dconf_w, dconf_b, dhidden).
@@ -265,6 +266,8 @@ class TPRank:
         rank_ = inp.markov_w2.shape[1] if markov else 0
         if markov:
             p.markov_w2 = ctypes.c_void_p(inp.markov_w2.data_ptr() + col0 * rank_ * 2)
+        if inp.lm_head is not None:  # the teacher from hidden states: this shard's lm_head rows
+            p.lm_head = ctypes.c_void_p(inp.lm_head.data_ptr() + col0 * inp.lm_head.shape[1] * 2)
         self.prob = p
         self.prm = params_struct(inp, invalid_row_mode)
         self.tp = abi.dspark_tp_t(tp_size, vocab_begin, vocab_size)

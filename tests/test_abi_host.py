@@ -306,9 +306,12 @@ def test_vocab_parallel_validation(abi):
     assert _tp_calls(abi, _problem(abi, V=1020), prm, tp) == every(abi.DSPARK_ERR_ALIGNMENT)
     assert _tp_calls(abi, p, prm, tp, ws_bytes=16) == every(abi.DSPARK_ERR_WORKSPACE)
     assert _tp_calls(abi, _problem(abi, target=False), prm, tp) == every(abi.DSPARK_ERR_MISSING_TARGET)
-    # the teacher from hidden states is not taken on the vocabulary-parallel path
-    assert _tp_calls(abi, _with_lm_head(abi, _problem(abi, target=False)), prm, tp) == \
-        every(abi.DSPARK_ERR_UNSUPPORTED)
+    # the teacher from hidden states on the vocabulary-parallel path keeps every supervised
+    # row's teacher shard in the workspace's teacher chunk: more than 512 rows are refused
+    # (up to 512 are served; that is tested on the GPU)
+    big = _with_lm_head(abi, _problem(abi, target=False))
+    big.N, big.K = 65, 8
+    assert _tp_calls(abi, big, prm, tp) == every(abi.DSPARK_ERR_UNSUPPORTED)
     # with the Markov head the shard's dE part and the ranks' parts are records too
     pm = _with_markov(abi, _problem(abi))
     g = abi.dspark_grads_t()

@@ -75,6 +75,30 @@ def test_tp_dropped_blocks_and_many_rows():
     _check_group(inp, ranks, oracle_run(inp))
 
 
+@pytest.mark.parametrize("T,prenorm,heads", [(2, False, False), (3, True, False), (2, False, True)])
+def test_tp_teacher_from_hidden_states(T, prenorm, heads):
+    """The teacher from the target's hidden states on the vocabulary-parallel path: each
+    rank computes its shard's teacher rows from its rows of lm_head (and, pre-norm, the
+    final RMS norm of the replicated hidden states); with the heads as well."""
+    kw = dict(markov=True, conf="head", markov_std=0.2, valid_p=0.8) if heads else {}
+    inp = make_inputs("recipe", device="cuda", B=2, N=5, K=7, V=4096, lm_head=True, target_hidden_size=256,
+                      target_prenorm=prenorm, mask_holes=True, seed=50 + T + 2 * int(prenorm), **kw)
+    ranks = _group(inp, T)
+    _check_group(inp, ranks, oracle_run(inp))
+
+
+def test_tp_teacher_from_hidden_states_refuses_more_than_one_chunk():
+    """All supervised rows' teacher rows stay in the workspace's teacher chunk through the
+    three calls: more than 512 rows are refused before anything is enqueued."""
+    inp = make_inputs("recipe", device="cuda", B=2, N=37, K=7, V=1024, lm_head=True, target_hidden_size=64,
+                      seed=55)
+    from speculative_decoding_draft_vocab_b200 import abi, torch_api
+    rank = torch_api.TPRank(inp, 2, 0, inp.V, col0=0, width=512)
+    with pytest.raises(abi.DSparkError) as e:
+        rank.partials()
+    assert e.value.status == abi.DSPARK_ERR_UNSUPPORTED
+
+
 def test_tp_given_confidence_gamma_none_grad_scale():
     inp = make_inputs("recipe", device="cuda", B=2, N=4, K=7, V=8192, conf="given", gamma=None,
                       grad_scale=0.37, seed=41)
