@@ -152,6 +152,9 @@ def tp_algorithmic_bytes(inp, n_sup: int, width: int) -> int:
     gradient written (the replicated heads' work is every rank's)."""
     es = 2 if inp.dtype == "bf16" else 4
     b = n_sup * width * es * (2 if inp.target_logits is not None else 1) + inp.R * width * es
+    if inp.lm_head is not None:  # the teacher from hidden states: lm_head's shard rows, the hidden rows
+        ht = inp.lm_head.shape[1]
+        b += width * ht * 2 + n_sup * ht * 2
     if inp.markov_w2 is not None:
         r = inp.markov_w2.shape[1]
         b += width * r * (2 + 4) + n_sup * r * (2 + 4)
@@ -162,8 +165,11 @@ def tp_algorithmic_bytes(inp, n_sup: int, width: int) -> int:
 
 def tp_algorithmic_flops(inp, n_sup: int, width: int) -> int:
     """One rank's tensor-core work: the Markov bias, dE and dW2 contractions against its
-    columns (2 * rows * width * rank each)."""
-    return 3 * 2 * n_sup * width * inp.markov_w2.shape[1] if inp.markov_w2 is not None else 0
+    columns (2 * rows * width * rank each), and the teacher's against its lm_head rows."""
+    f = 3 * 2 * n_sup * width * inp.markov_w2.shape[1] if inp.markov_w2 is not None else 0
+    if inp.lm_head is not None:
+        f += 2 * n_sup * width * inp.lm_head.shape[1]
+    return f
 
 
 def tp_launches_per_step(inp) -> int:
@@ -176,6 +182,8 @@ def tp_launches_per_step(inp) -> int:
         n += 1 + 3 + 1  # bias GEMM; dE GEMM, dW2 GEMM, split sum; the merge of the ranks' parts
     if conf:
         n += 3  # dproj partials, dproj final, dhidden
+    if inp.lm_head is not None:
+        n += 2  # hidden-state gather, the shard's teacher GEMM
     return n
 
 
