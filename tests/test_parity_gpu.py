@@ -142,6 +142,34 @@ def test_many_rows_dropped_blocks_and_bad_ids(B, N, K, V):
         assert bool((call.out.dlogits[b, n, k] == 0).all())
 
 
+@pytest.mark.parametrize("heads", [False, True])
+def test_fused_call_replays_in_a_cuda_graph(heads):
+    """The fused call captured into a CUDA graph (after one eager call, which sets the
+    launch attributes up) and replayed: the same outputs bit for bit as the eager call,
+    through the programmatic dependent launches of the sweep and the zero-row fill."""
+    from speculative_decoding_draft_vocab_b200 import torch_api
+    kw = dict(markov=True, conf="head", markov_std=0.2) if heads else {}
+    inp = make_inputs("recipe", device="cuda", B=2, N=4, K=7, V=8192, mask_holes=True, seed=61, **kw)
+    call = torch_api.Call(inp, grads=True, rows=True)
+    call.launch()
+    torch.cuda.synchronize()
+    assert call.check_status() == 0
+    eager = {k: v.clone() for k, v in (("loss", call.out.loss_num), ("report", call.out.report),
+                                       ("dlogits", call.out.dlogits), ("l1", call.out.l1_rows))}
+    for t in (call.out.loss_num, call.out.report, call.out.dlogits, call.out.l1_rows):
+        t.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call.launch()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert call.check_status() == 0
+    assert torch.equal(call.out.loss_num, eager["loss"])
+    assert torch.equal(call.out.report, eager["report"])
+    assert torch.equal(call.out.l1_rows, eager["l1"])
+    assert torch.equal(call.out.dlogits, eager["dlogits"])
+
+
 def test_all_masked_batch():
     inp = make_inputs("recipe", device="cuda", B=2, N=3, K=7, V=4096, prefix=(0, 0), seed=9)
     call, ref, _ = _run_and_compare(inp)
