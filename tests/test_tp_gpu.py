@@ -99,6 +99,34 @@ def test_tp_teacher_from_hidden_states_refuses_more_than_one_chunk():
     assert e.value.status == abi.DSPARK_ERR_UNSUPPORTED
 
 
+def test_tp_rank_replays_in_a_cuda_graph():
+    """One rank's three calls (programmatic dependent launches of steps 1-3) captured into
+    a CUDA graph with the group's records fixed, and replayed: rank 0's outputs bit for bit
+    as eagerly computed."""
+    inp = make_inputs("recipe", device="cuda", B=2, N=5, K=7, V=4096, mask_holes=True, seed=63)
+    ranks = _group(inp, 2)
+    r0 = ranks[0]
+    rec1_all = torch.stack([r.rec1 for r in ranks]).clone()
+    rec2_all = torch.stack([r.rec2 for r in ranks]).clone()
+    c0, c1 = r0.col0, r0.col0 + r0.width
+    eager = (r0.loss_num.clone(), r0.report.clone(), r0.l1_rows.clone(), r0.dlogits[..., c0:c1].clone())
+    for t in (r0.loss_num, r0.report, r0.l1_rows):
+        t.zero_()
+    r0.dlogits[..., c0:c1].zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        r0.partials()
+        r0.l1(rec1_all)
+        r0.finish(rec2_all)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert r0.check_status() == 0
+    assert torch.equal(r0.loss_num, eager[0])
+    assert torch.equal(r0.report, eager[1])
+    assert torch.equal(r0.l1_rows, eager[2])
+    assert torch.equal(r0.dlogits[..., c0:c1], eager[3])
+
+
 def test_tp_given_confidence_gamma_none_grad_scale():
     inp = make_inputs("recipe", device="cuda", B=2, N=4, K=7, V=8192, conf="given", gamma=None,
                       grad_scale=0.37, seed=41)
